@@ -1,0 +1,234 @@
+/*
+ * stattn.h -- C ABI of libstattn.so, the single-GPU (sm_100a) hot path of the
+ * attention block of a spatial-temporal diffusion transformer.
+ *
+ * Sources of each operation (page title, then section):
+ *   [SF]  "ScaleFusion: Scalable Inference of Spatial-Temporal Diffusion
+ *         Transformers for High-Resolution Long Video Generation" (paper
+ *         review), sections "三、技术架构" (layer table, distributed execution
+ *         flow, core formulas of spatial-temporal independence) and
+ *         "四、核心创新" (intra-layer schedule with N_T/N_S slices, inter-layer
+ *         schedule with L_T/L_S partitions, pseudo-code).
+ *   [SW]  "Technical Summary: SwiftFusion", Methodology 2 "Torus Attention"
+ *         (all-to-all broken into chunks, partial attention per chunk).
+ *   [xD]  "xDiT: an Inference Engine for Diffusion Transformers (DiTs) with
+ *         Massive Parallelism", section 3 (image-DiT full attention over
+ *         hundreds of thousands to millions of tokens).
+ *   [CC]  "CoCoDiff: Optimizing Collective Communications for Distributed
+ *         Diffusion Transformer Inference Under Ulysses Sequence
+ *         Parallelism", sections on Ulysses all-to-all, "V-First" (RMSNorm on
+ *         Q and K only) and "V-Major" (per-token L1 change of V, threshold,
+ *         cached data for inactive tokens, full refresh every 10 steps).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates or frees device memory and never synchronises
+ *     a stream (except st_check_device_status, which says so).
+ *   - Every call is stream-ordered on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and returns before the work finishes.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns its status and launches nothing.  A launch error
+ *     reported by the CUDA runtime returns ST_ERR_CUDA.  Waits inside the
+ *     tensor-core attention kernel are bounded; a wait that runs out sets a
+ *     device error word that st_check_device_status reports as
+ *     ST_ERR_TIMEOUT.  No call aborts the process or traps the GPU.
+ *   - bf16 is IEEE-style bfloat16 (1-8-7); reductions accumulate in fp32 and
+ *     round to bf16 once, to nearest even.
+ *   - Element strides are in ELEMENTS, not bytes.
+ */
+#ifndef STATTN_H
+#define STATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *st_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+  ST_OK = 0,
+  ST_ERR_NULL = -1,         /* a required pointer is NULL                      */
+  ST_ERR_SHAPE = -2,        /* a size is <= 0, out of range or inconsistent     */
+  ST_ERR_DIVISIBILITY = -3, /* P, N_T, N_S or the head count does not divide    */
+  ST_ERR_DTYPE = -4,        /* dtype / element size not supported by the call   */
+  ST_ERR_ALIGN = -5,        /* pointer or row pitch not aligned as required     */
+  ST_ERR_UNSUPPORTED = -6,  /* valid request this build has no kernel for       */
+  ST_ERR_CUDA = -7,         /* the CUDA runtime reported an error               */
+  ST_ERR_TIMEOUT = -8       /* a bounded device-side wait ran out               */
+} st_status;
+
+typedef enum { ST_F32 = 0, ST_BF16 = 1 } st_dtype;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *st_status_string(st_status s);
+
+/* ABI version of this header: 1. */
+int st_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Attention descriptor.
+ *
+ * Q, K, V and O are logical [B, T, S, H, D] tensors: B batches of T frames of
+ * S tokens, each token a row of C = H*D channels with head h at channels
+ * [h*D, (h+1)*D).  Element (b, t, s, h, d) lives at element offset
+ *
+ *   b*stride_b + (t / tb)*stride_tb + (t % tb)*stride_t
+ *              + (s / sb)*stride_sb + (s % sb)*stride_s + h*D + d
+ *
+ * with tb = t_block (T when t_block == 0) and sb = s_block (S when 0).  The
+ * two-level form addresses the sliced layouts [B,N_T,N_S,T/N_T,S/N_S/P,C] of
+ * the ScaleFusion intra-layer schedule [SF "四、核心创新"] directly.  Zero
+ * strides mean the dense layout [B, T, S, H*D].  Q, K, V and O share the
+ * descriptor's strides.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int size;               /* sizeof(st_attn_desc), for ABI versioning          */
+  int B, T, S, H, D;      /* sizes; D in {32, 64, 72, 80, 96, 128} for bf16      */
+  st_dtype dtype;         /* dtype of Q, K, V (and of O unless o_fp32)          */
+  float scale;            /* softmax scale; <= 0 means 1/sqrt(D)                */
+  long long stride_b, stride_t, stride_s;   /* elements; 0 -> dense              */
+  int t_block;            /* frames per frame block; 0 -> one level             */
+  long long stride_tb;    /* elements between frame blocks                      */
+  int s_block;            /* tokens per token block; 0 -> one level             */
+  long long stride_sb;    /* elements between token blocks                      */
+  int n_slices, slice;    /* compute slice `slice` of `n_slices` only (frames
+                             for the spatial call, tokens for the temporal
+                             call); slice < 0 or n_slices <= 1 -> everything   */
+  int kv_begin, kv_end;   /* spatial call: keys [kv_begin, kv_end) of each
+                             frame; 0,0 -> all S keys                           */
+  int o_fp32;             /* nonzero: write O as fp32 (a normalised partial for
+                             attn_chunk_merge) with the same element strides     */
+} st_attn_desc;
+
+/* Spatial attention [SF "三、技术架构" layer table; xD section 3]: for every
+ * (b, t, h) in the selected frames,
+ *     O[b,t,:,h,:] = softmax(Q[b,t,:,h,:] K[b,t,kv,h,:]^T * scale) V[b,t,kv,h,:]
+ * over the keys kv of frame t.  T = 1, S = N is image-DiT full attention.  A
+ * key range [kv_begin, kv_end) yields the partial result of one KV chunk of
+ * ring / Torus attention [SW Methodology 2]; merge chunks with
+ * attn_chunk_merge.
+ *   lse: optional fp32 [B, T, H, S] dense, natural-log log-sum-exp of the
+ *        scaled scores of each query row (-inf for an empty key range).
+ *   bf16 runs on the tcgen05 tensor-core kernel (fp32 accumulation); fp32 runs
+ *   on an fp32 FMA kernel.  Returns ST_ERR_ALIGN if a pointer or stride is not
+ *   16-byte aligned, ST_ERR_UNSUPPORTED for a bf16 head dim outside the set
+ *   above, ST_ERR_SHAPE for a bad key range. */
+st_status st_attn_spatial(const st_attn_desc *desc, const void *q, const void *k,
+                          const void *v, void *o, float *lse, st_stream_t stream);
+
+/* Temporal attention [SF "三、技术架构"]: for every (b, s, h) in the selected
+ * tokens, attention over the T frames of token s.  T <= 64.
+ *   lse: optional fp32 [B, S, H, T] dense.
+ *   kv_begin/kv_end must be 0.  bf16 uses tensor-core mma tiles with fp32
+ *   accumulation; fp32 uses fp32 FMA. */
+st_status st_attn_temporal(const st_attn_desc *desc, const void *q, const void *k,
+                           const void *v, void *o, float *lse, st_stream_t stream);
+
+/* Log-sum-exp merge of KV-chunk partials [SW Methodology 2]:
+ *     M = max_c lse_c,  lse = M + ln sum_c exp(lse_c - M),
+ *     o = sum_c exp(lse_c - lse) * o_c
+ *   o_parts, lse_parts: HOST arrays of n_chunks (1..16) DEVICE pointers;
+ *     o_parts[c] is fp32 dense [n_units, S, H, D] (n_units = B*T frames),
+ *     lse_parts[c] is fp32 dense [n_units, H, S].
+ *   o_out: dense [n_units, S, H, D] in out_dtype.  lse_out: optional
+ *   [n_units, H, S].  Rows whose every chunk has lse = -inf get o = 0. */
+st_status attn_chunk_merge(int n_chunks, const float *const *o_parts,
+                           const float *const *lse_parts, long long n_units, int S,
+                           int H, int D, void *o_out, st_dtype out_dtype,
+                           float *lse_out, st_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * All-to-all relayout on a virtual partition [SF "三、技术架构" distributed
+ * execution flow and "四、核心创新" pseudo-code; CC Ulysses section].
+ *
+ * The P shards of the distributed tensor are stacked as the outermost axis of
+ * one buffer; the all-to-all is a permutation of rows inside HBM.
+ *
+ * ST_S2T / ST_T2S (T_or_N = T, S_or_H = S, C_or_D = C):
+ *   x, shard p: [B, N_T, N_S, T/N_T, S/(N_S*P), C];  row (p,b,i,j,t1,s1) holds
+ *      frame t = i*T/N_T + t1, token s = j*S/N_S + p*S/(N_S*P) + s1.
+ *   y, shard q: [B, N_T, N_S, T/(N_T*P), S/N_S, C];  row (q,b,i,j,t2,s2) holds
+ *      frame t = i*T/N_T + q*T/(N_T*P) + t2, token s = j*S/N_S + s2.
+ *   S2T reads x and writes y; T2S reads y and writes x.  N_T = N_S = 1 gives
+ *   the plain [B,T,S/P,C] <-> [B,T/P,S,C] exchange.  Only destination rows
+ *   of blocks i0 <= i < i1, j0 <= j < j1 are written (one partition of the
+ *   inter-layer schedule); (0, N_T, 0, N_S) writes everything.
+ *   Requires N_T*P | T and N_S*P | S.
+ * ST_SEQ2HEAD / ST_HEAD2SEQ (T_or_N = N tokens, S_or_H = H, C_or_D = D):
+ *   in,  shard p: [B, N/P, H, D]; out, shard q: [B, H/P, N, D] (heads outer so
+ *   each head's sequence is contiguous).  HEAD2SEQ is the inverse.  n_t, n_s
+ *   must be 1 and the block range (0, 1, 0, 1).  Requires P | N and P | H.
+ * rms_gamma (optional, fp32 device [rms_head_dim]): apply per-head RMSNorm
+ *   y = x / sqrt(mean(x^2) + rms_eps) * gamma to every rms_head_dim-wide
+ *   head segment while moving it [CC "V-First"]; elem_bytes must then be 2
+ *   (bf16) or 4 (fp32) and rms_head_dim must divide C (ST) or equal D.
+ * elem_bytes: 1, 2, 4 or 8; rows are moved with the widest vector (up to 16
+ *   bytes) that the row pitch and both pointers allow.
+ * in and out must not overlap.
+ * ---------------------------------------------------------------------- */
+typedef enum { ST_S2T = 0, ST_T2S = 1, ST_SEQ2HEAD = 2, ST_HEAD2SEQ = 3 } st_relayout_mode;
+
+st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *out,
+                           int elem_bytes, int P, int B, int T_or_N, int S_or_H,
+                           int C_or_D, int n_t, int n_s, int i0, int i1, int j0,
+                           int j1, const float *rms_gamma, int rms_head_dim,
+                           float rms_eps, st_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * V-Major selective communication [CC "V-Major"].
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of device workspace vmajor_mask_compact needs for n_tokens. */
+size_t vmajor_workspace_bytes(long long n_tokens);
+
+/* Per-token change mask and compaction:
+ *     L1_n   = sum_c |v_cur[n,c] - v_prev[n,c]|   (fp32 accumulation)
+ *     mask_n = (L1_n > tau) || force_all
+ *     idx    = ascending list of active n,  *count = |idx|
+ *   v_cur, v_prev: dense [n_tokens, C] of dtype.  mask: u8 [n_tokens];
+ *   idx: int32 [n_tokens] (entries past *count are left untouched);
+ *   count: ONE int32 in device memory, so later kernels read it without a
+ *   host round trip.  l1_out: optional fp32 [n_tokens] copy of L1_n.
+ *   workspace: caller-owned device memory of at least
+ *   vmajor_workspace_bytes(n_tokens) bytes (no state is kept in it between
+ *   calls).  force_all = 1 is the periodic full refresh.
+ *   Requires C*elem size to be a multiple of 16 bytes and 16-byte aligned
+ *   v_cur/v_prev. */
+st_status vmajor_mask_compact(const void *v_cur, const void *v_prev,
+                              long long n_tokens, int C, st_dtype dtype, float tau,
+                              int force_all, unsigned char *mask, int *idx,
+                              int *count, float *l1_out, void *workspace,
+                              size_t workspace_bytes, st_stream_t stream);
+
+/* Cache update for the active tokens: for i < *count (read on the device),
+ *     dst_cache[t][idx[i], :] = src[t][idx[i], :]        for t < n_tensors
+ * and, when packed is not NULL, packed[t][i, :] = src[t][idx[i], :] (the
+ * message of active rows a rank would send).  Rows are C elements of
+ * elem_bytes each.  src, dst_cache, packed: HOST arrays of n_tensors (1..8)
+ * DEVICE pointers to dense [n_tokens, C] ([n_tokens, C] capacity for packed).
+ * Inactive tokens keep their cached rows. */
+st_status vmajor_scatter_rows(const int *idx, const int *count, long long n_tokens,
+                              int C, int elem_bytes, const void *const *src,
+                              void *const *dst_cache, int n_tensors,
+                              void *const *packed, st_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word that
+ * bounded waits set.  Returns ST_ERR_TIMEOUT if a wait ran out since the last
+ * call, ST_ERR_CUDA if the stream reports an error, else ST_OK. */
+st_status st_check_device_status(st_stream_t stream);
+
+/* Failure-detection self test: launches a one-thread kernel that waits, with
+ * a 20 ms limit, on an mbarrier nothing ever arrives on, through the same
+ * bounded-wait path the tensor-core attention kernel uses.  The wait runs
+ * out, the kernel records it and returns; a following
+ * st_check_device_status(stream) must report ST_ERR_TIMEOUT (and clears the
+ * word).  Nothing faults, traps or hangs. */
+st_status st_selftest_wait_timeout(st_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STATTN_H */

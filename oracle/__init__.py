@@ -32,14 +32,15 @@ Each pin of these functions lives in ``tests/test_oracle_*.py``.
 """
 from .attention import attention, spatial, temporal, merge_chunks, frames_view
 from .relayout import (st_x_rows, st_y_rows, st_relayout, seq_head_relayout,
-                       st_logical_from_x, st_logical_from_y)
+                       st_logical_from_x, st_logical_from_y, st_row_pairs, seq_head_row_pairs)
 from .rmsnorm import rmsnorm_heads
 from .vmajor import l1_change, change_mask, compact, scatter_rows, pack_rows, tau_for_fraction
 
 __all__ = [
     "attention", "spatial", "temporal", "merge_chunks", "frames_view",
     "st_x_rows", "st_y_rows", "st_relayout", "seq_head_relayout",
-    "st_logical_from_x", "st_logical_from_y", "rmsnorm_heads",
+    "st_logical_from_x", "st_logical_from_y", "st_row_pairs", "seq_head_row_pairs",
+    "rmsnorm_heads",
     "l1_change", "change_mask", "compact", "scatter_rows", "pack_rows",
     "tau_for_fraction",
 ]

@@ -112,6 +112,32 @@ def st_relayout(mode, buf, P, B, T, S, C, n_t=1, n_s=1, blocks=None, out=None, r
     return _move_rows(src, dst, src_log, dst_log, sel, C, rms)
 
 
+def st_row_pairs(mode, P, B, T, S, n_t=1, n_s=1, blocks=None):
+    """(dst_rows, src_rows): destination row r of the relayout holds source row src.
+
+    The same definition as st_relayout, returned as index arrays so that a
+    full-size result can be checked with one gather.
+    """
+    _check_st(P, T, S, n_t, n_s)
+    x_log, xi, xj = st_x_rows(P, B, T, S, n_t, n_s)
+    y_log, yi, yj = st_y_rows(P, B, T, S, n_t, n_s)
+    src_log, dst_log, di, dj = (x_log, y_log, yi, yj) if mode == "S2T" else (y_log, x_log, xi, xj)
+    i0, i1, j0, j1 = blocks if blocks is not None else (0, n_t, 0, n_s)
+    sel = np.flatnonzero((di >= i0) & (di < i1) & (dj >= j0) & (dj < j1))
+    pos = np.empty(src_log.size, dtype=np.int64)
+    pos[src_log] = np.arange(src_log.size)
+    return sel, pos[dst_log[sel]]
+
+
+def seq_head_row_pairs(mode, P, B, N, H):
+    """(dst_rows, src_rows) of the sequence<->head exchange (rows of D)."""
+    seq_log, head_log = _seq_rows(P, B, N, H), _head_rows(P, B, N, H)
+    src_log, dst_log = (seq_log, head_log) if mode == "SEQ2HEAD" else (head_log, seq_log)
+    pos = np.empty(src_log.size, dtype=np.int64)
+    pos[src_log] = np.arange(src_log.size)
+    return np.arange(dst_log.size), pos[dst_log]
+
+
 def st_logical_from_x(buf, P, B, T, S, C, n_t=1, n_s=1):
     """[B, T, S, C] logical tensor held by an x buffer."""
     x_log, _, _ = st_x_rows(P, B, T, S, n_t, n_s)

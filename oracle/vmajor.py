@@ -63,17 +63,28 @@ def pack_rows(idx, count, src):
     return np.stack([s[idx[i]] for i in range(count)]) if count else s[:0]
 
 
-def tau_for_fraction(l1, f):
-    """Threshold that leaves a fraction ``f`` of tokens active.
+def tau_for_fraction(l1, f, window=0.01):
+    """Threshold that leaves about a fraction ``f`` of tokens active.
 
-    tau is the midpoint of the two sorted L1 values that straddle the
-    (1 - f) quantile, so round(N * f) tokens are strictly above it.  Returns
-    (tau, margin) with margin = min_n |L1_n - tau| / tau.
+    Sort the L1 values; among the consecutive pairs whose rank lies within
+    ``window * N`` of N * (1 - f), take the pair with the widest relative gap
+    and put tau at its midpoint.  The widest gap keeps every L1 far from tau
+    compared with the rounding of an fp32 sum, so the mask does not depend on
+    the precision or order of the summation.  Returns (tau, margin,
+    active_fraction) with margin = min_n |L1_n - tau| / tau.
     """
     v = np.sort(np.asarray(l1, dtype=np.float64))
     n = v.size
-    k = n - int(round(n * f))                   # tokens at or below tau
-    k = min(max(k, 1), n - 1)
-    tau = 0.5 * (v[k - 1] + v[k])
+    k0 = n - int(round(n * f))                  # tokens at or below tau
+    w = int(round(window * n))
+    k0 = min(max(k0, 1), n - 1)
+    lo, hi = max(1, k0 - w), min(n - 1, k0 + w)
+    best, best_k = -1.0, k0
+    for k in range(lo, hi + 1):
+        mid = 0.5 * (v[k - 1] + v[k])
+        gap = (v[k] - v[k - 1]) / mid if mid > 0 else 0.0
+        if gap > best:
+            best, best_k = gap, k
+    tau = 0.5 * (v[best_k - 1] + v[best_k])
     margin = float(np.min(np.abs(v - tau)) / tau) if tau > 0 else 0.0
-    return float(tau), margin
+    return float(tau), margin, float((v > tau).sum()) / n

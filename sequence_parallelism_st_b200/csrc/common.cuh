@@ -1,0 +1,41 @@
+// Shared host/device helpers of libstattn (no kernels).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "stattn.h"
+
+#define ST_API extern "C" __attribute__((visibility("default")))
+
+namespace st {
+
+inline bool is_aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Status of the launch just issued on this thread.
+inline st_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ST_OK : ST_ERR_CUDA;
+}
+
+// SM count of the current device (cached per device ordinal).
+int num_sms();
+
+// Reads and clears the device error word of the tensor-core attention kernel
+// (defined next to that kernel).  Returns the word's previous value.
+unsigned int read_and_clear_attn_error(cudaStream_t stream, cudaError_t *err);
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// Round to nearest even; NaN stays NaN.
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+}  // namespace st

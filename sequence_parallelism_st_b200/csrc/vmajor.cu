@@ -1,0 +1,241 @@
+// V-Major selective communication (CoCoDiff article, "V-Major" section):
+// per-token L1 change of V against the previous step, threshold mask, the
+// ascending list of active tokens, and the cache update for active tokens.
+//
+// Design.  vmajor_mask_compact is two launches and no atomics, so its output
+// is deterministic:
+//   1. l1_mask: one warp per token streams both [C] rows with 16-byte loads
+//      (all of a lane's loads issued before any arithmetic), accumulates
+//      |cur - prev| in fp32, reduces over the warp with a fixed butterfly
+//      order, writes the mask byte, and each CTA writes the number of active
+//      tokens of its tile of TILE tokens to the workspace.
+//   2. compact: one CTA per 2048 tokens sums the counts of the L1 tiles
+//      before it (an exclusive prefix read straight from the workspace),
+//      ranks its active tokens with warp ballots and writes their indices in
+//      ascending order; the last CTA also writes the total count.
+// The read of 2 * N * C elements dominates; everything else is O(N).
+#include "common.cuh"
+
+namespace {
+
+constexpr int TILE = 32;          // tokens per CTA of the L1 pass (8 warps x 4 tokens)
+constexpr int THREADS = 256;
+constexpr int VMAX = 12;          // 16-byte vectors per lane per tensor in flight
+constexpr int CTILE = 2048;       // tokens per CTA of the compaction pass
+constexpr int ROUNDS = CTILE / THREADS;  // 32-token ballots per warp
+
+template <typename T>
+__global__ void __launch_bounds__(THREADS) l1_mask(const char *__restrict__ cur,
+                                                   const char *__restrict__ prev, long long n,
+                                                   int row_vecs, float tau, int force_all,
+                                                   unsigned char *__restrict__ mask,
+                                                   float *__restrict__ l1_out,
+                                                   int *__restrict__ tile_count) {
+  constexpr int EPV = 16 / int(sizeof(T));
+  __shared__ int warp_cnt[THREADS / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int active = 0;
+  for (int r = warp; r < TILE; r += THREADS / 32) {
+    const long long tok = (long long)blockIdx.x * TILE + r;
+    if (tok >= n) break;
+    const uint4 *a = reinterpret_cast<const uint4 *>(cur) + tok * row_vecs;
+    const uint4 *b = reinterpret_cast<const uint4 *>(prev) + tok * row_vecs;
+    float acc = 0.f;
+    for (int v0 = 0; v0 < row_vecs; v0 += 32 * VMAX) {
+      uint4 va[VMAX], vb[VMAX];
+#pragma unroll
+      for (int u = 0; u < VMAX; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < row_vecs) { va[u] = __ldg(a + v); vb[u] = __ldg(b + v); }
+      }
+#pragma unroll
+      for (int u = 0; u < VMAX; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < row_vecs) {
+#pragma unroll
+          for (int k = 0; k < EPV; ++k) {
+            float x, y;
+            if constexpr (sizeof(T) == 2) {
+              x = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(&va[u])[k]);
+              y = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(&vb[u])[k]);
+            } else {
+              x = reinterpret_cast<const float *>(&va[u])[k];
+              y = reinterpret_cast<const float *>(&vb[u])[k];
+            }
+            acc += fabsf(x - y);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const int m = (force_all || acc > tau) ? 1 : 0;
+    if (lane == 0) {
+      mask[tok] = (unsigned char)m;
+      if (l1_out) l1_out[tok] = acc;
+    }
+    active += m;
+  }
+  if (lane == 0) warp_cnt[warp] = active;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int c = 0;
+    for (int w = 0; w < THREADS / 32; ++w) c += warp_cnt[w];
+    tile_count[blockIdx.x] = c;
+  }
+}
+
+// One CTA per CTILE tokens.  Exclusive prefix = sum of the L1-pass counts of
+// the tiles before this CTA's first token, then warp ballots rank the active
+// tokens inside the CTA in ascending order.
+__global__ void __launch_bounds__(THREADS) compact(const unsigned char *__restrict__ mask, long long n,
+                                                   int n_ctas, const int *__restrict__ tile_count,
+                                                   int *__restrict__ idx, int *__restrict__ count) {
+  __shared__ int red[THREADS / 32];
+  __shared__ int warp_tot[THREADS / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long first_tile = (long long)blockIdx.x * (CTILE / TILE);
+  int part = 0;
+  for (long long t = threadIdx.x; t < first_tile; t += THREADS) part += tile_count[t];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if (lane == 0) red[warp] = part;
+  // each warp owns ROUNDS consecutive groups of 32 tokens
+  const long long tok0 = (long long)blockIdx.x * CTILE + (long long)warp * (ROUNDS * 32);
+  unsigned bal[ROUNDS];
+  int tot = 0;
+#pragma unroll
+  for (int r = 0; r < ROUNDS; ++r) {
+    const long long tok = tok0 + r * 32 + lane;
+    const int m = (tok < n) ? mask[tok] : 0;
+    bal[r] = __ballot_sync(0xffffffffu, m);
+    tot += __popc(bal[r]);
+  }
+  if (lane == 0) warp_tot[warp] = tot;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < THREADS / 32; ++w) base += red[w];
+  int total_cta = 0;
+  for (int w = 0; w < THREADS / 32; ++w) {
+    if (w < warp) base += warp_tot[w];
+    total_cta += warp_tot[w];
+  }
+#pragma unroll
+  for (int r = 0; r < ROUNDS; ++r) {
+    if ((bal[r] >> lane) & 1u) idx[base + __popc(bal[r] & ((1u << lane) - 1u))] = int(tok0 + r * 32 + lane);
+    base += __popc(bal[r]);
+  }
+  if (blockIdx.x == n_ctas - 1 && threadIdx.x == 0) {
+    int all = 0;
+    for (int w = 0; w < THREADS / 32; ++w) all += red[w];
+    *count = all + total_cta;
+  }
+}
+
+// One warp per active row: copies each tensor's row to its cache (and to the
+// packed message buffer when present).
+struct ScatterArgs {
+  const char *src[8];
+  char *dst[8];
+  char *packed[8];
+};
+
+__global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
+                                                    const int *__restrict__ count, long long n,
+                                                    long long row_bytes, int vec, int n_tensors,
+                                                    ScatterArgs a) {
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long cnt = *count;
+  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long i = w; i < cnt && i < n; i += n_warps) {
+    const long long row = idx[i];
+    if (row < 0 || row >= n) continue;
+    for (int t = 0; t < n_tensors; ++t) {
+      if (vec == 16) {
+        const uint4 *s = reinterpret_cast<const uint4 *>(a.src[t] + row * row_bytes);
+        uint4 *d = reinterpret_cast<uint4 *>(a.dst[t] + row * row_bytes);
+        uint4 *p = a.packed[t] ? reinterpret_cast<uint4 *>(a.packed[t] + i * row_bytes) : nullptr;
+        for (long long k = lane; k < row_bytes / 16; k += 32) {
+          const uint4 v = __ldg(s + k);
+          d[k] = v;
+          if (p) p[k] = v;
+        }
+      } else {
+        const char *s = a.src[t] + row * row_bytes;
+        char *d = a.dst[t] + row * row_bytes;
+        char *p = a.packed[t] ? a.packed[t] + i * row_bytes : nullptr;
+        for (long long k = lane; k < row_bytes; k += 32) {
+          const char v = s[k];
+          d[k] = v;
+          if (p) p[k] = v;
+        }
+      }
+    }
+  }
+}
+
+inline long long n_tiles_of(long long n) { return (n + TILE - 1) / TILE; }
+
+}  // namespace
+
+ST_API size_t vmajor_workspace_bytes(long long n_tokens) {
+  if (n_tokens <= 0) return 0;
+  return size_t(n_tiles_of(n_tokens)) * sizeof(int);
+}
+
+ST_API st_status vmajor_mask_compact(const void *v_cur, const void *v_prev, long long n_tokens, int C,
+                                     st_dtype dtype, float tau, int force_all, unsigned char *mask,
+                                     int *idx, int *count, float *l1_out, void *workspace,
+                                     size_t workspace_bytes, st_stream_t stream) {
+  if (!v_cur || !v_prev || !mask || !idx || !count) return ST_ERR_NULL;
+  if (n_tokens <= 0 || C <= 0 || n_tokens >= (1LL << 31)) return ST_ERR_SHAPE;
+  if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_DTYPE;
+  const int esize = dtype == ST_F32 ? 4 : 2;
+  if ((C * esize) % 16 || !st::is_aligned(v_cur, 16) || !st::is_aligned(v_prev, 16)) return ST_ERR_ALIGN;
+  if (!workspace) return ST_ERR_NULL;
+  if (workspace_bytes < vmajor_workspace_bytes(n_tokens)) return ST_ERR_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long tiles = n_tiles_of(n_tokens);
+  if (tiles > 0x7fffffffLL) return ST_ERR_SHAPE;
+  const int row_vecs = C * esize / 16;
+  int *tile_count = static_cast<int *>(workspace);
+  if (dtype == ST_BF16)
+    l1_mask<uint16_t><<<int(tiles), THREADS, 0, s>>>(static_cast<const char *>(v_cur),
+                                                     static_cast<const char *>(v_prev), n_tokens,
+                                                     row_vecs, tau, force_all, mask, l1_out, tile_count);
+  else
+    l1_mask<float><<<int(tiles), THREADS, 0, s>>>(static_cast<const char *>(v_cur),
+                                                  static_cast<const char *>(v_prev), n_tokens,
+                                                  row_vecs, tau, force_all, mask, l1_out, tile_count);
+  st_status st = st::launch_status();
+  if (st != ST_OK) return st;
+  const int ctas = int((n_tokens + CTILE - 1) / CTILE);
+  compact<<<ctas, THREADS, 0, s>>>(mask, n_tokens, ctas, tile_count, idx, count);
+  return st::launch_status();
+}
+
+ST_API st_status vmajor_scatter_rows(const int *idx, const int *count, long long n_tokens, int C,
+                                     int elem_bytes, const void *const *src, void *const *dst_cache,
+                                     int n_tensors, void *const *packed, st_stream_t stream) {
+  if (!idx || !count || !src || !dst_cache) return ST_ERR_NULL;
+  if (n_tensors < 1 || n_tensors > 8 || n_tokens <= 0 || C <= 0) return ST_ERR_SHAPE;
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8) return ST_ERR_DTYPE;
+  ScatterArgs a = {};
+  const long long row_bytes = (long long)C * elem_bytes;
+  bool all16 = (row_bytes % 16) == 0;
+  for (int t = 0; t < n_tensors; ++t) {
+    if (!src[t] || !dst_cache[t]) return ST_ERR_NULL;
+    a.src[t] = static_cast<const char *>(src[t]);
+    a.dst[t] = static_cast<char *>(dst_cache[t]);
+    a.packed[t] = packed ? static_cast<char *>(packed[t]) : nullptr;
+    all16 = all16 && st::is_aligned(src[t], 16) && st::is_aligned(dst_cache[t], 16) &&
+            (!a.packed[t] || st::is_aligned(a.packed[t], 16));
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long want = (n_tokens * 32 + 255) / 256;
+  const long long cap = (long long)st::num_sms() * 16;
+  const int grid = int(want < cap ? want : cap);
+  scatter_rows<<<grid, 256, 0, s>>>(idx, count, n_tokens, row_bytes, all16 ? 16 : 1, n_tensors, a);
+  return st::launch_status();
+}

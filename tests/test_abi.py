@@ -1,0 +1,124 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before launching anything (CPU only: no call here
+reaches the GPU)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def st():
+    from sequence_parallelism_st_b200 import build as b
+    if not os.path.exists(b.LIB):
+        b.build()
+    import sequence_parallelism_st_b200 as st
+    return st
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?(?:st_status|int|size_t|char|void)\s*\*?\s*(\w+)\s*\(",
+                             text, flags=re.M):
+            names.append(m.group(1))
+    return names
+
+
+def test_every_declared_symbol_is_exported(st):
+    names = declared_functions()
+    assert {"st_attn_spatial", "st_attn_temporal", "attn_chunk_merge", "ulysses_relayout",
+            "vmajor_mask_compact", "vmajor_scatter_rows", "st_check_device_status"} <= set(names)
+    raw = ctypes.CDLL(st.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in include/ but not exported"
+    assert set(names) <= set(st.EXPORTED)
+
+
+def test_status_strings_and_version(st):
+    assert st.st_status_string(0) == "ST_OK"
+    for code in range(-8, 0):
+        assert st.st_status_string(code).startswith("ST_ERR_")
+    assert st._c["st_abi_version"]() == 1
+    assert st.vmajor_workspace_bytes(20736) >= 4 * (20736 // 32)
+    assert st.vmajor_workspace_bytes(0) == 0
+
+
+FAKE_IN, FAKE_OUT = ctypes.c_void_p(0x100000), ctypes.c_void_p(0x90000000)
+
+
+def relayout(st, mode, elem=2, P=2, B=1, T=8, S=16, C=64, n_t=1, n_s=1, blk=None, inp=FAKE_IN, out=FAKE_OUT,
+             gamma=None, hd=0):
+    i0, i1, j0, j1 = blk if blk else (0, n_t, 0, n_s)
+    return st._c["ulysses_relayout"](mode, inp, out, elem, P, B, T, S, C, n_t, n_s, i0, i1, j0, j1, gamma, hd,
+                                     1e-6, None)
+
+
+def test_relayout_rejects(st):
+    assert relayout(st, st.ST_S2T, inp=None) == st.ST_ERR_NULL
+    assert relayout(st, st.ST_S2T, elem=3) == st.ST_ERR_DTYPE
+    assert relayout(st, st.ST_S2T, T=6, P=4) == st.ST_ERR_DIVISIBILITY
+    assert relayout(st, st.ST_S2T, n_t=2, T=6, P=2) == st.ST_ERR_DIVISIBILITY
+    assert relayout(st, st.ST_S2T, n_t=2, blk=(0, 3, 0, 1)) == st.ST_ERR_SHAPE
+    assert relayout(st, st.ST_S2T, n_t=2, blk=(1, 1, 0, 1)) == st.ST_ERR_SHAPE
+    assert relayout(st, st.ST_SEQ2HEAD, n_t=2) == st.ST_ERR_SHAPE
+    assert relayout(st, st.ST_SEQ2HEAD, S=3) == st.ST_ERR_DIVISIBILITY
+    assert relayout(st, 7) == st.ST_ERR_UNSUPPORTED
+    assert relayout(st, st.ST_S2T, P=0) == st.ST_ERR_SHAPE
+    assert relayout(st, st.ST_S2T, gamma=FAKE_IN, hd=48) == st.ST_ERR_SHAPE
+    assert relayout(st, st.ST_S2T, out=ctypes.c_void_p(0x100000 + 64)) == st.ST_ERR_SHAPE   # overlap
+
+
+def spatial(st, fn="st_attn_spatial", q=FAKE_IN, **kw):
+    d = dict(B=1, T=2, S=64, H=2, D=72, dtype=st.ST_BF16)
+    d.update(kw)
+    desc = st.make_desc(**d)
+    return st._c[fn](ctypes.byref(desc), q, FAKE_IN, FAKE_IN, FAKE_OUT, None, None)
+
+
+def test_attention_rejects(st):
+    assert st._c["st_attn_spatial"](None, FAKE_IN, FAKE_IN, FAKE_IN, FAKE_OUT, None, None) == st.ST_ERR_NULL
+    assert spatial(st, q=None) == st.ST_ERR_NULL
+    bad = st.make_desc(1, 2, 64, 2, 72)
+    bad.size = 12
+    assert st._c["st_attn_spatial"](ctypes.byref(bad), FAKE_IN, FAKE_IN, FAKE_IN, FAKE_OUT, None, None) == st.ST_ERR_SHAPE
+    assert spatial(st, B=0) == st.ST_ERR_SHAPE
+    assert spatial(st, dtype=5) == st.ST_ERR_DTYPE
+    assert spatial(st, D=48) == st.ST_ERR_UNSUPPORTED
+    assert spatial(st, q=ctypes.c_void_p(0x100008)) == st.ST_ERR_ALIGN
+    assert spatial(st, stride_s=148) == st.ST_ERR_ALIGN
+    assert spatial(st, kv_begin=10, kv_end=5) == st.ST_ERR_SHAPE
+    assert spatial(st, kv_begin=0, kv_end=65) == st.ST_ERR_SHAPE
+    assert spatial(st, n_slices=3, slice=0) == st.ST_ERR_DIVISIBILITY
+    assert spatial(st, n_slices=2, slice=2) == st.ST_ERR_SHAPE
+    assert spatial(st, t_block=3) == st.ST_ERR_DIVISIBILITY
+    assert spatial(st, "st_attn_temporal", T=65) == st.ST_ERR_UNSUPPORTED
+    assert spatial(st, "st_attn_temporal", kv_begin=1, kv_end=3) == st.ST_ERR_SHAPE
+    assert spatial(st, "st_attn_temporal", D=40) == st.ST_ERR_UNSUPPORTED
+
+
+def test_merge_and_vmajor_reject(st):
+    VP = ctypes.c_void_p
+    arr = (VP * 2)(0x100000, 0x200000)
+    f = st._c["attn_chunk_merge"]
+    assert f(0, arr, arr, 1, 8, 2, 64, FAKE_OUT, st.ST_BF16, None, None) == st.ST_ERR_SHAPE
+    assert f(17, arr, arr, 1, 8, 2, 64, FAKE_OUT, st.ST_BF16, None, None) == st.ST_ERR_SHAPE
+    assert f(2, arr, arr, 1, 8, 2, 66, FAKE_OUT, st.ST_BF16, None, None) == st.ST_ERR_ALIGN
+    assert f(2, arr, arr, 1, 8, 2, 64, None, st.ST_BF16, None, None) == st.ST_ERR_NULL
+    assert f(2, arr, arr, 1, 8, 2, 64, FAKE_OUT, 9, None, None) == st.ST_ERR_DTYPE
+    g = st._c["vmajor_mask_compact"]
+    ws = st.vmajor_workspace_bytes(100)
+    assert g(None, FAKE_IN, 100, 64, st.ST_BF16, 1.0, 0, FAKE_OUT, FAKE_OUT, FAKE_OUT, None, FAKE_OUT, ws, None) == st.ST_ERR_NULL
+    assert g(FAKE_IN, FAKE_IN, 100, 64, st.ST_BF16, 1.0, 0, FAKE_OUT, FAKE_OUT, FAKE_OUT, None, FAKE_OUT, ws - 4, None) == st.ST_ERR_SHAPE
+    assert g(FAKE_IN, FAKE_IN, 100, 60, st.ST_BF16, 1.0, 0, FAKE_OUT, FAKE_OUT, FAKE_OUT, None, FAKE_OUT, ws, None) == st.ST_ERR_ALIGN
+    assert g(FAKE_IN, FAKE_IN, 0, 64, st.ST_BF16, 1.0, 0, FAKE_OUT, FAKE_OUT, FAKE_OUT, None, FAKE_OUT, ws, None) == st.ST_ERR_SHAPE
+    h = st._c["vmajor_scatter_rows"]
+    assert h(FAKE_IN, FAKE_IN, 100, 64, 2, arr, arr, 0, None, None) == st.ST_ERR_SHAPE
+    assert h(FAKE_IN, FAKE_IN, 100, 64, 2, arr, arr, 9, None, None) == st.ST_ERR_SHAPE
+    assert h(FAKE_IN, FAKE_IN, 100, 64, 3, arr, arr, 2, None, None) == st.ST_ERR_DTYPE

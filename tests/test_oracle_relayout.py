@@ -151,9 +151,11 @@ def test_vmajor_pins():
 def test_tau_for_fraction():
     l1 = np.random.default_rng(12).lognormal(size=1000)
     for f in (0.1, 0.5, 0.9):
-        tau, margin = oracle.tau_for_fraction(l1, f)
-        assert (l1 > tau).sum() == round(1000 * f)
+        tau, margin, frac = oracle.tau_for_fraction(l1, f, window=0.0)
+        assert (l1 > tau).sum() == round(1000 * f) and frac == (l1 > tau).mean()
         assert margin > 0
+        tau2, margin2, frac2 = oracle.tau_for_fraction(l1, f, window=0.02)
+        assert abs(frac2 - f) <= 0.021 and margin2 >= margin
 
 
 def test_vmajor_recipe_small_sigma_rounds_back():
@@ -163,3 +165,17 @@ def test_vmajor_recipe_small_sigma_rounds_back():
     sig = synth.token_sigma(w, 512)
     l1 = oracle.l1_change(cur, prev)
     assert l1[sig < 2e-4].mean() < l1[sig > 5e-2].mean() / 50
+
+
+def test_row_pairs_agree_with_relayout():
+    r = np.random.default_rng(13)
+    P, B, T, S, C, n_t, n_s = 2, 1, 8, 12, 3, 2, 3
+    x = r.normal(size=P * B * T * (S // P) * C)
+    dst, src = oracle.st_row_pairs("S2T", P, B, T, S, n_t, n_s, blocks=(1, 2, 0, 2))
+    full = oracle.st_relayout("S2T", x, P, B, T, S, C, n_t, n_s, blocks=(1, 2, 0, 2))
+    np.testing.assert_array_equal(full.reshape(-1, C)[dst], x.reshape(-1, C)[src])
+    P, N, H, D = 4, 8, 8, 2
+    y = r.normal(size=B * N * H * D)
+    dst, src = oracle.seq_head_row_pairs("HEAD2SEQ", P, B, N, H)
+    np.testing.assert_array_equal(oracle.seq_head_relayout("HEAD2SEQ", y, P, B, N, H, D).reshape(-1, D)[dst],
+                                  y.reshape(-1, D)[src])
