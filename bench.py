@@ -1,0 +1,447 @@
+"""Benchmark of the spatial-temporal attention hot path on B200.
+
+One step = one pass of every hot-path step over one ST-DiT attention block of
+the OpenSora-like low-resolution workload (B=1, T=16 frames, S=1200 tokens,
+16 heads x 72, bf16, virtual P=4, N_T=N_S=4, KV chunks R=2):
+
+  1. all-to-all S->T of Q and K with the fused per-head RMSNorm, and of V
+     (ulysses_relayout on the [B,N_T,N_S,T/N_T,S/N_S/P,C] slice layouts);
+  2. V-Major change mask of V against the previous step's V, compaction of
+     the active tokens (vmajor_mask_compact), cache update of K/V rows of the
+     active tokens (vmajor_scatter_rows);
+  3. spatial attention of the fresh Q against the cached K/V in R KV chunks
+     (st_attn_spatial, fp32 partials + LSE) and their log-sum-exp merge
+     (attn_chunk_merge);
+  4. all-to-all T->S of the spatial output;
+  5. temporal attention over the T frames of every token, read in place from
+     the spatially sharded slice layout (st_attn_temporal).
+
+value = attention FLOP of the step (4*rows*keys*D per head, spatial and
+temporal) / device time of the step; the per-kernel breakdown (TFLOP/s or
+GB/s) is in "kernels".  Inputs are resident in HBM; L2 is flushed (a
+256 MiB write) between timed steps, outside the timed events.  Under torchrun
+every rank runs its own replica (weak scaling, no collective on the data
+path); the time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "attention TFLOP/s & relayout GB/s on 1 B200, as fraction of bf16/HBM peak"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 11
+SPATIAL_SRC = os.path.join(ROOT, "sequence_parallelism_st_b200", "csrc", "attn_spatial_sm100.cu")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK, "fallback"
+
+
+def kernel_traffic():
+    """DRAM bytes per launch of the spatial kernel from the committed ncu summary,
+    or None when the kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    h = hashlib.sha256(open(SPATIAL_SRC, "rb").read()).hexdigest()[:16]
+    e = d.get("st_attn_spatial", {})
+    if e.get("source_sha") != h or e.get("workload") != "opensora_low":
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.stop_ev, self.thread, self.index = period, threading.Event(), None, index
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self.stop_ev.set()
+        if self.thread:
+            self.thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- our arm
+class Step:
+    """Buffers and launches of one ST-DiT attention block step (all on one stream)."""
+
+    def __init__(self, st, w, dev):
+        self.st, self.w, self.dev = st, w, dev
+        B, T, S, H, D, C, P = w.B, w.T, w.S, w.H, w.D, w.C, w.P
+        n = B * T * S
+        q, k, v = synth.qkv(w)                                # logical [B,T,S,H,D]
+        vcur, vprev = synth.vmajor_pair(w, n, C)              # logical token order (b, t, s)
+        self.tau = json.load(open(os.path.join(ROOT, "tests", "golden", "vmajor_tau.json")))[
+            "workloads"][w.name]["0.5"]["tau"]
+        self.n = n
+        # the block's V is the V-Major "current" V; x layout holds shard p of every frame
+        v = vcur.reshape(B, T, S, H, D)
+        self.host = {"q": self.to_x(q), "k": self.to_x(k), "v": self.to_x(v)}
+        self.gamma = synth.rms_gamma(w).to(dev)
+        # previous step's V and K/V caches, already in the temporally sharded (y) layout
+        vprev_y = self.x_to_y_host(self.to_x(vprev.reshape(B, T, S, H, D)))
+        kprev = synth.randn(w, "kprev", (B, T, S, H, D))
+        kprev_y = self.x_to_y_host(self.to_x(kprev))
+        self.d = {name: t.to(dev) for name, t in self.host.items()}
+        self.vprev_y = vprev_y.to(dev)
+        self.kcache0, self.vcache0 = kprev_y.to(dev), vprev_y.to(dev)
+        self.kc, self.vc = self.kcache0.clone(), self.vcache0.clone()
+        mk = lambda dt=torch.bfloat16: torch.empty(n * C, dtype=dt, device=dev)
+        self.qy, self.ky, self.vy, self.oy, self.ox, self.ot = mk(), mk(), mk(), mk(), mk(), mk()
+        self.parts = [torch.empty(n * C, dtype=torch.float32, device=dev) for _ in range(w.R)]
+        self.lses = [torch.empty(n * H, dtype=torch.float32, device=dev) for _ in range(w.R)]
+        self.mask = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.idx = torch.empty(n, dtype=torch.int32, device=dev)
+        self.count = torch.empty(1, dtype=torch.int32, device=dev)
+        self.ws = torch.empty(max(16, st.vmajor_workspace_bytes(n)), dtype=torch.uint8, device=dev)
+        # y layout with T/(N_T P) = 1: frames (q, i) of S contiguous tokens -> dense [1, T, S, H, D]
+        assert T % (w.n_t * P) == 0 and T // (w.n_t * P) == 1
+        self.sdesc = [st.make_desc(1, T, S, H, D, st.ST_BF16, kv_begin=c * S // w.R, kv_end=(c + 1) * S // w.R,
+                                   o_fp32=1) for c in range(w.R)]
+        Tb, Sb = T // w.n_t, S // (w.n_s * P)
+        self.tdesc = st.make_desc(P * B, T, S // P, H, D, st.ST_BF16, stride_b=w.n_t * w.n_s * Tb * Sb * C,
+                                  stride_t=Sb * C, stride_s=C, t_block=Tb, stride_tb=w.n_s * Tb * Sb * C,
+                                  s_block=Sb, stride_sb=Tb * Sb * C)
+        # per-kernel timing events (launching stream = torch's current stream)
+        self.ev = {}
+
+    def to_x(self, t):
+        """Logical [B,T,S,H,D] -> stacked x shards [P,B,N_T,N_S,T/N_T,S/(N_S P),C]."""
+        w = self.w
+        X = t.reshape(w.B, w.T, w.S, w.C)
+        Tb, Sb = w.T // w.n_t, w.S // (w.n_s * w.P)
+        return X.reshape(w.B, w.n_t, Tb, w.n_s, w.P, Sb, w.C).permute(4, 0, 1, 3, 2, 5, 6).contiguous().reshape(-1)
+
+    def x_to_y_host(self, x):
+        """Host-side layout change used only to prepare the previous step's buffers."""
+        w = self.w
+        Tb, Sb = w.T // w.n_t, w.S // (w.n_s * w.P)
+        X = x.reshape(w.P, w.B, w.n_t, w.n_s, Tb, Sb, w.C).permute(1, 2, 4, 3, 0, 5, 6)  # b i t1 j p s1 c
+        X = X.reshape(w.B, w.T, w.S, w.C)        # logical
+        Tq, Ss = w.T // (w.n_t * w.P), w.S // w.n_s
+        Y = X.reshape(w.B, w.n_t, w.P, Tq, w.n_s, Ss, w.C).permute(2, 0, 1, 4, 3, 5, 6)
+        return Y.contiguous().reshape(-1)
+
+    def reset_caches(self):
+        self.kc.copy_(self.kcache0)
+        self.vc.copy_(self.vcache0)
+
+    def _mark(self, name, start):
+        if self.timing:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            self.ev.setdefault(name, []).append(e) if start else self.ev[name].append(e)
+
+    def run(self, timing=False):
+        st, w, d = self.st, self.w, self.d
+        self.timing = timing
+        P, B, T, S, C, D = w.P, w.B, w.T, w.S, w.C, w.D
+        self._mark("relayout_s2t", True)
+        st.ulysses_relayout("S2T", d["q"], self.qy, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
+                            rms_head_dim=D, rms_eps=w.rms_eps)
+        st.ulysses_relayout("S2T", d["k"], self.ky, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
+                            rms_head_dim=D, rms_eps=w.rms_eps)
+        st.ulysses_relayout("S2T", d["v"], self.vy, P, B, T, S, C, w.n_t, w.n_s)
+        self._mark("relayout_s2t", False)
+        self._mark("vmajor", True)
+        st.vmajor_mask_compact(self.vy.view(self.n, C), self.vprev_y.view(self.n, C), self.tau, self.mask,
+                               self.idx, self.count, self.ws)
+        st.vmajor_scatter_rows(self.idx, self.count, [self.ky.view(self.n, C), self.vy.view(self.n, C)],
+                               [self.kc.view(self.n, C), self.vc.view(self.n, C)])
+        self._mark("vmajor", False)
+        self._mark("spatial", True)
+        for c in range(w.R):
+            st.st_attn_spatial(self.qy, self.kc, self.vc, self.parts[c], self.lses[c], desc=self.sdesc[c])
+        self._mark("spatial", False)
+        self._mark("merge", True)
+        st.attn_chunk_merge(self.parts, self.lses, B * T, S, w.H, D, self.oy)
+        self._mark("merge", False)
+        self._mark("relayout_t2s", True)
+        st.ulysses_relayout("T2S", self.oy, self.ox, P, B, T, S, C, w.n_t, w.n_s)
+        self._mark("relayout_t2s", False)
+        self._mark("temporal", True)
+        st.st_attn_temporal(d["q"], d["k"], d["v"], self.ot, None, desc=self.tdesc)
+        self._mark("temporal", False)
+
+    def kernel_times(self):
+        out = {}
+        for name, evs in self.ev.items():
+            ts = [evs[i].elapsed_time(evs[i + 1]) for i in range(0, len(evs) - 1, 2)]
+            out[name] = sum(ts) / len(ts)
+        return out
+
+
+def flops(w):
+    return w.spatial_flops() + w.temporal_flops()
+
+
+def kernel_bytes(w, frac_active):
+    """Algorithmic HBM bytes per step of each memory-bound kernel group."""
+    e = w.elem_bytes
+    t = w.B * w.T * w.S * w.C * e               # one [B,T,S,C] tensor
+    rows = w.B * w.T * w.S * w.H
+    return {
+        "relayout_s2t": 3 * 2 * t,
+        "vmajor": 2 * t + 2 * 2 * frac_active * t,
+        "merge": w.R * (2 * t + rows * 4) + t,  # fp32 partials + LSE in, bf16 out
+        "relayout_t2s": 2 * t,
+        "temporal": 4 * t,
+    }
+
+
+def run_ours(args, w, rank, world, dev):
+    import sequence_parallelism_st_b200 as st
+    stp = Step(st, w, dev)
+    pk, pk_src = peaks()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        stp.run()
+    torch.cuda.synchronize()
+    if st.st_check_device_status() != st.ST_OK:
+        raise RuntimeError("device status not OK after warm-up")
+    active = int(stp.count.item())
+    # ---- timed: device time of exactly K steps, L2 flushed between steps outside the events
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                      else int(os.environ.get("LOCAL_RANK", 0))) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record()
+            stp.run(timing=True)
+            ends[i].record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = st.st_check_device_status()
+    ktimes = stp.kernel_times()
+    # ---- end to end through the C ABI with host buffers: H2D of the step's inputs,
+    #      the step, D2H of its outputs, all inside the events
+    pinned_in = {k: v.pin_memory() for k, v in stp.host.items()}
+    out_host = [torch.empty(stp.n * w.C, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    h2d = sum(v.numel() * v.element_size() for v in pinned_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host)
+    e2e_ms = []
+    for i in range(max(3, args.steps // 4) + 2):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for k2, v2 in pinned_in.items():
+            stp.d[k2].copy_(v2, non_blocking=True)
+        stp.run()
+        out_host[0].copy_(stp.ox, non_blocking=True)
+        out_host[1].copy_(stp.ot, non_blocking=True)
+        b.record()
+        b.synchronize()
+        if i >= 2:
+            e2e_ms.append(a.elapsed_time(b))
+    if rank != 0:
+        return None
+    f = flops(w)
+    n_steps = args.steps
+    ms = total_ms / n_steps
+    value = world * f / (ms * 1e-3) / 1e12
+    e2e_val = world * f / (statistics.mean(e2e_ms) * 1e-3) / 1e12
+    frac_active = active / stp.n
+    kb = kernel_bytes(w, frac_active)
+    kernels = {}
+    for name, t in ktimes.items():
+        ent = {"ms": round(t, 5)}
+        if name == "spatial":
+            ent["tflops"] = round(w.spatial_flops() / (t * 1e-3) / 1e12, 2)
+            ent["frac_of_bf16_peak"] = round(ent["tflops"] / pk["bf16_tflops"], 4)
+        else:
+            ent["gbs"] = round(kb[name] / (t * 1e-3) / 1e9, 1)
+            ent["frac_of_hbm_peak"] = round(ent["gbs"] / pk["hbm_gbs"], 4)
+            if name == "temporal":
+                ent["tflops"] = round(w.temporal_flops() / (t * 1e-3) / 1e12, 2)
+        kernels[name] = ent
+    # roofline of the dominant kernel: spatial attention, R launches per step
+    sp_launch_ms = ktimes["spatial"] / w.R
+    achieved = (w.spatial_flops() / w.R) / (sp_launch_ms * 1e-3) / 1e12
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": n_steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "H": w.H, "D": w.D, "P": w.P,
+                   "N_T": w.n_t, "N_S": w.n_s, "kv_chunks": w.R, "vmajor_active": round(frac_active, 4),
+                   "parallelism": f"replicas{world}", "l2": "flushed between timed steps (256 MiB write, "
+                   "outside the step events)"},
+        "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(statistics.mean(e2e_ms), 5)},
+        "roofline": {"bound": "tensor", "kernel": "st_attn_spatial", "achieved": round(achieved, 2),
+                     "peak": pk["bf16_tflops"], "peak_source": f"{pk_src} bf16 burst", "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": kernel_traffic(),
+                     "algorithmic_flop_per_launch": w.spatial_flops() / w.R},
+        "kernels": kernels,
+        "gpu_launches": LAUNCHES_PER_STEP * n_steps,
+        "device_status": st.st_status_string(status),
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu_baseline(w, budget_s=args.cpu_budget) if world == 1 else None,
+    }
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample(w, n_frames, n_tokens):
+    """The oracle on a bounded sample of the step: spatial attention of n_frames
+    frames and temporal attention of n_tokens tokens.  Returns (seconds, flop)."""
+    import numpy as np
+    import oracle
+    q, k, v = synth.qkv(w)
+    frames = list(range(n_frames))
+    toks = np.arange(n_tokens)
+    t0 = time.perf_counter()
+    oracle.spatial(q, k, v, frames=frames)
+    oracle.temporal(q, k, v, tokens=toks)
+    dt = time.perf_counter() - t0
+    fl = 4.0 * w.B * n_frames * w.S * w.S * w.C + 4.0 * w.B * n_tokens * w.T * w.T * w.C
+    return dt, fl
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, budget_s=15.0):
+    dt, fl = oracle_sample(w, 1, 256)
+    n_frames = max(1, min(w.T, int(budget_s / max(dt, 1e-3))))
+    dt, fl = oracle_sample(w, n_frames, 1200)
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle: spatial attention of {n_frames} of {w.T} frames (all heads, all "
+                      f"{w.S} queries and keys) + temporal attention of 1200 of {w.S} tokens; {dt:.1f} s"}
+
+
+def run_reference(args, w):
+    dt, fl = oracle_sample(w, 1, 256)
+    n_frames = max(1, min(w.T, int(args.cpu_budget / max(args.steps, 1) / max(dt, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample(w, 1, 64)
+    times, fls = [], []
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(w, n_frames, 300)
+        times.append(dt)
+        fls.append(fl)
+    tot = sum(times)
+    val = sum(fls) / tot / 1e12
+    ms = 1e3 * tot / args.steps
+    sample = (f"fp64 numpy oracle per step: spatial attention of {n_frames} of {w.T} frames (all heads, all "
+              f"{w.S} queries and keys) + temporal attention of 300 of {w.S} tokens")
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "H": w.H, "D": w.D},
+            "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="opensora_low")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = synth.BY_NAME[args.workload]
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        res = run_ours(args, w, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -126,7 +126,8 @@ def merge_chunks(o_parts, lse_parts):
     o_c = np.stack([_f64(x) for x in o_parts])                # [R, ..., D]
     M = lse_c.max(axis=0)
     Ms = np.where(np.isfinite(M), M, 0.0)
-    lse = Ms + np.log(np.exp(lse_c - Ms).sum(axis=0))
+    with np.errstate(divide="ignore"):                        # rows with no keys: ln 0 = -inf
+        lse = Ms + np.log(np.exp(lse_c - Ms).sum(axis=0))
     lse = np.where(np.isfinite(M), lse, -np.inf)
     w = np.where(np.isfinite(lse), np.exp(lse_c - np.where(np.isfinite(lse), lse, 0.0)), 0.0)
     o = (w[..., None] * o_c).sum(axis=0)
