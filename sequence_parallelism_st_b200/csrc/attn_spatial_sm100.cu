@@ -64,6 +64,35 @@ template <int D> struct Cfg {
   static_assert(NS >= 2, "ring too shallow");
 };
 
+// ---------------------------------------------------------------- exp2
+// 2^x on the special-function unit (one MUFU op, flush-to-zero).
+__device__ __forceinline__ float ex2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe, for x <= 8.  Range reduction x = j + f with j the
+// nearest integer (adding 1.5 * 2^23 leaves j in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients were
+// fitted for this kernel by a Remez exchange on relative error over
+// [-1/2, 1/2] (max relative error 7.5e-5, far below the bf16 rounding of P);
+// 2^j is added into the exponent field.  x is clamped at -125 so the result
+// stays a normal number (masked scores give 2^-125, i.e. 0 for all purposes).
+constexpr float kP0 = 0.9999280571937561f, kP1 = 0.6932609677314758f;
+constexpr float kP2 = 0.2426111251115799f, kP3 = 0.0551716685295105f;
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(kP3, f, kP2), f, kP1), f, kP0);
+  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
+}
+
+// Of every 8 consecutive score pairs, this many take ex2_poly and the rest the
+// MUFU, so the two pipes share the exponentials of the softmax.
+constexpr int kPolyPairs = 3;
+
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -467,8 +496,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const float e0 = exp2f(fmaf(__uint_as_float(sr[c0 + c]), p.scale_log2, -m));
-            const float e1 = exp2f(fmaf(__uint_as_float(sr[c0 + c + 1]), p.scale_log2, -m));
+            const float x0 = fmaf(__uint_as_float(sr[c0 + c]), p.scale_log2, -m);
+            const float x1 = fmaf(__uint_as_float(sr[c0 + c + 1]), p.scale_log2, -m);
+            float e0, e1;
+            if (((c >> 1) & 7) < kPolyPairs) {
+              e0 = ex2_poly(x0);
+              e1 = ex2_poly(x1);
+            } else {
+              e0 = ex2_mufu(x0);
+              e1 = ex2_mufu(x1);
+            }
             sp[(c >> 1) & 7] += e0 + e1;
             pk[c >> 1] = st::pack_bf16x2(e0, e1);
           }

@@ -88,7 +88,7 @@ WORKLOADS = [
     Workload("opensora_low", 1, B=1, T=16, S=1200, H=16, D=72, dtype="bf16",
              P=4, n_t=4, n_s=4, L_T=1, L_S=3, R=2, rms=True, vmajor_f=(0.5,)),
     Workload("video_1080p", 2, B=1, T=32, S=8160, H=16, D=72, dtype="bf16",
-             P=8, n_t=4, n_s=4, L_T=1, L_S=3, R=2),
+             P=8, n_t=4, n_s=4, L_T=1, L_S=3, R=2, vmajor_f=(0.5,)),
     Workload("image_4096px", 3, B=1, T=1, S=65536, H=24, D=128, dtype="bf16",
              P=8, R=8, rms=True),
     Workload("vmajor_2304px", 4, B=1, T=1, S=20736, H=24, D=128, dtype="bf16",
