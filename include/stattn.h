@@ -202,6 +202,28 @@ st_status vmajor_mask_compact(const void *v_cur, const void *v_prev,
                               int *count, float *l1_out, void *workspace,
                               size_t workspace_bytes, st_stream_t stream);
 
+/* vmajor_mask_compact without a workspace argument, for callers that may not
+ * allocate device memory while they run (a serving loop bound to a fixed
+ * memory pool, or code that must not risk cudaMalloc stalling or failing
+ * mid-step).  The paper has no counterpart; this is a library convenience.
+ * Same arguments, results and errors as vmajor_mask_compact, except that the
+ * per-tile counts live in a file-scope device array of 512 KiB that every GPU
+ * loading the library keeps until the process exits.
+ *   n_tokens above 4,194,304 (1 << 22) returns ST_ERR_SHAPE.
+ *   Allocates nothing: no cudaMalloc/cudaFree and no allocating library call.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   All calls share the one array (it keeps the last call's contents, and
+ *   nothing in it needs to start at zero): calls whose work overlaps on the GPU
+ *   (two streams, or two host threads) race and must be serialised by the
+ *   caller. */
+st_status vmajor_mask_compact_noalloc(const void *v_cur, const void *v_prev,
+                                      long long n_tokens, int C, st_dtype dtype,
+                                      float tau, int force_all, unsigned char *mask,
+                                      int *idx, int *count, float *l1_out,
+                                      st_stream_t stream);
+
 /* Cache update for the active tokens: for i < *count (read on the device),
  *     dst_cache[t][idx[i], :] = src[t][idx[i], :]        for t < n_tensors
  * and, when packed is not NULL, packed[t][i, :] = src[t][idx[i], :] (the

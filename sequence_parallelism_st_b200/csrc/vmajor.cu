@@ -239,3 +239,70 @@ ST_API st_status vmajor_scatter_rows(const int *idx, const int *count, long long
   scatter_rows<<<grid, 256, 0, s>>>(idx, count, n_tokens, row_bytes, all16 ? 16 : 1, n_tensors, a);
   return st::launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of vmajor_mask_compact.
+//
+// Some callers may not allocate device memory while they run: a serving loop
+// that owns a fixed memory pool (or a budget fixed at start-up) must not grow
+// it, and cudaMalloc can stall behind work in flight or fail under memory
+// pressure at the worst moment.  This variant keeps its per-tile counts in a
+// file-scope device array instead of a caller-provided workspace.  The array
+// holds kStaticMaxTokens / TILE ints (512 KiB) on every GPU that loads the
+// library, for the life of the process; larger inputs are rejected.
+#include <mutex>
+
+namespace {
+
+constexpr long long kStaticMaxTokens = 1LL << 22;  // 4,194,304 tokens
+constexpr long long kStaticTiles = kStaticMaxTokens / TILE;
+__device__ __align__(256) int g_vmajor_static_counts[kStaticTiles];
+
+// Device address of the array on the current device.  The first call on a
+// device looks it up with that device current and caches it.
+int *static_counts_on_current_device() {
+  static std::mutex mu;
+  static int *addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_vmajor_static_counts) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int *>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+ST_API st_status vmajor_mask_compact_noalloc(const void *v_cur, const void *v_prev, long long n_tokens, int C,
+                                             st_dtype dtype, float tau, int force_all, unsigned char *mask,
+                                             int *idx, int *count, float *l1_out, st_stream_t stream) {
+  if (!v_cur || !v_prev || !mask || !idx || !count) return ST_ERR_NULL;
+  if (n_tokens <= 0 || C <= 0) return ST_ERR_SHAPE;
+  if (n_tokens > kStaticMaxTokens) return ST_ERR_SHAPE;  // beyond the static scratch capacity
+  if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_DTYPE;
+  const int esize = dtype == ST_F32 ? 4 : 2;
+  if ((C * esize) % 16 || !st::is_aligned(v_cur, 16) || !st::is_aligned(v_prev, 16)) return ST_ERR_ALIGN;
+  int *tile_count = static_counts_on_current_device();
+  if (!tile_count) return ST_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long tiles = n_tiles_of(n_tokens);
+  const int row_vecs = C * esize / 16;
+  // every tile count is written by the first launch before the second reads
+  // it, so nothing in the array has to start at zero
+  if (dtype == ST_BF16)
+    l1_mask<uint16_t><<<int(tiles), THREADS, 0, s>>>(static_cast<const char *>(v_cur),
+                                                     static_cast<const char *>(v_prev), n_tokens, row_vecs, tau,
+                                                     force_all, mask, l1_out, tile_count);
+  else
+    l1_mask<float><<<int(tiles), THREADS, 0, s>>>(static_cast<const char *>(v_cur),
+                                                  static_cast<const char *>(v_prev), n_tokens, row_vecs, tau,
+                                                  force_all, mask, l1_out, tile_count);
+  st_status st = st::launch_status();
+  if (st != ST_OK) return st;
+  const int ctas = int((n_tokens + CTILE - 1) / CTILE);
+  compact<<<ctas, THREADS, 0, s>>>(mask, n_tokens, ctas, tile_count, idx, count);
+  return st::launch_status();
+}
