@@ -1,6 +1,7 @@
 """Build libstattn.so in-tree: nvcc for sm_100a, one object per source.
 
-Usage: ``python -m sequence_parallelism_st_b200.build [-v] [--force]``.
+Usage: ``python sequence_parallelism_st_b200/build.py [-v] [--force] [--ptxas-v]``
+(run as a file: importing the package itself needs the built library).
 The library lands next to this file; objects go to ``_build/`` at the
 repository root.  nvcc cross-compiles, so no GPU is needed to build.
 """
@@ -12,6 +13,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
+
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")

@@ -13,9 +13,12 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def st():
-    from sequence_parallelism_st_b200 import build as b
-    if not os.path.exists(b.LIB):
-        b.build()
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "stattn_build", os.path.join(ROOT, "sequence_parallelism_st_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    b.build()
     import sequence_parallelism_st_b200 as st
     return st
 
