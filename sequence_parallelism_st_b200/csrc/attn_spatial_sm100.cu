@@ -44,10 +44,12 @@ namespace {
 __device__ unsigned int g_attn_error;        // sites of waits that ran out
 __device__ unsigned int g_attn_abort_epoch;  // launch epoch that must abort
 
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 384;             // 3 warpgroups
 constexpr int BLOCK_M = 128;                 // rows per tile
 constexpr int BLOCK_N = 128;                 // keys per K/V tile
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s per wait
+constexpr int REG_SOFTMAX = 184;             // registers of the two softmax warpgroups
+constexpr int REG_OTHER = 136;                // registers of the load / MMA warpgroup
 
 template <int D> struct Cfg {
   static constexpr int C0 = D >= 64 ? 64 : 32;
@@ -57,9 +59,11 @@ template <int D> struct Cfg {
   static constexpr int SW0 = C0 * 2, SW1 = C1 * 2;     // row bytes = swizzle span
   static constexpr int T0 = BLOCK_M * SW0, T1 = BLOCK_M * SW1;
   static constexpr int TILE = T0 + T1;                 // bytes of one Q/K/V tile
-  static constexpr int NS_RAW = (204800 - 2 * TILE) / (2 * TILE);
+  static constexpr int BUDGET = 204800;
+  static constexpr int QB = (4 * TILE + 4 * TILE <= BUDGET) ? 2 : 1;  // Q double buffer if 2 KV stages fit
+  static constexpr int NS_RAW = (BUDGET - 2 * QB * TILE) / (2 * TILE);
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;   // K/V ring depth
-  static constexpr int SMEM = 1024 + 2 * TILE + 2 * NS * TILE + 256;
+  static constexpr int SMEM = 1024 + 2 * QB * TILE + 2 * NS * TILE + 512;
   static_assert(DP <= 128, "head dim too large");
   static_assert(NS >= 2, "ring too shallow");
 };
@@ -125,7 +129,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of the given parity to complete.
-__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t epoch, int site) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t epoch, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
@@ -205,6 +209,14 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   d |= (uint64_t)(layout & 7u) << 61;
   return d;
 }
+// The same descriptor with everything but the start address fixed at compile
+// time: only one 32-bit add per MMA operand at issue time.
+template <uint32_t LBO, uint32_t SBO, uint32_t LAYOUT>
+__device__ __forceinline__ uint64_t sdesc_c(uint32_t saddr) {
+  constexpr uint32_t hi = ((SBO >> 4) & 0x3FFFu) | (1u << 14) | (LAYOUT << 29);
+  constexpr uint32_t lo_const = ((LBO >> 4) & 0x3FFFu) << 16;
+  return ((uint64_t)hi << 32) | (uint64_t)(((saddr >> 4) & 0x3FFFu) | lo_const);
+}
 __host__ __device__ constexpr uint32_t layout_of(int swizzle_bytes) {
   return swizzle_bytes == 128 ? 2u : (swizzle_bytes == 64 ? 4u : 6u);
 }
@@ -227,6 +239,76 @@ struct Params {
   uint32_t epoch;
 };
 
+// Packed fp32 pair arithmetic (sm_100 f32x2 instructions).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// The polynomial 2^x of ex2_poly on a pair, with packed arithmetic.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 j = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);
+  float2 q = ffma2(make_float2(kP3, kP3), f, make_float2(kP2, kP2));
+  q = ffma2(q, f, make_float2(kP1, kP1));
+  q = ffma2(q, f, make_float2(kP0, kP0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
+}
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_OTHER));
+}
+
+// Work item -> (q block, head, frame); q block fastest so that the CTAs that
+// run together share K/V tiles in L2.
+struct Item {
+  int qb, h, t, b, q0, n_qt, c3, c4;
+};
+__device__ __forceinline__ Item decode(const Params &p, int x) {
+  Item it;
+  it.qb = x % p.q_blocks;
+  x /= p.q_blocks;
+  it.h = x % p.g.H;
+  x /= p.g.H;
+  it.t = p.lo + x % p.n_frames;
+  it.b = x / p.n_frames;
+  it.q0 = it.qb * 2 * BLOCK_M;
+  it.n_qt = (p.g.S - it.q0) > BLOCK_M ? 2 : 1;
+  if (p.tmode) {
+    it.c3 = it.t % p.g.tblk;
+    it.c4 = it.b * (p.g.T / p.g.tblk) + it.t / p.g.tblk;
+  } else {
+    it.c3 = it.t;
+    it.c4 = it.b;
+  }
+  return it;
+}
+
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
@@ -234,51 +316,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                    const __grid_constant__ CUtensorMap tv0, const __grid_constant__ CUtensorMap tv1,
                    const Params p) {
   using K = Cfg<D>;
-  constexpr int NS = K::NS;
+  constexpr int NS = K::NS, QB = K::QB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = base;                          // 2 tiles
-  uint8_t *sK = sQ + 2 * K::TILE;              // NS tiles
+  uint8_t *sQ = base;                          // QB x 2 tiles
+  uint8_t *sK = sQ + QB * 2 * K::TILE;         // NS tiles
   uint8_t *sV = sK + NS * K::TILE;             // NS tiles
   uint64_t *bars = reinterpret_cast<uint64_t *>(sV + NS * K::TILE);
-  uint64_t *q_full = bars;                     // 1
-  uint64_t *k_full = bars + 1;                 // NS
+  uint64_t *q_full = bars;                     // QB
+  uint64_t *q_empty = q_full + QB;             // QB
+  uint64_t *k_full = q_empty + QB;             // NS
   uint64_t *k_empty = k_full + NS;             // NS
   uint64_t *v_full = k_empty + NS;             // NS
   uint64_t *v_empty = v_full + NS;             // NS
   uint64_t *s_full = v_empty + NS;             // 2
   uint64_t *p_full = s_full + 2;               // 2
   uint64_t *o_full = p_full + 2;               // 2
-  uint64_t *mma_done = o_full + 2;             // 1
+  uint64_t *o_empty = o_full + 2;              // 2
+  uint64_t *mma_done = o_empty + 2;            // 1
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
-  int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const st::Geom &g = p.g;
-
-  // ---- work item: (q block, head, frame), q block fastest so that the CTAs
-  //      that run together share K/V tiles in L2
-  int x = blockIdx.x;
-  const int qb = x % p.q_blocks;
-  x /= p.q_blocks;
-  const int h = x % g.H;
-  x /= g.H;
-  const int t = p.lo + x % p.n_frames;
-  const int b = x / p.n_frames;
-  const int q0 = qb * 2 * BLOCK_M;
-  const int n_qt = (g.S - q0) > BLOCK_M ? 2 : 1;
+  const int n_items = p.q_blocks * g.H * p.n_frames * g.B;
   const int n_kv = (p.kv1 - p.kv0 + BLOCK_N - 1) / BLOCK_N;
-  int c3, c4;
-  if (p.tmode) {
-    c3 = t % g.tblk;
-    c4 = b * (g.T / g.tblk) + t / g.tblk;
-  } else {
-    c3 = t;
-    c4 = b;
-  }
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int i = 0; i < QB; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_empty + i, 1);
+    }
     for (int i = 0; i < NS; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 1);
@@ -289,9 +356,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(s_full + i, 1);
       mbar_init(p_full + i, BLOCK_M);
       mbar_init(o_full + i, 1);
+      mbar_init(o_empty + i, BLOCK_M);
     }
     mbar_init(mma_done, 1);
-    *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 9) {
@@ -306,128 +373,149 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t epoch = p.epoch;
 
-  if (warp == 8) {
-    // ================= TMA producer =================
-    if (lane == 0 && n_kv > 0) {
+  if (warp >= 8) {
+    setmaxnreg_dec();
+    if (warp == 8 && lane == 0 && n_kv > 0) {
+      // ================= TMA producer =================
       bool ok = true;
-      int issued = 0;  // K/V loads issued (each j issues one K and one V)
-      mbar_expect_tx(q_full, n_qt * K::TILE);
-      for (int X = 0; X < n_qt; ++X) {
-        uint8_t *dst = sQ + X * K::TILE;
-        tma_load_5d(dst, &tq0, q_full, 0, h, q0 + X * BLOCK_M, c3, c4);
-        if (K::C1) tma_load_5d(dst + K::T0, &tq1, q_full, 64, h, q0 + X * BLOCK_M, c3, c4);
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j % NS;
-        const uint32_t ph = (j / NS) & 1;
-        const int key = p.kv0 + j * BLOCK_N;
-        if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 0))) break;
-        mbar_expect_tx(k_full + st, K::TILE);
-        uint8_t *dk = sK + st * K::TILE;
-        tma_load_5d(dk, &tk0, k_full + st, 0, h, key, c3, c4);
-        if (K::C1) tma_load_5d(dk + K::T0, &tk1, k_full + st, 64, h, key, c3, c4);
-        if (!(ok = mbar_wait(v_empty + st, ph ^ 1, epoch, 1))) { issued = 2 * j + 1; break; }
-        mbar_expect_tx(v_full + st, K::TILE);
-        uint8_t *dv = sV + st * K::TILE;
-        tma_load_5d(dv, &tv0, v_full + st, 0, h, key, c3, c4);
-        if (K::C1) tma_load_5d(dv + K::T0, &tv1, v_full + st, 64, h, key, c3, c4);
-        issued = 2 * (j + 1);
+      uint32_t kv = 0;                              // K/V ring position over all items
+      int c = 0;                                    // items handled by this CTA
+      int last_kv = -1;                             // ring position of the last K/V issued
+      for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++c) {
+        const Item it = decode(p, x);
+        const int qb = c % QB;
+        if (!(ok = mbar_wait(q_empty + qb, ((c / QB) & 1) ^ 1, epoch, 0))) break;
+        mbar_expect_tx(q_full + qb, it.n_qt * K::TILE);
+        for (int X = 0; X < it.n_qt; ++X) {
+          uint8_t *dst = sQ + (qb * 2 + X) * K::TILE;
+          tma_load_5d(dst, &tq0, q_full + qb, 0, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
+          if (K::C1) tma_load_5d(dst + K::T0, &tq1, q_full + qb, 64, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
+        }
+        for (int j = 0; j < n_kv; ++j, ++kv) {
+          const int st = kv % NS;
+          const uint32_t ph = (kv / NS) & 1;
+          const int key = p.kv0 + j * BLOCK_N;
+          if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 1))) break;
+          mbar_expect_tx(k_full + st, K::TILE);
+          uint8_t *dk = sK + st * K::TILE;
+          tma_load_5d(dk, &tk0, k_full + st, 0, it.h, key, it.c3, it.c4);
+          if (K::C1) tma_load_5d(dk + K::T0, &tk1, k_full + st, 64, it.h, key, it.c3, it.c4);
+          if (!(ok = mbar_wait(v_empty + st, ph ^ 1, epoch, 2))) break;
+          mbar_expect_tx(v_full + st, K::TILE);
+          uint8_t *dv = sV + st * K::TILE;
+          tma_load_5d(dv, &tv0, v_full + st, 0, it.h, key, it.c3, it.c4);
+          if (K::C1) tma_load_5d(dv + K::T0, &tv1, v_full + st, 64, it.h, key, it.c3, it.c4);
+          last_kv = (int)kv;
+        }
       }
       if (!ok) {
-        *reinterpret_cast<volatile int *>(abort_flag) = 1;
-        // drain: wait (bounded, ignoring the abort epoch) for the last loads issued
+        // drain (bounded, ignoring the abort epoch): the last load issued into every slot
         const unsigned long long t0 = globaltimer();
-        for (int i = (issued > 2 * NS ? issued - 2 * NS : 0); i < issued; ++i) {
-          const int j = i >> 1;
-          uint64_t *bar = (i & 1) ? v_full + (j % NS) : k_full + (j % NS);
-          const uint32_t ph = (j / NS) & 1;
-          while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < WAIT_NS) {
+        for (int i = (last_kv - NS + 1 > 0 ? last_kv - NS + 1 : 0); i <= last_kv; ++i) {
+          const uint32_t ph = (i / NS) & 1;
+          while (!mbar_try_wait(k_full + i % NS, ph) && globaltimer() - t0 < WAIT_NS) {
+          }
+          while (!mbar_try_wait(v_full + i % NS, ph) && globaltimer() - t0 < WAIT_NS) {
           }
         }
-        while (!mbar_try_wait(q_full, 0) && globaltimer() - t0 < WAIT_NS) {
+        for (int i = (c - QB + 1 > 0 ? c - QB + 1 : 0); i <= c && i >= 0; ++i) {
+          while (!mbar_try_wait(q_full + i % QB, (i / QB) & 1) && globaltimer() - t0 < WAIT_NS) {
+          }
         }
       }
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ================= MMA issuer =================
-    if (lane == 0 && n_kv > 0) {
+    } else if (warp == 9 && lane == 0 && n_kv > 0) {
+      // ================= MMA issuer =================
       constexpr uint32_t IDS = idesc_bf16(BLOCK_M, BLOCK_N, 0, 0);
       constexpr uint32_t IDP0 = idesc_bf16(BLOCK_M, K::C0, 0, 1);
       constexpr uint32_t IDP1 = idesc_bf16(BLOCK_M, K::C1 ? K::C1 : 16, 0, 1);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      auto issue_s = [&](int X, int st) {
-        const uint32_t d = tmem + X * 128;
-        const uint32_t qa = aQ + X * K::TILE, ka = aK + st * K::TILE;
+      bool ok = true;
+      uint32_t kv = 0, pc[2] = {0, 0}, oc[2] = {0, 0};
+      int c = 0;
+      for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++c) {
+        const Item it = decode(p, x);
+        const int qb = c % QB;
+        auto issue_s = [&](int X, int st) {
+          const uint32_t d = tmem + X * 128;
+          const uint32_t qa = aQ + (qb * 2 + X) * K::TILE, ka = aK + st * K::TILE;
 #pragma unroll
-        for (int kk = 0; kk < K::C0 / 16; ++kk)
-          mma_ss(d, sdesc(qa + kk * 32, 16, 8 * K::SW0, layout_of(K::SW0)),
-                 sdesc(ka + kk * 32, 16, 8 * K::SW0, layout_of(K::SW0)), IDS, kk > 0);
-        if (K::C1) {
+          for (int kk = 0; kk < K::C0 / 16; ++kk)
+            mma_ss(d, sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(qa + kk * 32),
+                   sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(ka + kk * 32), IDS, kk > 0);
+          if (K::C1) {
 #pragma unroll
-          for (int kk = 0; kk < (K::C1 ? K::C1 : 16) / 16; ++kk)
-            mma_ss(d, sdesc(qa + K::T0 + kk * 32, 16, 8 * K::SW1, layout_of(K::SW1)),
-                   sdesc(ka + K::T0 + kk * 32, 16, 8 * K::SW1, layout_of(K::SW1)), IDS, 1);
-        }
-      };
-      auto issue_pv = [&](int X, int st, bool acc) {
-        const uint32_t d = tmem + 256 + X * 128;
-        const uint32_t pa = tmem + X * 128;  // P (bf16 pairs) over the S columns
-        const uint32_t va = aV + st * K::TILE;
+            for (int kk = 0; kk < (K::C1 ? K::C1 : 16) / 16; ++kk)
+              mma_ss(d, sdesc_c<16, 8 * K::SW1, layout_of(K::SW1)>(qa + K::T0 + kk * 32),
+                     sdesc_c<16, 8 * K::SW1, layout_of(K::SW1)>(ka + K::T0 + kk * 32), IDS, 1);
+          }
+        };
+        auto issue_pv = [&](int X, int st, bool acc) {
+          const uint32_t d = tmem + 256 + X * 128;
+          const uint32_t pa = tmem + X * 128;     // P (bf16 pairs) over the S columns
+          const uint32_t va = aV + st * K::TILE;
 #pragma unroll
-        for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
-          mma_ts(d, pa + kk * 8, sdesc(va + kk * 16 * K::SW0, K::T0, 8 * K::SW0, layout_of(K::SW0)), IDP0,
-                 (acc || kk > 0) ? 1u : 0u);
-          if (K::C1)
-            mma_ts(d + K::C0, pa + kk * 8,
-                   sdesc(va + K::T0 + kk * 16 * K::SW1, K::T1, 8 * K::SW1, layout_of(K::SW1)), IDP1,
+          for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
+            mma_ts(d, pa + kk * 8, sdesc_c<K::T0, 8 * K::SW0, layout_of(K::SW0)>(va + kk * 16 * K::SW0), IDP0,
                    (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(q_full, 0, epoch, 2) && mbar_wait(k_full, 0, epoch, 3);
-      if (ok) {
+            if (K::C1)
+              mma_ts(d + K::C0, pa + kk * 8,
+                     sdesc_c<(K::T1 ? K::T1 : 16), 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(
+                         va + K::T0 + kk * 16 * K::SW1),
+                     IDP1, (acc || kk > 0) ? 1u : 0u);
+          }
+        };
+        if (!(ok = mbar_wait(q_full + qb, (c / QB) & 1, epoch, 3))) break;
+        if (!(ok = mbar_wait(k_full + kv % NS, (kv / NS) & 1, epoch, 4))) break;
         tc_fence_after();
-        issue_s(0, 0);
+        issue_s(0, kv % NS);
         tc_commit(s_full + 0);
-        if (n_qt == 2) {
-          issue_s(1, 0);
+        if (it.n_qt == 2) {
+          issue_s(1, kv % NS);
           tc_commit(s_full + 1);
         }
-        tc_commit(k_empty + 0);
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j % NS;
-        const uint32_t ph = (j / NS) & 1;
-        const bool more = j + 1 < n_kv;
-        const int st1 = (j + 1) % NS;
-        const uint32_t ph1 = ((j + 1) / NS) & 1;
-        if (!(ok = mbar_wait(v_full + st, ph, epoch, 4))) break;
-        if (!(ok = mbar_wait(p_full + 0, j & 1, epoch, 5))) break;
-        tc_fence_after();
-        issue_pv(0, st, j > 0);
-        if (more) {
-          if (!(ok = mbar_wait(k_full + st1, ph1, epoch, 6))) break;
+        if (n_kv == 1) tc_commit(q_empty + qb);
+        tc_commit(k_empty + kv % NS);
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const uint32_t g0 = kv + j, g1 = kv + j + 1;
+          const int st = g0 % NS, st1 = g1 % NS;
+          const bool more = j + 1 < n_kv;
+          if (!(ok = mbar_wait(v_full + st, (g0 / NS) & 1, epoch, 5))) break;
+          if (!(ok = mbar_wait(p_full + 0, pc[0] & 1, epoch, 6))) break;
+          ++pc[0];
+          if (j == 0 && !(ok = mbar_wait(o_empty + 0, (oc[0] & 1) ^ 1, epoch, 7))) break;
           tc_fence_after();
-          issue_s(0, st1);
-          tc_commit(s_full + 0);
-        }
-        if (n_qt == 2) {
-          if (!(ok = mbar_wait(p_full + 1, j & 1, epoch, 7))) break;
-          tc_fence_after();
-          issue_pv(1, st, j > 0);
+          issue_pv(0, st, j > 0);
           if (more) {
-            issue_s(1, st1);
-            tc_commit(s_full + 1);
+            if (!(ok = mbar_wait(k_full + st1, (g1 / NS) & 1, epoch, 8))) break;
+            tc_fence_after();
+            issue_s(0, st1);
+            tc_commit(s_full + 0);
           }
+          if (it.n_qt == 2) {
+            if (!(ok = mbar_wait(p_full + 1, pc[1] & 1, epoch, 9))) break;
+            ++pc[1];
+            if (j == 0 && !(ok = mbar_wait(o_empty + 1, (oc[1] & 1) ^ 1, epoch, 10))) break;
+            tc_fence_after();
+            issue_pv(1, st, j > 0);
+            if (more) {
+              issue_s(1, st1);
+              tc_commit(s_full + 1);
+            }
+          }
+          if (more) {
+            if (j + 2 == n_kv) tc_commit(q_empty + qb);   // last S of this item issued
+            tc_commit(k_empty + st1);
+          }
+          tc_commit(v_empty + st);
         }
-        if (more) tc_commit(k_empty + st1);
-        tc_commit(v_empty + st);
-      }
-      if (ok) {
+        if (!ok) break;
         tc_commit(o_full + 0);
-        if (n_qt == 2) tc_commit(o_full + 1);
-      } else {
-        *reinterpret_cast<volatile int *>(abort_flag) = 1;
+        ++oc[0];
+        if (it.n_qt == 2) {
+          tc_commit(o_full + 1);
+          ++oc[1];
+        }
+        kv += n_kv;
       }
       // every MMA issued by this thread completes before TMEM is released
       tc_commit(mma_done);
@@ -438,17 +526,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else {
     // ================= softmax warpgroups =================
+    setmaxnreg_inc();
     const int X = warp >> 2;                   // tile
     const int r = ((warp & 3) << 5) + lane;    // row in tile == TMEM lane
-    const int qrow = q0 + X * BLOCK_M + r;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + X * 128;
     const uint32_t tO = tmem + lane_off + 256 + X * 128;
-    float m = -INFINITY, l = 0.f;
+    const float sl2 = p.scale_log2;
+    uint32_t sc = 0, oc = 0;                   // s_full waits, o_full waits of this tile
     bool ok = true;
-    if (X < n_qt && n_kv > 0) {
-      for (int j = 0; j < n_kv; ++j) {
-        if (!(ok = mbar_wait(s_full + X, j & 1, epoch, 8 + X))) break;
+    for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
+      const Item it = decode(p, x);
+      if (X >= it.n_qt) continue;
+      const int qrow = it.q0 + X * BLOCK_M + r;
+      const bool valid = qrow < g.S;
+      const long long off = g.frame(it.b, it.t) + g.token(valid ? qrow : 0) + (long long)it.h * D;
+      const long long lse_idx = (((long long)it.b * g.T + it.t) * g.H + it.h) * g.S + qrow;
+      if (n_kv == 0) {
+        // empty key range: o = 0, lse = -inf
+        if (valid) {
+          for (int d = 0; d < D; ++d) {
+            if (p.o_f32) static_cast<float *>(p.o)[off + d] = 0.f;
+            else static_cast<uint16_t *>(p.o)[off + d] = 0;
+          }
+          if (p.lse) p.lse[lse_idx] = -INFINITY;
+        }
+        continue;
+      }
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_kv; ++j, ++sc) {
+        if (!(ok = mbar_wait(s_full + X, sc & 1, epoch, 11 + X))) break;
         tc_fence_after();
         uint32_t sr[BLOCK_N];
 #pragma unroll
@@ -460,25 +567,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < BLOCK_N; ++c)
             if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mxp[8];
+        float mxp[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mxp[e] = __uint_as_float(sr[e]);
+        for (int e = 0; e < 4; ++e) mxp[e] = __uint_as_float(sr[e]);
 #pragma unroll
-        for (int c = 8; c < BLOCK_N; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], __uint_as_float(sr[c]));
-        float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
-        mx *= p.scale_log2;
+        for (int c = 4; c < BLOCK_N; c += 8) {
+          mxp[0] = fmax3(mxp[0], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+          mxp[1] = fmax3(mxp[1], __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+          if (c + 4 < BLOCK_N) {
+            mxp[2] = fmax3(mxp[2], __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+            mxp[3] = fmax3(mxp[3], __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+          }
+        }
+        const float mx = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]), mxp[3]) * sl2;
         if (j == 0) {
           m = mx;
         } else {
           const bool need = mx > m + 8.0f;
           if (__any_sync(0xffffffffu, need)) {
-            const float corr = need ? exp2f(m - mx) : 1.0f;
+            const float corr = need ? ex2_mufu(m - mx) : 1.0f;
             if (need) {
               l *= corr;
               m = mx;
             }
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < K::DP / 16; ++c) {
               uint32_t ov[16];
               TMEM_LD16(tO + c * 16, ov);
@@ -490,82 +602,72 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_wait_st();
           }
         }
-        float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float2 scale2 = make_float2(sl2, sl2), negm = make_float2(-m, -m);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c0 = 0; c0 < BLOCK_N; c0 += 32) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const float x0 = fmaf(__uint_as_float(sr[c0 + c]), p.scale_log2, -m);
-            const float x1 = fmaf(__uint_as_float(sr[c0 + c + 1]), p.scale_log2, -m);
-            float e0, e1;
+            const float2 xx = ffma2(make_float2(__uint_as_float(sr[c0 + c]), __uint_as_float(sr[c0 + c + 1])),
+                                    scale2, negm);
+            float2 e;
             if (((c >> 1) & 7) < kPolyPairs) {
-              e0 = ex2_poly(x0);
-              e1 = ex2_poly(x1);
+              e = ex2_poly2(xx);
             } else {
-              e0 = ex2_mufu(x0);
-              e1 = ex2_mufu(x1);
+              e.x = ex2_mufu(xx.x);
+              e.y = ex2_mufu(xx.y);
             }
-            sp[(c >> 1) & 7] += e0 + e1;
-            pk[c >> 1] = st::pack_bf16x2(e0, e1);
+            acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], e);
+            pk[c >> 1] = st::pack_bf16x2(e.x, e.y);
           }
           TMEM_ST16(tS + (c0 >> 1), pk);
         }
-        l += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+        const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+        const float2 a = fadd2(a01, a23);
+        l += a.x + a.y;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + X);
       }
-      if (ok) ok = mbar_wait(o_full + X, 0, epoch, 10 + X);
-      if (ok) {
-        tc_fence_after();
-        const float inv = 1.0f / l;
-        const bool valid = qrow < g.S;
-        const long long off = g.frame(b, t) + g.token(valid ? qrow : 0) + (long long)h * D;
+      if (!ok) break;
+      if (!(ok = mbar_wait(o_full + X, oc & 1, epoch, 13 + X))) break;
+      ++oc;
+      tc_fence_after();
+      const float inv = 1.0f / l;
+#pragma unroll 1
+      for (int c = 0; c < K::DP / 16; ++c) {
+        uint32_t ov[16];
+        TMEM_LD16(tO + c * 16, ov);
+        tmem_wait_ld();
+        if (valid && c * 16 < D) {
+          if (p.o_f32) {
+            float *dst = static_cast<float *>(p.o) + off + c * 16;
 #pragma unroll
-        for (int c = 0; c < K::DP / 16; ++c) {
-          uint32_t ov[16];
-          TMEM_LD16(tO + c * 16, ov);
-          tmem_wait_ld();
-          if (valid && c * 16 < D) {
-            if (p.o_f32) {
-              float *dst = static_cast<float *>(p.o) + off + c * 16;
+            for (int e = 0; e < 16; e += 4)
+              if (c * 16 + e < D)
+                *reinterpret_cast<float4 *>(dst + e) =
+                    make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
+                                __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+          } else {
+            uint16_t *dst = static_cast<uint16_t *>(p.o) + off + c * 16;
 #pragma unroll
-              for (int e = 0; e < 16; e += 4)
-                if (c * 16 + e < D)
-                  *reinterpret_cast<float4 *>(dst + e) =
-                      make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
-                                  __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
-            } else {
-              uint16_t *dst = static_cast<uint16_t *>(p.o) + off + c * 16;
-#pragma unroll
-              for (int e = 0; e < 16; e += 8)
-                if (c * 16 + e < D) {
-                  uint4 w;
-                  w.x = st::pack_bf16x2(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv);
-                  w.y = st::pack_bf16x2(__uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
-                  w.z = st::pack_bf16x2(__uint_as_float(ov[e + 4]) * inv, __uint_as_float(ov[e + 5]) * inv);
-                  w.w = st::pack_bf16x2(__uint_as_float(ov[e + 6]) * inv, __uint_as_float(ov[e + 7]) * inv);
-                  *reinterpret_cast<uint4 *>(dst + e) = w;
-                }
-            }
+            for (int e = 0; e < 16; e += 8)
+              if (c * 16 + e < D) {
+                uint4 w;
+                w.x = st::pack_bf16x2(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv);
+                w.y = st::pack_bf16x2(__uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+                w.z = st::pack_bf16x2(__uint_as_float(ov[e + 4]) * inv, __uint_as_float(ov[e + 5]) * inv);
+                w.w = st::pack_bf16x2(__uint_as_float(ov[e + 6]) * inv, __uint_as_float(ov[e + 7]) * inv);
+                *reinterpret_cast<uint4 *>(dst + e) = w;
+              }
           }
         }
-        if (valid && p.lse)
-          p.lse[(((long long)b * g.T + t) * g.H + h) * g.S + qrow] = (m + log2f(l)) * 0.6931471805599453f;
-      } else {
-        *reinterpret_cast<volatile int *>(abort_flag) = 1;
       }
-    } else if (X < n_qt && n_kv == 0) {
-      // empty key range: o = 0, lse = -inf
-      if (qrow < g.S) {
-        const long long off = g.frame(b, t) + g.token(qrow) + (long long)h * D;
-        for (int d = 0; d < D; ++d) {
-          if (p.o_f32) static_cast<float *>(p.o)[off + d] = 0.f;
-          else static_cast<uint16_t *>(p.o)[off + d] = 0;
-        }
-        if (p.lse) p.lse[(((long long)b * g.T + t) * g.H + h) * g.S + qrow] = -INFINITY;
-      }
+      tc_fence_before();
+      mbar_arrive(o_empty + X);                 // O of this tile may be overwritten
+      if (valid && p.lse) p.lse[lse_idx] = (m + log2f(l)) * 0.6931471805599453f;
     }
   }
 
@@ -675,13 +777,14 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   p.lse = lse;
   p.o_f32 = o_f32;
   p.epoch = g_epoch.fetch_add(1) + 1;
-  const long long ctas = (long long)p.q_blocks * g.H * g.B * p.n_frames;
-  if (ctas <= 0) return ST_OK;
-  if (ctas > 0x7fffffffLL) return ST_ERR_SHAPE;
+  const long long items = (long long)p.q_blocks * g.H * g.B * p.n_frames;
+  if (items <= 0) return ST_OK;
+  if (items > 0x7fffffffLL) return ST_ERR_SHAPE;
+  const int ctas = int(items < st::num_sms() ? items : st::num_sms());  // persistent: one CTA per SM
   auto kern = attn_fwd_sm100<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM) != cudaSuccess)
     return ST_ERR_CUDA;
-  kern<<<int(ctas), NUM_THREADS, K::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
+  kern<<<ctas, NUM_THREADS, K::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
   return st::launch_status();
 }
 
