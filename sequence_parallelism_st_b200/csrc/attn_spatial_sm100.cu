@@ -55,16 +55,24 @@ template <int D> struct Cfg {
   static constexpr int C0 = D >= 64 ? 64 : 32;
   static constexpr int R1 = D > 64 ? D - 64 : 0;
   static constexpr int C1 = R1 == 0 ? 0 : (R1 <= 16 ? 16 : (R1 <= 32 ? 32 : 64));
-  static constexpr int DP = C0 + C1;                   // padded head dim
+  static constexpr int DP = C0 + C1;                   // padded head dim of Q and K
   static constexpr int SW0 = C0 * 2, SW1 = C1 * 2;     // row bytes = swizzle span
   static constexpr int T0 = BLOCK_M * SW0, T1 = BLOCK_M * SW1;
-  static constexpr int TILE = T0 + T1;                 // bytes of one Q/K/V tile
+  static constexpr int TILE = T0 + T1;                 // bytes of one Q or K tile
+  // V is stored as DPV / VW column atoms of VW elements (MN-major for PV), so
+  // that O += P V is one instruction with N = DPV per 16 keys.
+  static constexpr int VW = (D == 72 || D == 80) ? 16 : ((D == 96 || D == 32) ? 32 : 64);
+  static constexpr int DPV = ((D + VW - 1) / VW) * VW; // padded head dim of V and O
+  static constexpr int VA = DPV / VW;                  // atoms
+  static constexpr int VSW = VW * 2;                   // atom row bytes = swizzle span
+  static constexpr int VAT = BLOCK_N * VSW;            // bytes of one atom region
+  static constexpr int VTILE = VA * VAT;               // bytes of one V tile
   static constexpr int BUDGET = 204800;
-  static constexpr int QB = (4 * TILE + 4 * TILE <= BUDGET) ? 2 : 1;  // Q double buffer if 2 KV stages fit
-  static constexpr int NS_RAW = (BUDGET - 2 * QB * TILE) / (2 * TILE);
+  static constexpr int QB = (4 * TILE + 2 * (TILE + VTILE) <= BUDGET) ? 2 : 1;  // Q double buffer if 2 stages fit
+  static constexpr int NS_RAW = (BUDGET - 2 * QB * TILE) / (TILE + VTILE);
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;   // K/V ring depth
-  static constexpr int SMEM = 1024 + 2 * QB * TILE + 2 * NS * TILE + 512;
-  static_assert(DP <= 128, "head dim too large");
+  static constexpr int SMEM = 1024 + 2 * QB * TILE + NS * (TILE + VTILE) + 512;
+  static_assert(DP <= 128 && DPV <= 128, "head dim too large");
   static_assert(NS >= 2, "ring too shallow");
 };
 
@@ -76,22 +84,16 @@ __device__ __forceinline__ float ex2_mufu(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 8.  Range reduction x = j + f with j the
-// nearest integer (adding 1.5 * 2^23 leaves j in the low mantissa bits) and
-// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients were
-// fitted for this kernel by a Remez exchange on relative error over
-// [-1/2, 1/2] (max relative error 7.5e-5, far below the bf16 rounding of P);
-// 2^j is added into the exponent field.  x is clamped at -125 so the result
-// stays a normal number (masked scores give 2^-125, i.e. 0 for all purposes).
+// 2^x on the FMA pipe (see ex2_poly2 below), for x <= 8: range reduction
+// x = j + f with j the nearest integer (adding 1.5 * 2^23 leaves j in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
+// coefficients were fitted for this kernel by a Remez exchange on relative
+// error over [-1/2, 1/2] (max relative error 7.5e-5, far below the bf16
+// rounding of P); 2^j is added into the exponent field.  x is clamped at -125
+// so the result stays a normal number (masked scores give 2^-125, i.e. 0 for
+// all purposes).
 constexpr float kP0 = 0.9999280571937561f, kP1 = 0.6932609677314758f;
 constexpr float kP2 = 0.2426111251115799f, kP3 = 0.0551716685295105f;
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(kP3, f, kP2), f, kP1), f, kP0);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
 
 // Of every 8 consecutive score pairs, this many take ex2_poly and the rest the
 // MUFU, so the two pipes share the exponentials of the softmax.
@@ -128,19 +130,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase of the given parity to complete.
+// try_wait that lets the hardware suspend the thread until the phase
+// completes or about `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of the given parity to complete.  The thread
+// sleeps in the barrier (woken when the phase completes); the wall clock and
+// the abort epoch are only consulted after a sleep of ~0.1 ms that ended
+// without the phase, so a normal wait costs no global memory traffic.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t epoch, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0) {
-      if (*reinterpret_cast<volatile unsigned int *>(&g_attn_abort_epoch) == epoch) return false;
-      if (globaltimer() - t0 > WAIT_NS) {
-        atomicOr(&g_attn_error, 1u << (site & 31));
-        atomicExch(&g_attn_abort_epoch, epoch);
-        return false;
-      }
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (*reinterpret_cast<volatile unsigned int *>(&g_attn_abort_epoch) == epoch) return false;
+    if (globaltimer() - t0 > WAIT_NS) {
+      atomicOr(&g_attn_error, 1u << (site & 31));
+      atomicExch(&g_attn_abort_epoch, epoch);
+      return false;
     }
   }
 }
@@ -198,17 +215,9 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint3
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Shared-memory matrix descriptor (tcgen05 format): start, LBO, SBO in bytes,
-// layout 2 = 128B swizzle, 4 = 64B, 6 = 32B.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;                      // descriptor version for sm_100
-  d |= (uint64_t)(layout & 7u) << 61;
-  return d;
-}
+// Shared-memory matrix descriptor (tcgen05 format): start address, leading
+// and stride byte offsets (LBO, SBO), version 1 for sm_100, swizzle layout
+// 2 = 128B, 4 = 64B, 6 = 32B.
 // The same descriptor with everything but the start address fixed at compile
 // time: only one 32-bit add per MMA operand at issue time.
 template <uint32_t LBO, uint32_t SBO, uint32_t LAYOUT>
@@ -321,15 +330,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = base;                          // QB x 2 tiles
   uint8_t *sK = sQ + QB * 2 * K::TILE;         // NS tiles
-  uint8_t *sV = sK + NS * K::TILE;             // NS tiles
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + NS * K::TILE);
+  uint8_t *sV = sK + NS * K::TILE;             // NS V tiles
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + NS * K::VTILE);
   uint64_t *q_full = bars;                     // QB
   uint64_t *q_empty = q_full + QB;             // QB
   uint64_t *k_full = q_empty + QB;             // NS
-  uint64_t *k_empty = k_full + NS;             // NS
-  uint64_t *v_full = k_empty + NS;             // NS
-  uint64_t *v_empty = v_full + NS;             // NS
-  uint64_t *s_full = v_empty + NS;             // 2
+  uint64_t *kv_empty = k_full + NS;            // NS: K and V of a stage both consumed
+  uint64_t *v_full = kv_empty + NS;            // NS
+  uint64_t *s_full = v_full + NS;              // 2
   uint64_t *p_full = s_full + 2;               // 2
   uint64_t *o_full = p_full + 2;               // 2
   uint64_t *o_empty = o_full + 2;              // 2
@@ -348,9 +356,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(k_full + i, 1);
-      mbar_init(k_empty + i, 1);
+      mbar_init(kv_empty + i, 1);
       mbar_init(v_full + i, 1);
-      mbar_init(v_empty + i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
@@ -395,16 +402,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int st = kv % NS;
           const uint32_t ph = (kv / NS) & 1;
           const int key = p.kv0 + j * BLOCK_N;
-          if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 1))) break;
+          if (!(ok = mbar_wait(kv_empty + st, ph ^ 1, epoch, 1))) break;
           mbar_expect_tx(k_full + st, K::TILE);
           uint8_t *dk = sK + st * K::TILE;
           tma_load_5d(dk, &tk0, k_full + st, 0, it.h, key, it.c3, it.c4);
           if (K::C1) tma_load_5d(dk + K::T0, &tk1, k_full + st, 64, it.h, key, it.c3, it.c4);
-          if (!(ok = mbar_wait(v_empty + st, ph ^ 1, epoch, 2))) break;
-          mbar_expect_tx(v_full + st, K::TILE);
-          uint8_t *dv = sV + st * K::TILE;
-          tma_load_5d(dv, &tv0, v_full + st, 0, it.h, key, it.c3, it.c4);
-          if (K::C1) tma_load_5d(dv + K::T0, &tv1, v_full + st, 64, it.h, key, it.c3, it.c4);
+          mbar_expect_tx(v_full + st, K::VTILE);
+          uint8_t *dv = sV + st * K::VTILE;
+#pragma unroll
+          for (int a = 0; a < K::VA; ++a)
+            tma_load_5d(dv + a * K::VAT, &tv0, v_full + st, a * K::VW, it.h, key, it.c3, it.c4);
           last_kv = (int)kv;
         }
       }
@@ -426,8 +433,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == 9 && lane == 0 && n_kv > 0) {
       // ================= MMA issuer =================
       constexpr uint32_t IDS = idesc_bf16(BLOCK_M, BLOCK_N, 0, 0);
-      constexpr uint32_t IDP0 = idesc_bf16(BLOCK_M, K::C0, 0, 1);
-      constexpr uint32_t IDP1 = idesc_bf16(BLOCK_M, K::C1 ? K::C1 : 16, 0, 1);
+      constexpr uint32_t IDPV = idesc_bf16(BLOCK_M, K::DPV, 0, 1);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       bool ok = true;
       uint32_t kv = 0, pc[2] = {0, 0}, oc[2] = {0, 0};
@@ -452,16 +458,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         auto issue_pv = [&](int X, int st, bool acc) {
           const uint32_t d = tmem + 256 + X * 128;
           const uint32_t pa = tmem + X * 128;     // P (bf16 pairs) over the S columns
-          const uint32_t va = aV + st * K::TILE;
+          const uint32_t va = aV + st * K::VTILE;
 #pragma unroll
           for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
-            mma_ts(d, pa + kk * 8, sdesc_c<K::T0, 8 * K::SW0, layout_of(K::SW0)>(va + kk * 16 * K::SW0), IDP0,
+            mma_ts(d, pa + kk * 8, sdesc_c<K::VAT, 8 * K::VSW, layout_of(K::VSW)>(va + kk * 16 * K::VSW), IDPV,
                    (acc || kk > 0) ? 1u : 0u);
-            if (K::C1)
-              mma_ts(d + K::C0, pa + kk * 8,
-                     sdesc_c<(K::T1 ? K::T1 : 16), 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(
-                         va + K::T0 + kk * 16 * K::SW1),
-                     IDP1, (acc || kk > 0) ? 1u : 0u);
           }
         };
         if (!(ok = mbar_wait(q_full + qb, (c / QB) & 1, epoch, 3))) break;
@@ -474,7 +475,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_commit(s_full + 1);
         }
         if (n_kv == 1) tc_commit(q_empty + qb);
-        tc_commit(k_empty + kv % NS);
         for (int j = 0; j < n_kv && ok; ++j) {
           const uint32_t g0 = kv + j, g1 = kv + j + 1;
           const int st = g0 % NS, st1 = g1 % NS;
@@ -502,11 +502,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               tc_commit(s_full + 1);
             }
           }
-          if (more) {
-            if (j + 2 == n_kv) tc_commit(q_empty + qb);   // last S of this item issued
-            tc_commit(k_empty + st1);
-          }
-          tc_commit(v_empty + st);
+          if (more && j + 2 == n_kv) tc_commit(q_empty + qb);   // last S of this item issued
+          tc_commit(kv_empty + st);                              // K_j and V_j both consumed
         }
         if (!ok) break;
         tc_commit(o_full + 0);
@@ -591,7 +588,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               m = mx;
             }
 #pragma unroll 1
-            for (int c = 0; c < K::DP / 16; ++c) {
+            for (int c = 0; c < K::DPV / 16; ++c) {
               uint32_t ov[16];
               TMEM_LD16(tO + c * 16, ov);
               tmem_wait_ld();
@@ -637,7 +634,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const float inv = 1.0f / l;
 #pragma unroll 1
-      for (int c = 0; c < K::DP / 16; ++c) {
+      for (int c = 0; c < K::DPV / 16; ++c) {
         uint32_t ov[16];
         TMEM_LD16(tO + c * 16, ov);
         tmem_wait_ld();
@@ -761,7 +758,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   const int c1 = K::C1 ? K::C1 : 16;
   if (!make_map(&m[0], q, g, tmode, K::C0, K::SW0) || !make_map(&m[1], q, g, tmode, c1, c1 * 2) ||
       !make_map(&m[2], k, g, tmode, K::C0, K::SW0) || !make_map(&m[3], k, g, tmode, c1, c1 * 2) ||
-      !make_map(&m[4], v, g, tmode, K::C0, K::SW0) || !make_map(&m[5], v, g, tmode, c1, c1 * 2))
+      !make_map(&m[4], v, g, tmode, K::VW, K::VSW) || !make_map(&m[5], v, g, tmode, K::VW, K::VSW))
     return ST_ERR_CUDA;
   Params p;
   p.g = g;
