@@ -7,26 +7,33 @@
 // per-chunk step of ring / Torus attention (SwiftFusion summary,
 // Methodology 2).
 //
-// Design (one CTA per SM, warp-specialised, 10 warps):
-//   * A CTA owns 256 query rows of one (b, t, head) as two 128-row tiles A
-//     and B.  Q tiles stay resident in shared memory; K and V tiles of 128
-//     keys stream through an NS-deep ring of TMA loads (warp 8).
-//   * Warp 9 issues the tensor-core work from one thread: S = Q K^T into
-//     TMEM (fp32, 128 columns per tile), and O += P V with P read straight
-//     from TMEM (the "TS" form), O accumulating in TMEM.  Issue order
-//     S_A(j+1) right after PV_A(j) and S_B(j+1) right after PV_B(j) keeps the
-//     tensor pipe busy with one tile while the other tile's softmax runs.
+// Design (one persistent CTA per SM, warp-specialised, 16 warps):
+//   * A work item is 256 query rows of one (b, t, head) as two 128-row tiles
+//     A and B; CTAs walk the items with a static stride.  Q tiles stay
+//     resident in shared memory (double-buffered across items when they fit);
+//     K and V tiles of 64 keys stream through a ring of TMA loads (warp 12).
+//   * Tensor-core work runs on three issuer warps: S = Q K^T into TMEM (fp32)
+//     for tile A (warp 13) and tile B (warp 14), and O += P V for both tiles
+//     (warp 15) with P read straight from TMEM (the "TS" form).  A single
+//     thread can only issue about one tcgen05.mma per hundred cycles, so the
+//     streams are split over several warps to keep the tensor pipe fed.  S is
+//     double-buffered per tile, so S of step j+1 is ready before the softmax
+//     of step j ends; S(j+2) reuses the buffer of S(j) once PV(j) has read
+//     P(j) from it.
 //   * Warps 0-3 (tile A) and 4-7 (tile B) are the softmax warpgroups: one
-//     thread per query row (TMEM lane), 128 scores per row loaded with
-//     tcgen05.ld, row max, exp2 with the softmax scale folded in, row sum in
-//     fp32, P packed to bf16 and written back over the S columns.  The
-//     running max is only raised (and O rescaled in TMEM) when it grows by
-//     more than 2^8, so the O correction is rare.
-//   * The epilogue divides by the row sum, rounds once to bf16 (or keeps fp32
-//     partials) and writes each row, plus the natural-log LSE.
-//   * Head dims 32..128: the D axis is split into a 64-wide 128B-swizzled
-//     chunk and a remainder chunk padded to 16/32/64 (zero-filled by TMA
-//     beyond D), each with its own swizzle mode, so D = 72 costs K = 80.
+//     thread per query row (TMEM lane), 64 scores per step loaded with
+//     tcgen05.ld, row max, exp2 with the softmax scale folded in (part of the
+//     exponentials on the FMA pipe with a polynomial), row sum in fp32, P
+//     packed to bf16 and written back over the S columns.  The running max is
+//     only raised (and O rescaled in TMEM) when it grows by more than 2^8.
+//   * Warps 8-11 are the epilogue warpgroup: once the last PV of a tile is
+//     done they read O from TMEM, divide by the row sum handed over by the
+//     softmax, round once to bf16 (or keep fp32 partials), stage 32 x 16
+//     blocks in shared memory and write them with bulk tensor stores, plus the
+//     natural-log LSE.  The softmax warps go straight on to the next item.
+//   * Head dims 32..128: Q and K split D into a 64-wide 128B-swizzled chunk and
+//     a remainder chunk padded to 16/32/64 (zero-filled by TMA beyond D); V is
+//     stored as column atoms so that PV is one instruction of N = padded D.
 //   * Every wait on an mbarrier is bounded (wall clock).  A wait that runs out
 //     records its site in a device error word, raises an abort epoch that
 //     makes every other wait of the same launch give up, drains in-flight
@@ -44,12 +51,19 @@ namespace {
 __device__ unsigned int g_attn_error;        // sites of waits that ran out
 __device__ unsigned int g_attn_abort_epoch;  // launch epoch that must abort
 
-constexpr int NUM_THREADS = 384;             // 3 warpgroups
-constexpr int BLOCK_M = 128;                 // rows per tile
-constexpr int BLOCK_N = 128;                 // keys per K/V tile
+constexpr int NUM_THREADS = 512;             // 16 warps
+constexpr int BLOCK_M = 128;                 // query rows per tile
+constexpr int BLOCK_N = 64;                  // keys per K/V tile (one softmax step)
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s per wait
-constexpr int REG_SOFTMAX = 184;             // registers of the two softmax warpgroups
-constexpr int REG_OTHER = 136;                // registers of the load / MMA warpgroup
+// warp roles (warps 0-7: softmax of tiles A and B)
+constexpr int W_EPI = 8;                     // epilogue warpgroup: warps 8-11
+constexpr int W_LOAD = 12;                   // TMA producer
+constexpr int W_S0 = 13;                     // S issuer of tile A (tile B: W_S0 + 1); also allocates TMEM
+constexpr int W_PV = 15;                     // PV issuer of both tiles
+constexpr int EPI_COLS = 16;                 // O columns per staged store
+constexpr int EPI_BUF = 32 * EPI_COLS * 4;   // bytes of one staging buffer (32 rows, fp32)
+// TMEM columns: per tile two S buffers of BLOCK_N fp32 columns, then O.
+constexpr int TM_O = 256;                    // O(tile X) at TM_O + X * 128
 
 template <int D> struct Cfg {
   static constexpr int C0 = D >= 64 ? 64 : 32;
@@ -57,8 +71,10 @@ template <int D> struct Cfg {
   static constexpr int C1 = R1 == 0 ? 0 : (R1 <= 16 ? 16 : (R1 <= 32 ? 32 : 64));
   static constexpr int DP = C0 + C1;                   // padded head dim of Q and K
   static constexpr int SW0 = C0 * 2, SW1 = C1 * 2;     // row bytes = swizzle span
-  static constexpr int T0 = BLOCK_M * SW0, T1 = BLOCK_M * SW1;
-  static constexpr int TILE = T0 + T1;                 // bytes of one Q or K tile
+  static constexpr int QT0 = BLOCK_M * SW0, QT1 = BLOCK_M * SW1;
+  static constexpr int QTILE = QT0 + QT1;              // bytes of one Q tile (128 rows)
+  static constexpr int KT0 = BLOCK_N * SW0, KT1 = BLOCK_N * SW1;
+  static constexpr int KTILE = KT0 + KT1;              // bytes of one K tile (64 keys)
   // V is stored as DPV / VW column atoms of VW elements (MN-major for PV), so
   // that O += P V is one instruction with N = DPV per 16 keys.
   static constexpr int VW = (D == 72 || D == 80) ? 16 : ((D == 96 || D == 32) ? 32 : 64);
@@ -68,12 +84,15 @@ template <int D> struct Cfg {
   static constexpr int VAT = BLOCK_N * VSW;            // bytes of one atom region
   static constexpr int VTILE = VA * VAT;               // bytes of one V tile
   static constexpr int BUDGET = 204800;
-  static constexpr int QB = (4 * TILE + 2 * (TILE + VTILE) <= BUDGET) ? 2 : 1;  // Q double buffer if 2 stages fit
-  static constexpr int NS_RAW = (BUDGET - 2 * QB * TILE) / (TILE + VTILE);
-  static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;   // K/V ring depth
-  static constexpr int SMEM = 1024 + 2 * QB * TILE + NS * (TILE + VTILE) + 512;
+  static constexpr int QB = (4 * QTILE + 4 * (KTILE + VTILE) <= BUDGET) ? 2 : 1;   // Q double buffer if 4 stages fit
+  static constexpr int NS_RAW = (BUDGET - 2 * QB * QTILE) / (KTILE + VTILE);
+  static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;   // K/V ring depth
+  // epilogue: two staging buffers per epilogue warp, then the row statistics (m, l) of both tiles
+  static constexpr int EPI = 4 * 2 * EPI_BUF + 2 * 2 * BLOCK_M * 4;
+  static constexpr int SMEM = 1024 + 2 * QB * QTILE + NS * (KTILE + VTILE) + EPI + 512;
+  static_assert(SMEM <= 232448, "shared memory");
   static_assert(DP <= 128 && DPV <= 128, "head dim too large");
-  static_assert(NS >= 2, "ring too shallow");
+  static_assert(NS >= 4, "ring too shallow");
 };
 
 // ---------------------------------------------------------------- exp2
@@ -171,6 +190,20 @@ __device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, u
         "r"(c2), "r"(c3), "r"(c4)
       : "memory");
 }
+
+// Tiled bulk store shared -> global (out-of-range rows and columns are dropped).
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, const void *src, int c0, int c1, int c2, int c3,
+                                             int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one committed bulk store may still be reading its shared memory
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -286,13 +319,6 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
-__device__ __forceinline__ void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
-}
-__device__ __forceinline__ void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_OTHER));
-}
-
 // Work item -> (q block, head, frame); q block fastest so that the CTAs that
 // run together share K/V tiles in L2.
 struct Item {
@@ -323,26 +349,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
                    const __grid_constant__ CUtensorMap tk0, const __grid_constant__ CUtensorMap tk1,
                    const __grid_constant__ CUtensorMap tv0, const __grid_constant__ CUtensorMap tv1,
-                   const Params p) {
+                   const __grid_constant__ CUtensorMap to, const Params p) {
   using K = Cfg<D>;
   constexpr int NS = K::NS, QB = K::QB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = base;                          // QB x 2 tiles
-  uint8_t *sK = sQ + QB * 2 * K::TILE;         // NS tiles
-  uint8_t *sV = sK + NS * K::TILE;             // NS V tiles
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sV + NS * K::VTILE);
+  uint8_t *sQ = base;                          // QB x 2 Q tiles
+  uint8_t *sK = sQ + QB * 2 * K::QTILE;        // NS K tiles
+  uint8_t *sV = sK + NS * K::KTILE;            // NS V tiles
+  uint8_t *sEpi = sV + NS * K::VTILE;          // 4 warps x 2 staging buffers
+  float *sStat = reinterpret_cast<float *>(sEpi + 4 * 2 * EPI_BUF);   // [tile][m | l][row]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + K::EPI);
   uint64_t *q_full = bars;                     // QB
-  uint64_t *q_empty = q_full + QB;             // QB
+  uint64_t *q_empty = q_full + QB;             // QB, 2 arrivals (the two S issuers)
   uint64_t *k_full = q_empty + QB;             // NS
-  uint64_t *kv_empty = k_full + NS;            // NS: K and V of a stage both consumed
-  uint64_t *v_full = kv_empty + NS;            // NS
-  uint64_t *s_full = v_full + NS;              // 2
-  uint64_t *p_full = s_full + 2;               // 2
-  uint64_t *o_full = p_full + 2;               // 2
-  uint64_t *o_empty = o_full + 2;              // 2
-  uint64_t *mma_done = o_empty + 2;            // 1
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+  uint64_t *k_empty = k_full + NS;             // NS, 2 arrivals (the two S issuers)
+  uint64_t *v_full = k_empty + NS;             // NS
+  uint64_t *v_empty = v_full + NS;             // NS
+  // Per (tile X, S buffer b) at index 2X + b.  With two buffers one side can
+  // run a step ahead of the other; per-buffer barriers keep every parity wait
+  // within one phase.
+  uint64_t *s_full = v_empty + NS;             // 4
+  uint64_t *p_full = s_full + 4;               // 4, 128 arrivals (softmax threads)
+  uint64_t *pv_done = p_full + 4;              // 4
+  uint64_t *o_full = pv_done + 4;              // 2
+  uint64_t *o_empty = o_full + 2;              // 2, 128 arrivals
+  uint64_t *mma_done = o_empty + 2;            // 4, one per issuer
+  uint64_t *stat_full = mma_done + 4;          // 2, 128 arrivals (softmax threads)
+  uint64_t *stat_empty = stat_full + 2;        // 2, 128 arrivals (epilogue threads)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(stat_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const st::Geom &g = p.g;
@@ -352,23 +387,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < QB; ++i) {
       mbar_init(q_full + i, 1);
-      mbar_init(q_empty + i, 1);
+      mbar_init(q_empty + i, 2);
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(k_full + i, 1);
-      mbar_init(kv_empty + i, 1);
+      mbar_init(k_empty + i, 2);
       mbar_init(v_full + i, 1);
+      mbar_init(v_empty + i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(p_full + i, BLOCK_M);
+      mbar_init(pv_done + i, 1);
+      mbar_init(mma_done + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(o_full + i, 1);
       mbar_init(o_empty + i, BLOCK_M);
+      mbar_init(stat_full + i, BLOCK_M);
+      mbar_init(stat_empty + i, BLOCK_M);
     }
-    mbar_init(mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 9) {
+  if (warp == W_S0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(512)
                  : "memory");
@@ -380,9 +421,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t epoch = p.epoch;
 
-  if (warp >= 8) {
-    setmaxnreg_dec();
-    if (warp == 8 && lane == 0 && n_kv > 0) {
+  if (warp == W_LOAD) {
+    if (lane == 0 && n_kv > 0) {
       // ================= TMA producer =================
       bool ok = true;
       uint32_t kv = 0;                              // K/V ring position over all items
@@ -392,21 +432,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const Item it = decode(p, x);
         const int qb = c % QB;
         if (!(ok = mbar_wait(q_empty + qb, ((c / QB) & 1) ^ 1, epoch, 0))) break;
-        mbar_expect_tx(q_full + qb, it.n_qt * K::TILE);
+        mbar_expect_tx(q_full + qb, it.n_qt * K::QTILE);
         for (int X = 0; X < it.n_qt; ++X) {
-          uint8_t *dst = sQ + (qb * 2 + X) * K::TILE;
+          uint8_t *dst = sQ + (qb * 2 + X) * K::QTILE;
           tma_load_5d(dst, &tq0, q_full + qb, 0, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
-          if (K::C1) tma_load_5d(dst + K::T0, &tq1, q_full + qb, 64, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
+          if (K::C1) tma_load_5d(dst + K::QT0, &tq1, q_full + qb, 64, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
         }
         for (int j = 0; j < n_kv; ++j, ++kv) {
           const int st = kv % NS;
           const uint32_t ph = (kv / NS) & 1;
           const int key = p.kv0 + j * BLOCK_N;
-          if (!(ok = mbar_wait(kv_empty + st, ph ^ 1, epoch, 1))) break;
-          mbar_expect_tx(k_full + st, K::TILE);
-          uint8_t *dk = sK + st * K::TILE;
+          if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 1))) break;
+          mbar_expect_tx(k_full + st, K::KTILE);
+          uint8_t *dk = sK + st * K::KTILE;
           tma_load_5d(dk, &tk0, k_full + st, 0, it.h, key, it.c3, it.c4);
-          if (K::C1) tma_load_5d(dk + K::T0, &tk1, k_full + st, 64, it.h, key, it.c3, it.c4);
+          if (K::C1) tma_load_5d(dk + K::KT0, &tk1, k_full + st, 64, it.h, key, it.c3, it.c4);
+          if (!(ok = mbar_wait(v_empty + st, ph ^ 1, epoch, 2))) break;
           mbar_expect_tx(v_full + st, K::VTILE);
           uint8_t *dv = sV + st * K::VTILE;
 #pragma unroll
@@ -430,133 +471,127 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-    } else if (warp == 9 && lane == 0 && n_kv > 0) {
-      // ================= MMA issuer =================
-      constexpr uint32_t IDS = idesc_bf16(BLOCK_M, BLOCK_N, 0, 0);
-      constexpr uint32_t IDPV = idesc_bf16(BLOCK_M, K::DPV, 0, 1);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = true;
-      uint32_t kv = 0, pc[2] = {0, 0}, oc[2] = {0, 0};
-      int c = 0;
-      for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++c) {
-        const Item it = decode(p, x);
-        const int qb = c % QB;
-        auto issue_s = [&](int X, int st) {
-          const uint32_t d = tmem + X * 128;
-          const uint32_t qa = aQ + (qb * 2 + X) * K::TILE, ka = aK + st * K::TILE;
-#pragma unroll
-          for (int kk = 0; kk < K::C0 / 16; ++kk)
-            mma_ss(d, sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(qa + kk * 32),
-                   sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(ka + kk * 32), IDS, kk > 0);
-          if (K::C1) {
-#pragma unroll
-            for (int kk = 0; kk < (K::C1 ? K::C1 : 16) / 16; ++kk)
-              mma_ss(d, sdesc_c<16, 8 * K::SW1, layout_of(K::SW1)>(qa + K::T0 + kk * 32),
-                     sdesc_c<16, 8 * K::SW1, layout_of(K::SW1)>(ka + K::T0 + kk * 32), IDS, 1);
-          }
-        };
-        auto issue_pv = [&](int X, int st, bool acc) {
-          const uint32_t d = tmem + 256 + X * 128;
-          const uint32_t pa = tmem + X * 128;     // P (bf16 pairs) over the S columns
-          const uint32_t va = aV + st * K::VTILE;
-#pragma unroll
-          for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
-            mma_ts(d, pa + kk * 8, sdesc_c<K::VAT, 8 * K::VSW, layout_of(K::VSW)>(va + kk * 16 * K::VSW), IDPV,
-                   (acc || kk > 0) ? 1u : 0u);
-          }
-        };
-        if (!(ok = mbar_wait(q_full + qb, (c / QB) & 1, epoch, 3))) break;
-        if (!(ok = mbar_wait(k_full + kv % NS, (kv / NS) & 1, epoch, 4))) break;
-        tc_fence_after();
-        issue_s(0, kv % NS);
-        tc_commit(s_full + 0);
-        if (it.n_qt == 2) {
-          issue_s(1, kv % NS);
-          tc_commit(s_full + 1);
-        }
-        if (n_kv == 1) tc_commit(q_empty + qb);
-        for (int j = 0; j < n_kv && ok; ++j) {
-          const uint32_t g0 = kv + j, g1 = kv + j + 1;
-          const int st = g0 % NS, st1 = g1 % NS;
-          const bool more = j + 1 < n_kv;
-          if (!(ok = mbar_wait(v_full + st, (g0 / NS) & 1, epoch, 5))) break;
-          if (!(ok = mbar_wait(p_full + 0, pc[0] & 1, epoch, 6))) break;
-          ++pc[0];
-          if (j == 0 && !(ok = mbar_wait(o_empty + 0, (oc[0] & 1) ^ 1, epoch, 7))) break;
-          tc_fence_after();
-          issue_pv(0, st, j > 0);
-          if (more) {
-            if (!(ok = mbar_wait(k_full + st1, (g1 / NS) & 1, epoch, 8))) break;
-            tc_fence_after();
-            issue_s(0, st1);
-            tc_commit(s_full + 0);
-          }
-          if (it.n_qt == 2) {
-            if (!(ok = mbar_wait(p_full + 1, pc[1] & 1, epoch, 9))) break;
-            ++pc[1];
-            if (j == 0 && !(ok = mbar_wait(o_empty + 1, (oc[1] & 1) ^ 1, epoch, 10))) break;
-            tc_fence_after();
-            issue_pv(1, st, j > 0);
-            if (more) {
-              issue_s(1, st1);
-              tc_commit(s_full + 1);
-            }
-          }
-          if (more && j + 2 == n_kv) tc_commit(q_empty + qb);   // last S of this item issued
-          tc_commit(kv_empty + st);                              // K_j and V_j both consumed
-        }
-        if (!ok) break;
-        tc_commit(o_full + 0);
-        ++oc[0];
-        if (it.n_qt == 2) {
-          tc_commit(o_full + 1);
-          ++oc[1];
-        }
-        kv += n_kv;
-      }
-      // every MMA issued by this thread completes before TMEM is released
-      tc_commit(mma_done);
-      const unsigned long long t0 = globaltimer();
-      while (!mbar_try_wait(mma_done, 0) && globaltimer() - t0 < WAIT_NS) {
-      }
     }
     __syncwarp();
-  } else {
+  } else if ((warp == W_S0 || warp == W_S0 + 1) && lane == 0 && n_kv > 0) {
+    // ================= S issuer of tile X: S(X, step) = Q_X K^T =================
+    const int X = warp - W_S0;
+    constexpr uint32_t IDS = idesc_bf16(BLOCK_M, BLOCK_N, 0, 0);
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
+    bool ok = true;
+    uint32_t kv = 0, step = 0;                       // K ring position, S steps of this tile
+    int c = 0;
+    for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++c) {
+      const Item it = decode(p, x);
+      const int qb = c % QB;
+      if (!(ok = mbar_wait(q_full + qb, (c / QB) & 1, epoch, 3))) break;
+      if (X >= it.n_qt) {
+        // tile absent from this item: release the shared K stages and Q in step
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const uint32_t g0 = kv + j;
+          if (!(ok = mbar_wait(k_full + g0 % NS, (g0 / NS) & 1, epoch, 4))) break;
+          mbar_arrive(k_empty + g0 % NS);
+        }
+        if (!ok) break;
+        mbar_arrive(q_empty + qb);
+        kv += n_kv;
+        continue;
+      }
+      const uint32_t qa = aQ + (qb * 2 + X) * K::QTILE;
+      for (int j = 0; j < n_kv && ok; ++j, ++step) {
+        const uint32_t g0 = kv + j;
+        const int st = g0 % NS;
+        const uint32_t b = step & 1;
+        // S(step) overwrites P(step - 2) in the same buffer: PV(step - 2) must be done
+        if (step >= 2 && !(ok = mbar_wait(pv_done + 2 * X + b, ((step - 2) >> 1) & 1, epoch, 5))) break;
+        if (!(ok = mbar_wait(k_full + st, (g0 / NS) & 1, epoch, 4))) break;
+        tc_fence_after();
+        const uint32_t d = tmem + X * 2 * BLOCK_N + b * BLOCK_N;
+        const uint32_t ka = aK + st * K::KTILE;
+#pragma unroll
+        for (int kk = 0; kk < K::C0 / 16; ++kk)
+          mma_ss(d, sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(qa + kk * 32),
+                 sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(ka + kk * 32), IDS, kk > 0);
+        if (K::C1) {
+#pragma unroll
+          for (int kk = 0; kk < (K::C1 ? K::C1 : 16) / 16; ++kk)
+            mma_ss(d, sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(qa + K::QT0 + kk * 32),
+                   sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(ka + K::KT0 + kk * 32),
+                   IDS, 1);
+        }
+        tc_commit(s_full + 2 * X + b);
+        tc_commit(k_empty + st);
+        if (j + 1 == n_kv) tc_commit(q_empty + qb);   // last S of this item issued
+      }
+      kv += n_kv;
+    }
+    // every MMA issued by this thread completes before TMEM is released
+    tc_commit(mma_done + warp - W_S0);
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(mma_done + warp - W_S0, 0) && globaltimer() - t0 < WAIT_NS) {
+    }
+  } else if (warp == W_PV && lane == 0 && n_kv > 0) {
+    // ================= PV issuer: O_X += P(X, step) V for both tiles =================
+    constexpr uint32_t IDPV = idesc_bf16(BLOCK_M, K::DPV, 0, 1);
+    const uint32_t aV = smem_u32(sV);
+    bool ok = true;
+    uint32_t kv = 0, step[2] = {0, 0}, oc[2] = {0, 0};
+    for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
+      const Item it = decode(p, x);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const uint32_t g0 = kv + j;
+        const int st = g0 % NS;
+        if (!(ok = mbar_wait(v_full + st, (g0 / NS) & 1, epoch, 6))) break;
+        const uint32_t va = aV + st * K::VTILE;
+        for (int X = 0; X < it.n_qt; ++X) {
+          const uint32_t b = step[X] & 1;
+          if (!(ok = mbar_wait(p_full + 2 * X + b, (step[X] >> 1) & 1, epoch, 7 + X))) break;
+          if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc[X] & 1) ^ 1, epoch, 9 + X))) break;
+          tc_fence_after();
+          const uint32_t d = tmem + TM_O + X * 128;
+          const uint32_t pa = tmem + X * 2 * BLOCK_N + b * BLOCK_N;   // P (bf16 pairs) over the S columns
+#pragma unroll
+          for (int kk = 0; kk < BLOCK_N / 16; ++kk)
+            mma_ts(d, pa + kk * 8, sdesc_c<K::VAT, 8 * K::VSW, layout_of(K::VSW)>(va + kk * 16 * K::VSW), IDPV,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(pv_done + 2 * X + b);
+          if (j + 1 == n_kv) {
+            tc_commit(o_full + X);
+            ++oc[X];
+          }
+          ++step[X];
+        }
+        if (!ok) break;
+        tc_commit(v_empty + st);
+      }
+      kv += n_kv;
+    }
+    tc_commit(mma_done + 2);
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(mma_done + 2, 0) && globaltimer() - t0 < WAIT_NS) {
+    }
+  } else if (warp < 8) {
     // ================= softmax warpgroups =================
-    setmaxnreg_inc();
     const int X = warp >> 2;                   // tile
     const int r = ((warp & 3) << 5) + lane;    // row in tile == TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + X * 128;
-    const uint32_t tO = tmem + lane_off + 256 + X * 128;
+    const uint32_t tS = tmem + lane_off + X * 2 * BLOCK_N;
+    const uint32_t tO = tmem + lane_off + TM_O + X * 128;
     const float sl2 = p.scale_log2;
-    uint32_t sc = 0, oc = 0;                   // s_full waits, o_full waits of this tile
-    bool ok = true;
+    const float2 scale2 = make_float2(sl2, sl2);
+    uint32_t gs = 0, oc = 0;                   // S steps and items of this tile
+    bool ok = n_kv > 0;                        // an empty key range is written by the epilogue alone
     for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
       const Item it = decode(p, x);
       if (X >= it.n_qt) continue;
-      const int qrow = it.q0 + X * BLOCK_M + r;
-      const bool valid = qrow < g.S;
-      const long long off = g.frame(it.b, it.t) + g.token(valid ? qrow : 0) + (long long)it.h * D;
-      const long long lse_idx = (((long long)it.b * g.T + it.t) * g.H + it.h) * g.S + qrow;
-      if (n_kv == 0) {
-        // empty key range: o = 0, lse = -inf
-        if (valid) {
-          for (int d = 0; d < D; ++d) {
-            if (p.o_f32) static_cast<float *>(p.o)[off + d] = 0.f;
-            else static_cast<uint16_t *>(p.o)[off + d] = 0;
-          }
-          if (p.lse) p.lse[lse_idx] = -INFINITY;
-        }
-        continue;
-      }
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_kv; ++j, ++sc) {
-        if (!(ok = mbar_wait(s_full + X, sc & 1, epoch, 11 + X))) break;
+      for (int j = 0; j < n_kv; ++j, ++gs) {
+        const uint32_t b = gs & 1;
+        if (!(ok = mbar_wait(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
         tc_fence_after();
         uint32_t sr[BLOCK_N];
 #pragma unroll
-        for (int c = 0; c < BLOCK_N / 16; ++c) TMEM_LD16(tS + c * 16, (sr + c * 16));
+        for (int c = 0; c < BLOCK_N / 16; ++c) TMEM_LD16(tS + b * BLOCK_N + c * 16, (sr + c * 16));
         tmem_wait_ld();
         const int nvalid = p.kv1 - (p.kv0 + j * BLOCK_N);
         if (nvalid < BLOCK_N) {
@@ -582,6 +617,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         } else {
           const bool need = mx > m + 8.0f;
           if (__any_sync(0xffffffffu, need)) {
+            // O holds PV up to step gs-1: wait for that PV, then rescale in TMEM
+            if (!(ok = mbar_wait(pv_done + 2 * X + ((gs - 1) & 1), ((gs - 1) >> 1) & 1, epoch, 15 + X))) break;
+            tc_fence_after();
             const float corr = need ? ex2_mufu(m - mx) : 1.0f;
             if (need) {
               l *= corr;
@@ -599,7 +637,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_wait_st();
           }
         }
-        const float2 scale2 = make_float2(sl2, sl2), negm = make_float2(-m, -m);
+        const float2 negm = make_float2(-m, -m);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                          make_float2(0.f, 0.f)};
 #pragma unroll
@@ -619,58 +657,116 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], e);
             pk[c >> 1] = st::pack_bf16x2(e.x, e.y);
           }
-          TMEM_ST16(tS + (c0 >> 1), pk);
+          TMEM_ST16(tS + b * BLOCK_N + (c0 >> 1), pk);
         }
         const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
         const float2 a = fadd2(a01, a23);
         l += a.x + a.y;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full + X);
+        mbar_arrive(p_full + 2 * X + b);
       }
       if (!ok) break;
-      if (!(ok = mbar_wait(o_full + X, oc & 1, epoch, 13 + X))) break;
+      // hand the row statistics to the epilogue warpgroup
+      if (!(ok = mbar_wait(stat_empty + X, (oc & 1) ^ 1, epoch, 13 + X))) break;
+      sStat[(X * 2 + 0) * BLOCK_M + r] = m;
+      sStat[(X * 2 + 1) * BLOCK_M + r] = l;
+      mbar_arrive(stat_full + X);
       ++oc;
-      tc_fence_after();
-      const float inv = 1.0f / l;
+    }
+  } else if (warp >= W_EPI && warp < W_EPI + 4) {
+    // ================= epilogue warpgroup =================
+    // Per tile: wait for the last PV and the row statistics, read O out of
+    // TMEM 16 columns at a time (TMEM is released after the last read),
+    // divide by the row sum, stage the 32 x 16 block of this warp in shared
+    // memory in the swizzled layout of the output tensor map, and let one
+    // lane write it with a bulk tensor store (rows past S and columns past D
+    // are dropped by the copy engine).  The LSE is written per row.
+    const int qd = warp - W_EPI;               // TMEM lane quadrant
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    uint8_t *stg = sEpi + qd * 2 * EPI_BUF;
+    uint32_t oc[2] = {0, 0}, nst = 0;          // items per tile, bulk stores issued by this warp
+    bool ok = true;
+    for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
+      const Item it = decode(p, x);
+      for (int X = 0; X < it.n_qt && ok; ++X) {
+        const int r = qd * 32 + lane;
+        const int qrow = it.q0 + X * BLOCK_M + r;
+        const bool valid = qrow < g.S;
+        const long long lse_idx = (((long long)it.b * g.T + it.t) * g.H + it.h) * g.S + qrow;
+        if (n_kv == 0) {
+          // empty key range: o = 0, lse = -inf
+          if (valid) {
+            const long long off = g.frame(it.b, it.t) + g.token(qrow) + (long long)it.h * D;
+            for (int d = 0; d < D; ++d) {
+              if (p.o_f32) static_cast<float *>(p.o)[off + d] = 0.f;
+              else static_cast<uint16_t *>(p.o)[off + d] = 0;
+            }
+            if (p.lse) p.lse[lse_idx] = -INFINITY;
+          }
+          continue;
+        }
+        if (!(ok = mbar_wait(o_full + X, oc[X] & 1, epoch, 17 + X))) break;
+        if (!(ok = mbar_wait(stat_full + X, oc[X] & 1, epoch, 19 + X))) break;
+        ++oc[X];
+        tc_fence_after();
+        const float m = sStat[(X * 2 + 0) * BLOCK_M + r];
+        const float l = sStat[(X * 2 + 1) * BLOCK_M + r];
+        mbar_arrive(stat_empty + X);
+        const float inv = 1.0f / l;
+        const uint32_t tO = tmem + lane_off + TM_O + X * 128;
+        constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;
 #pragma unroll 1
-      for (int c = 0; c < K::DPV / 16; ++c) {
-        uint32_t ov[16];
-        TMEM_LD16(tO + c * 16, ov);
-        tmem_wait_ld();
-        if (valid && c * 16 < D) {
+        for (int c = 0; c < NCH; ++c, ++nst) {
+          uint32_t ov[16];
+          TMEM_LD16(tO + c * 16, ov);
+          tmem_wait_ld();
+          if (c + 1 == NCH) {
+            tc_fence_before();
+            mbar_arrive(o_empty + X);          // O of this tile may be overwritten
+          }
+          uint8_t *buf = stg + (nst & 1) * EPI_BUF;
+          if (lane == 0) bulk_wait_read1();    // the store that used this buffer has read it
+          __syncwarp();
           if (p.o_f32) {
-            float *dst = static_cast<float *>(p.o) + off + c * 16;
+            // 64-byte rows, 64B swizzle: 16-byte chunk f of row r at f ^ ((r >> 1) & 3)
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              if (c * 16 + e < D)
-                *reinterpret_cast<float4 *>(dst + e) =
-                    make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
-                                __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+            for (int f = 0; f < 4; ++f)
+              *reinterpret_cast<float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4)) =
+                  make_float4(__uint_as_float(ov[4 * f]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
+                              __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
           } else {
-            uint16_t *dst = static_cast<uint16_t *>(p.o) + off + c * 16;
+            // 32-byte rows, 32B swizzle: 16-byte chunk f of row r at f ^ ((r >> 2) & 1)
 #pragma unroll
-            for (int e = 0; e < 16; e += 8)
-              if (c * 16 + e < D) {
-                uint4 w;
-                w.x = st::pack_bf16x2(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv);
-                w.y = st::pack_bf16x2(__uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
-                w.z = st::pack_bf16x2(__uint_as_float(ov[e + 4]) * inv, __uint_as_float(ov[e + 5]) * inv);
-                w.w = st::pack_bf16x2(__uint_as_float(ov[e + 6]) * inv, __uint_as_float(ov[e + 7]) * inv);
-                *reinterpret_cast<uint4 *>(dst + e) = w;
-              }
+            for (int f = 0; f < 2; ++f) {
+              uint4 w;
+              w.x = st::pack_bf16x2(__uint_as_float(ov[8 * f]) * inv, __uint_as_float(ov[8 * f + 1]) * inv);
+              w.y = st::pack_bf16x2(__uint_as_float(ov[8 * f + 2]) * inv, __uint_as_float(ov[8 * f + 3]) * inv);
+              w.z = st::pack_bf16x2(__uint_as_float(ov[8 * f + 4]) * inv, __uint_as_float(ov[8 * f + 5]) * inv);
+              w.w = st::pack_bf16x2(__uint_as_float(ov[8 * f + 6]) * inv, __uint_as_float(ov[8 * f + 7]) * inv);
+              *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
+            }
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            // a block wholly past the last row stores nothing, but still
+            // commits a (empty) group so the buffer accounting stays in step
+            const int row0 = it.q0 + X * BLOCK_M + qd * 32;
+            if (row0 < g.S) tma_store_5d(&to, buf, c * EPI_COLS, it.h, row0, it.c3, it.c4);
+            bulk_commit();
           }
         }
+        if (valid && p.lse) p.lse[lse_idx] = (m + log2f(l)) * 0.6931471805599453f;
       }
-      tc_fence_before();
-      mbar_arrive(o_empty + X);                 // O of this tile may be overwritten
-      if (valid && p.lse) p.lse[lse_idx] = (m + log2f(l)) * 0.6931471805599453f;
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == W_S0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
   }
@@ -718,30 +814,34 @@ CUtensorMapSwizzle swz(int bytes) {
                       : (bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
-// 5-D map over (d, h, s, frame-in-block, block) with a box of (box_d, 1, 128, 1, 1).
-bool make_map(CUtensorMap *m, const void *ptr, const st::Geom &g, int tmode, int box_d, int swizzle_bytes) {
+// 5-D map over (d, h, s, frame-in-block, block) with a box of (box_d, 1, box_rows, 1, 1);
+// elements are bf16, or fp32 when f32 is set.
+bool make_map(CUtensorMap *m, const void *ptr, const st::Geom &g, int tmode, int box_d, int swizzle_bytes,
+              int box_rows, int f32 = 0) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const cuuint64_t es_bytes = f32 ? 4 : 2;
   cuuint64_t dims[5], strides[4];
   dims[0] = (cuuint64_t)g.D;
   dims[1] = (cuuint64_t)g.H;
   dims[2] = (cuuint64_t)g.S;
-  strides[0] = (cuuint64_t)g.D * 2;
-  strides[1] = (cuuint64_t)g.ss * 2;
+  strides[0] = (cuuint64_t)g.D * es_bytes;
+  strides[1] = (cuuint64_t)g.ss * es_bytes;
   if (tmode) {
     dims[3] = (cuuint64_t)g.tblk;
     dims[4] = (cuuint64_t)g.B * (g.T / g.tblk);
-    strides[2] = (cuuint64_t)g.st * 2;
-    strides[3] = (cuuint64_t)g.stb * 2;
+    strides[2] = (cuuint64_t)g.st * es_bytes;
+    strides[3] = (cuuint64_t)g.stb * es_bytes;
   } else {
     dims[3] = (cuuint64_t)g.T;
     dims[4] = (cuuint64_t)g.B;
-    strides[2] = (cuuint64_t)g.st * 2;
-    strides[3] = (cuuint64_t)g.sb * 2;
+    strides[2] = (cuuint64_t)g.st * es_bytes;
+    strides[3] = (cuuint64_t)g.sb * es_bytes;
   }
-  cuuint32_t box[5] = {(cuuint32_t)box_d, 1, BLOCK_M, 1, 1};
+  cuuint32_t box[5] = {(cuuint32_t)box_d, 1, (cuuint32_t)box_rows, 1, 1};
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(ptr), dims, strides, box, es,
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+                  const_cast<void *>(ptr), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz(swizzle_bytes), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -754,11 +854,12 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
                          const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s) {
   using K = Cfg<D>;
   const int tmode = g.tblk != g.T ? 1 : 0;
-  CUtensorMap m[6];
+  CUtensorMap m[7];
   const int c1 = K::C1 ? K::C1 : 16;
-  if (!make_map(&m[0], q, g, tmode, K::C0, K::SW0) || !make_map(&m[1], q, g, tmode, c1, c1 * 2) ||
-      !make_map(&m[2], k, g, tmode, K::C0, K::SW0) || !make_map(&m[3], k, g, tmode, c1, c1 * 2) ||
-      !make_map(&m[4], v, g, tmode, K::VW, K::VSW) || !make_map(&m[5], v, g, tmode, K::VW, K::VSW))
+  if (!make_map(&m[0], q, g, tmode, K::C0, K::SW0, BLOCK_M) || !make_map(&m[1], q, g, tmode, c1, c1 * 2, BLOCK_M) ||
+      !make_map(&m[2], k, g, tmode, K::C0, K::SW0, BLOCK_N) || !make_map(&m[3], k, g, tmode, c1, c1 * 2, BLOCK_N) ||
+      !make_map(&m[4], v, g, tmode, K::VW, K::VSW, BLOCK_N) || !make_map(&m[5], v, g, tmode, K::VW, K::VSW, BLOCK_N) ||
+      !make_map(&m[6], o, g, tmode, EPI_COLS, EPI_COLS * (o_f32 ? 4 : 2), 32, o_f32))
     return ST_ERR_CUDA;
   Params p;
   p.g = g;
@@ -781,7 +882,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   auto kern = attn_fwd_sm100<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM) != cudaSuccess)
     return ST_ERR_CUDA;
-  kern<<<ctas, NUM_THREADS, K::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
+  kern<<<ctas, NUM_THREADS, K::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
   return st::launch_status();
 }
 
