@@ -7,16 +7,18 @@
 // per-chunk step of ring / Torus attention (SwiftFusion summary,
 // Methodology 2).
 //
-// Design (one persistent CTA per SM, warp-specialised, 16 warps):
+// Design (one persistent CTA per SM, warp-specialised, 20 warps):
 //   * A work item is 256 query rows of one (b, t, head) as two 128-row tiles
 //     A and B; CTAs walk the items with a static stride.  Q tiles stay
 //     resident in shared memory (double-buffered across items when they fit);
 //     K and V tiles of 64 keys stream through a ring of TMA loads (warp 12).
-//   * Tensor-core work runs on three issuer warps: S = Q K^T into TMEM (fp32)
-//     for tile A (warp 13) and tile B (warp 14), and O += P V for both tiles
-//     (warp 15) with P read straight from TMEM (the "TS" form).  A single
-//     thread can only issue about one tcgen05.mma per hundred cycles, so the
-//     streams are split over several warps to keep the tensor pipe fed.  S is
+//   * Tensor-core work runs on four issuer warps, one per (tile, product):
+//     S = Q K^T into TMEM (fp32) for tile A (warp 13) and tile B (warp 14),
+//     O += P V (warps 15 and 16) with P read straight from TMEM (the "TS"
+//     form).  A single thread issues about one tcgen05 operation (MMA or
+//     commit) per hundred cycles, so the streams are split over four warps to
+//     keep the tensor pipe fed.  Registers are rebalanced per warpgroup with
+//     setmaxnreg: the single-thread roles give theirs to the softmax.  S is
 //     double-buffered per tile, so S of step j+1 is ready before the softmax
 //     of step j ends; S(j+2) reuses the buffer of S(j) once PV(j) has read
 //     P(j) from it.
@@ -51,7 +53,7 @@ namespace {
 __device__ unsigned int g_attn_error;        // sites of waits that ran out
 __device__ unsigned int g_attn_abort_epoch;  // launch epoch that must abort
 
-constexpr int NUM_THREADS = 512;             // 16 warps
+constexpr int NUM_THREADS = 640;             // 20 warps = 5 warpgroups
 constexpr int BLOCK_M = 128;                 // query rows per tile
 constexpr int BLOCK_N = 64;                  // keys per K/V tile (one softmax step)
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s per wait
@@ -59,7 +61,13 @@ constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr int W_EPI = 8;                     // epilogue warpgroup: warps 8-11
 constexpr int W_LOAD = 12;                   // TMA producer
 constexpr int W_S0 = 13;                     // S issuer of tile A (tile B: W_S0 + 1); also allocates TMEM
-constexpr int W_PV = 15;                     // PV issuer of both tiles
+constexpr int W_PV0 = 15;                    // PV issuer of tile A (tile B: W_PV0 + 1); warps 17-19 idle
+// Registers per thread after the split (setmaxnreg): the launch gives every
+// thread 96 (640 x 96 = 61440); the two softmax warpgroups take 128, the
+// epilogue 112, and the issuer / loader warpgroups give back down to 56:
+// 256 x 128 + 128 x 112 + 256 x 56 = 61440.
+constexpr int REG_SOFTMAX = 128, REG_EPI = 112, REG_ISSUE = 56;
+static_assert(256 * REG_SOFTMAX + 128 * REG_EPI + 256 * REG_ISSUE <= NUM_THREADS * 96, "register split");
 constexpr int EPI_COLS = 16;                 // O columns per staged store
 constexpr int EPI_BUF = 32 * EPI_COLS * 4;   // bytes of one staging buffer (32 rows, fp32)
 // TMEM columns: per tile two S buffers of BLOCK_N fp32 columns, then O.
@@ -365,7 +373,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *k_full = q_empty + QB;             // NS
   uint64_t *k_empty = k_full + NS;             // NS, 2 arrivals (the two S issuers)
   uint64_t *v_full = k_empty + NS;             // NS
-  uint64_t *v_empty = v_full + NS;             // NS
+  uint64_t *v_empty = v_full + NS;             // NS, 2 arrivals (the two PV issuers)
   // Per (tile X, S buffer b) at index 2X + b.  With two buffers one side can
   // run a step ahead of the other; per-buffer barriers keep every parity wait
   // within one phase.
@@ -393,7 +401,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 2);
       mbar_init(v_full + i, 1);
-      mbar_init(v_empty + i, 1);
+      mbar_init(v_empty + i, 2);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(s_full + i, 1);
@@ -421,156 +429,167 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t epoch = p.epoch;
 
-  if (warp == W_LOAD) {
-    if (lane == 0 && n_kv > 0) {
-      // ================= TMA producer =================
+  if (warp >= W_LOAD) {
+    // warpgroups 3 and 4: TMA producer, MMA issuers, idle warps
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_ISSUE));
+    if (warp == W_LOAD) {
+      if (lane == 0 && n_kv > 0) {
+        // ================= TMA producer =================
+        bool ok = true;
+        uint32_t kv = 0;                              // K/V ring position over all items
+        int c = 0;                                    // items handled by this CTA
+        int last_kv = -1;                             // ring position of the last K/V issued
+        for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++c) {
+          const Item it = decode(p, x);
+          const int qb = c % QB;
+          if (!(ok = mbar_wait(q_empty + qb, ((c / QB) & 1) ^ 1, epoch, 0))) break;
+          mbar_expect_tx(q_full + qb, it.n_qt * K::QTILE);
+          for (int X = 0; X < it.n_qt; ++X) {
+            uint8_t *dst = sQ + (qb * 2 + X) * K::QTILE;
+            tma_load_5d(dst, &tq0, q_full + qb, 0, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
+            if (K::C1) tma_load_5d(dst + K::QT0, &tq1, q_full + qb, 64, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
+          }
+          for (int j = 0; j < n_kv; ++j, ++kv) {
+            const int st = kv % NS;
+            const uint32_t ph = (kv / NS) & 1;
+            const int key = p.kv0 + j * BLOCK_N;
+            if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 1))) break;
+            mbar_expect_tx(k_full + st, K::KTILE);
+            uint8_t *dk = sK + st * K::KTILE;
+            tma_load_5d(dk, &tk0, k_full + st, 0, it.h, key, it.c3, it.c4);
+            if (K::C1) tma_load_5d(dk + K::KT0, &tk1, k_full + st, 64, it.h, key, it.c3, it.c4);
+            if (!(ok = mbar_wait(v_empty + st, ph ^ 1, epoch, 2))) break;
+            mbar_expect_tx(v_full + st, K::VTILE);
+            uint8_t *dv = sV + st * K::VTILE;
+  #pragma unroll
+            for (int a = 0; a < K::VA; ++a)
+              tma_load_5d(dv + a * K::VAT, &tv0, v_full + st, a * K::VW, it.h, key, it.c3, it.c4);
+            last_kv = (int)kv;
+          }
+        }
+        if (!ok) {
+          // drain (bounded, ignoring the abort epoch): the last load issued into every slot
+          const unsigned long long t0 = globaltimer();
+          for (int i = (last_kv - NS + 1 > 0 ? last_kv - NS + 1 : 0); i <= last_kv; ++i) {
+            const uint32_t ph = (i / NS) & 1;
+            while (!mbar_try_wait(k_full + i % NS, ph) && globaltimer() - t0 < WAIT_NS) {
+            }
+            while (!mbar_try_wait(v_full + i % NS, ph) && globaltimer() - t0 < WAIT_NS) {
+            }
+          }
+          for (int i = (c - QB + 1 > 0 ? c - QB + 1 : 0); i <= c && i >= 0; ++i) {
+            while (!mbar_try_wait(q_full + i % QB, (i / QB) & 1) && globaltimer() - t0 < WAIT_NS) {
+            }
+          }
+        }
+      }
+      __syncwarp();
+    } else if ((warp == W_S0 || warp == W_S0 + 1) && lane == 0 && n_kv > 0) {
+      // ================= S issuer of tile X: S(X, step) = Q_X K^T =================
+      const int X = warp - W_S0;
+      constexpr uint32_t IDS = idesc_bf16(BLOCK_M, BLOCK_N, 0, 0);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
       bool ok = true;
-      uint32_t kv = 0;                              // K/V ring position over all items
-      int c = 0;                                    // items handled by this CTA
-      int last_kv = -1;                             // ring position of the last K/V issued
+      uint32_t kv = 0, step = 0;                       // K ring position, S steps of this tile
+      int c = 0;
       for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++c) {
         const Item it = decode(p, x);
         const int qb = c % QB;
-        if (!(ok = mbar_wait(q_empty + qb, ((c / QB) & 1) ^ 1, epoch, 0))) break;
-        mbar_expect_tx(q_full + qb, it.n_qt * K::QTILE);
-        for (int X = 0; X < it.n_qt; ++X) {
-          uint8_t *dst = sQ + (qb * 2 + X) * K::QTILE;
-          tma_load_5d(dst, &tq0, q_full + qb, 0, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
-          if (K::C1) tma_load_5d(dst + K::QT0, &tq1, q_full + qb, 64, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
-        }
-        for (int j = 0; j < n_kv; ++j, ++kv) {
-          const int st = kv % NS;
-          const uint32_t ph = (kv / NS) & 1;
-          const int key = p.kv0 + j * BLOCK_N;
-          if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 1))) break;
-          mbar_expect_tx(k_full + st, K::KTILE);
-          uint8_t *dk = sK + st * K::KTILE;
-          tma_load_5d(dk, &tk0, k_full + st, 0, it.h, key, it.c3, it.c4);
-          if (K::C1) tma_load_5d(dk + K::KT0, &tk1, k_full + st, 64, it.h, key, it.c3, it.c4);
-          if (!(ok = mbar_wait(v_empty + st, ph ^ 1, epoch, 2))) break;
-          mbar_expect_tx(v_full + st, K::VTILE);
-          uint8_t *dv = sV + st * K::VTILE;
-#pragma unroll
-          for (int a = 0; a < K::VA; ++a)
-            tma_load_5d(dv + a * K::VAT, &tv0, v_full + st, a * K::VW, it.h, key, it.c3, it.c4);
-          last_kv = (int)kv;
-        }
-      }
-      if (!ok) {
-        // drain (bounded, ignoring the abort epoch): the last load issued into every slot
-        const unsigned long long t0 = globaltimer();
-        for (int i = (last_kv - NS + 1 > 0 ? last_kv - NS + 1 : 0); i <= last_kv; ++i) {
-          const uint32_t ph = (i / NS) & 1;
-          while (!mbar_try_wait(k_full + i % NS, ph) && globaltimer() - t0 < WAIT_NS) {
+        if (!(ok = mbar_wait(q_full + qb, (c / QB) & 1, epoch, 3))) break;
+        if (X >= it.n_qt) {
+          // tile absent from this item: release the shared K stages and Q in step
+          for (int j = 0; j < n_kv && ok; ++j) {
+            const uint32_t g0 = kv + j;
+            if (!(ok = mbar_wait(k_full + g0 % NS, (g0 / NS) & 1, epoch, 4))) break;
+            mbar_arrive(k_empty + g0 % NS);
           }
-          while (!mbar_try_wait(v_full + i % NS, ph) && globaltimer() - t0 < WAIT_NS) {
-          }
+          if (!ok) break;
+          mbar_arrive(q_empty + qb);
+          kv += n_kv;
+          continue;
         }
-        for (int i = (c - QB + 1 > 0 ? c - QB + 1 : 0); i <= c && i >= 0; ++i) {
-          while (!mbar_try_wait(q_full + i % QB, (i / QB) & 1) && globaltimer() - t0 < WAIT_NS) {
-          }
-        }
-      }
-    }
-    __syncwarp();
-  } else if ((warp == W_S0 || warp == W_S0 + 1) && lane == 0 && n_kv > 0) {
-    // ================= S issuer of tile X: S(X, step) = Q_X K^T =================
-    const int X = warp - W_S0;
-    constexpr uint32_t IDS = idesc_bf16(BLOCK_M, BLOCK_N, 0, 0);
-    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
-    bool ok = true;
-    uint32_t kv = 0, step = 0;                       // K ring position, S steps of this tile
-    int c = 0;
-    for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++c) {
-      const Item it = decode(p, x);
-      const int qb = c % QB;
-      if (!(ok = mbar_wait(q_full + qb, (c / QB) & 1, epoch, 3))) break;
-      if (X >= it.n_qt) {
-        // tile absent from this item: release the shared K stages and Q in step
-        for (int j = 0; j < n_kv && ok; ++j) {
+        const uint32_t qa = aQ + (qb * 2 + X) * K::QTILE;
+        for (int j = 0; j < n_kv && ok; ++j, ++step) {
           const uint32_t g0 = kv + j;
-          if (!(ok = mbar_wait(k_full + g0 % NS, (g0 / NS) & 1, epoch, 4))) break;
-          mbar_arrive(k_empty + g0 % NS);
+          const int st = g0 % NS;
+          const uint32_t b = step & 1;
+          // S(step) overwrites P(step - 2) in the same buffer: PV(step - 2) must be done
+          if (step >= 2 && !(ok = mbar_wait(pv_done + 2 * X + b, ((step - 2) >> 1) & 1, epoch, 5))) break;
+          if (!(ok = mbar_wait(k_full + st, (g0 / NS) & 1, epoch, 4))) break;
+          tc_fence_after();
+          const uint32_t d = tmem + X * 2 * BLOCK_N + b * BLOCK_N;
+          const uint32_t ka = aK + st * K::KTILE;
+  #pragma unroll
+          for (int kk = 0; kk < K::C0 / 16; ++kk)
+            mma_ss(d, sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(qa + kk * 32),
+                   sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(ka + kk * 32), IDS, kk > 0);
+          if (K::C1) {
+  #pragma unroll
+            for (int kk = 0; kk < (K::C1 ? K::C1 : 16) / 16; ++kk)
+              mma_ss(d, sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(qa + K::QT0 + kk * 32),
+                     sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(ka + K::KT0 + kk * 32),
+                     IDS, 1);
+          }
+          tc_commit(s_full + 2 * X + b);
+          tc_commit(k_empty + st);
+          if (j + 1 == n_kv) tc_commit(q_empty + qb);   // last S of this item issued
         }
-        if (!ok) break;
-        mbar_arrive(q_empty + qb);
         kv += n_kv;
-        continue;
       }
-      const uint32_t qa = aQ + (qb * 2 + X) * K::QTILE;
-      for (int j = 0; j < n_kv && ok; ++j, ++step) {
-        const uint32_t g0 = kv + j;
-        const int st = g0 % NS;
-        const uint32_t b = step & 1;
-        // S(step) overwrites P(step - 2) in the same buffer: PV(step - 2) must be done
-        if (step >= 2 && !(ok = mbar_wait(pv_done + 2 * X + b, ((step - 2) >> 1) & 1, epoch, 5))) break;
-        if (!(ok = mbar_wait(k_full + st, (g0 / NS) & 1, epoch, 4))) break;
-        tc_fence_after();
-        const uint32_t d = tmem + X * 2 * BLOCK_N + b * BLOCK_N;
-        const uint32_t ka = aK + st * K::KTILE;
-#pragma unroll
-        for (int kk = 0; kk < K::C0 / 16; ++kk)
-          mma_ss(d, sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(qa + kk * 32),
-                 sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(ka + kk * 32), IDS, kk > 0);
-        if (K::C1) {
-#pragma unroll
-          for (int kk = 0; kk < (K::C1 ? K::C1 : 16) / 16; ++kk)
-            mma_ss(d, sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(qa + K::QT0 + kk * 32),
-                   sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(ka + K::KT0 + kk * 32),
-                   IDS, 1);
+      // every MMA issued by this thread completes before TMEM is released
+      tc_commit(mma_done + warp - W_S0);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(mma_done + warp - W_S0, 0) && globaltimer() - t0 < WAIT_NS) {
+      }
+    } else if ((warp == W_PV0 || warp == W_PV0 + 1) && lane == 0 && n_kv > 0) {
+      // ================= PV issuer of tile X: O_X += P(X, step) V =================
+      const int X = warp - W_PV0;
+      constexpr uint32_t IDPV = idesc_bf16(BLOCK_M, K::DPV, 0, 1);
+      const uint32_t aV = smem_u32(sV);
+      bool ok = true;
+      uint32_t kv = 0, step = 0, oc = 0;
+      for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
+        const Item it = decode(p, x);
+        if (X >= it.n_qt) {
+          // tile absent from this item: release the shared V stages in step
+          for (int j = 0; j < n_kv && ok; ++j) {
+            const uint32_t g0 = kv + j;
+            if (!(ok = mbar_wait(v_full + g0 % NS, (g0 / NS) & 1, epoch, 6))) break;
+            mbar_arrive(v_empty + g0 % NS);
+          }
+          kv += n_kv;
+          continue;
         }
-        tc_commit(s_full + 2 * X + b);
-        tc_commit(k_empty + st);
-        if (j + 1 == n_kv) tc_commit(q_empty + qb);   // last S of this item issued
-      }
-      kv += n_kv;
-    }
-    // every MMA issued by this thread completes before TMEM is released
-    tc_commit(mma_done + warp - W_S0);
-    const unsigned long long t0 = globaltimer();
-    while (!mbar_try_wait(mma_done + warp - W_S0, 0) && globaltimer() - t0 < WAIT_NS) {
-    }
-  } else if (warp == W_PV && lane == 0 && n_kv > 0) {
-    // ================= PV issuer: O_X += P(X, step) V for both tiles =================
-    constexpr uint32_t IDPV = idesc_bf16(BLOCK_M, K::DPV, 0, 1);
-    const uint32_t aV = smem_u32(sV);
-    bool ok = true;
-    uint32_t kv = 0, step[2] = {0, 0}, oc[2] = {0, 0};
-    for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
-      const Item it = decode(p, x);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const uint32_t g0 = kv + j;
-        const int st = g0 % NS;
-        if (!(ok = mbar_wait(v_full + st, (g0 / NS) & 1, epoch, 6))) break;
-        const uint32_t va = aV + st * K::VTILE;
-        for (int X = 0; X < it.n_qt; ++X) {
-          const uint32_t b = step[X] & 1;
-          if (!(ok = mbar_wait(p_full + 2 * X + b, (step[X] >> 1) & 1, epoch, 7 + X))) break;
-          if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc[X] & 1) ^ 1, epoch, 9 + X))) break;
+        for (int j = 0; j < n_kv && ok; ++j, ++step) {
+          const uint32_t g0 = kv + j;
+          const int st = g0 % NS;
+          const uint32_t b = step & 1;
+          if (!(ok = mbar_wait(v_full + st, (g0 / NS) & 1, epoch, 6))) break;
+          if (!(ok = mbar_wait(p_full + 2 * X + b, (step >> 1) & 1, epoch, 7 + X))) break;
+          if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc & 1) ^ 1, epoch, 9 + X))) break;
           tc_fence_after();
           const uint32_t d = tmem + TM_O + X * 128;
           const uint32_t pa = tmem + X * 2 * BLOCK_N + b * BLOCK_N;   // P (bf16 pairs) over the S columns
-#pragma unroll
+          const uint32_t va = aV + st * K::VTILE;
+  #pragma unroll
           for (int kk = 0; kk < BLOCK_N / 16; ++kk)
             mma_ts(d, pa + kk * 8, sdesc_c<K::VAT, 8 * K::VSW, layout_of(K::VSW)>(va + kk * 16 * K::VSW), IDPV,
                    (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(pv_done + 2 * X + b);
-          if (j + 1 == n_kv) {
-            tc_commit(o_full + X);
-            ++oc[X];
-          }
-          ++step[X];
+          tc_commit(v_empty + st);
         }
         if (!ok) break;
-        tc_commit(v_empty + st);
+        tc_commit(o_full + X);
+        ++oc;
+        kv += n_kv;
       }
-      kv += n_kv;
-    }
-    tc_commit(mma_done + 2);
-    const unsigned long long t0 = globaltimer();
-    while (!mbar_try_wait(mma_done + 2, 0) && globaltimer() - t0 < WAIT_NS) {
+      tc_commit(mma_done + 2 + X);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(mma_done + 2 + X, 0) && globaltimer() - t0 < WAIT_NS) {
+      }
     }
   } else if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
     // ================= softmax warpgroups =================
     const int X = warp >> 2;                   // tile
     const int r = ((warp & 3) << 5) + lane;    // row in tile == TMEM lane
@@ -674,14 +693,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive(stat_full + X);
       ++oc;
     }
-  } else if (warp >= W_EPI && warp < W_EPI + 4) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_EPI));
     // ================= epilogue warpgroup =================
     // Per tile: wait for the last PV and the row statistics, read O out of
-    // TMEM 16 columns at a time (TMEM is released after the last read),
-    // divide by the row sum, stage the 32 x 16 block of this warp in shared
-    // memory in the swizzled layout of the output tensor map, and let one
-    // lane write it with a bulk tensor store (rows past S and columns past D
-    // are dropped by the copy engine).  The LSE is written per row.
+    // TMEM into registers (TMEM is released right after), divide by the row
+    // sum, stage each 32 x 16 block of this warp in shared memory in the
+    // swizzled layout of the output tensor map, and let one lane write it
+    // with a bulk tensor store (rows past S and columns past D are dropped by
+    // the copy engine).  The LSE is written per row.
     const int qd = warp - W_EPI;               // TMEM lane quadrant
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     uint8_t *stg = sEpi + qd * 2 * EPI_BUF;
@@ -715,46 +735,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive(stat_empty + X);
         const float inv = 1.0f / l;
         const uint32_t tO = tmem + lane_off + TM_O + X * 128;
-        constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;
-#pragma unroll 1
-        for (int c = 0; c < NCH; ++c, ++nst) {
-          uint32_t ov[16];
-          TMEM_LD16(tO + c * 16, ov);
+        constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;    // 16-column chunks holding data
+        constexpr int G0 = NCH > 5 ? 4 : NCH;                  // chunks of the first register group
+        // O leaves TMEM in at most two register groups; TMEM is released as
+        // soon as the last group is loaded, before anything is stored.
+#pragma unroll
+        for (int grp = 0; grp < (NCH > G0 ? 2 : 1); ++grp) {
+          const int c0 = grp * G0;
+          const int nch = grp == 0 ? G0 : NCH - G0;
+          uint32_t ov[G0][16];
+#pragma unroll
+          for (int c = 0; c < G0; ++c)
+            if (c < nch) TMEM_LD16(tO + (c0 + c) * 16, ov[c]);
           tmem_wait_ld();
-          if (c + 1 == NCH) {
+          if (c0 + nch == NCH) {
             tc_fence_before();
             mbar_arrive(o_empty + X);          // O of this tile may be overwritten
           }
-          uint8_t *buf = stg + (nst & 1) * EPI_BUF;
-          if (lane == 0) bulk_wait_read1();    // the store that used this buffer has read it
-          __syncwarp();
-          if (p.o_f32) {
-            // 64-byte rows, 64B swizzle: 16-byte chunk f of row r at f ^ ((r >> 1) & 3)
 #pragma unroll
-            for (int f = 0; f < 4; ++f)
-              *reinterpret_cast<float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4)) =
-                  make_float4(__uint_as_float(ov[4 * f]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
-                              __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
-          } else {
-            // 32-byte rows, 32B swizzle: 16-byte chunk f of row r at f ^ ((r >> 2) & 1)
+          for (int c = 0; c < G0; ++c, ++nst) {
+            if (c >= nch) break;
+            uint8_t *buf = stg + (nst & 1) * EPI_BUF;
+            if (lane == 0) bulk_wait_read1();  // the store that used this buffer has read it
+            __syncwarp();
+            if (p.o_f32) {
+              // 64-byte rows, 64B swizzle: 16-byte chunk f of row r at f ^ ((r >> 1) & 3)
 #pragma unroll
-            for (int f = 0; f < 2; ++f) {
-              uint4 w;
-              w.x = st::pack_bf16x2(__uint_as_float(ov[8 * f]) * inv, __uint_as_float(ov[8 * f + 1]) * inv);
-              w.y = st::pack_bf16x2(__uint_as_float(ov[8 * f + 2]) * inv, __uint_as_float(ov[8 * f + 3]) * inv);
-              w.z = st::pack_bf16x2(__uint_as_float(ov[8 * f + 4]) * inv, __uint_as_float(ov[8 * f + 5]) * inv);
-              w.w = st::pack_bf16x2(__uint_as_float(ov[8 * f + 6]) * inv, __uint_as_float(ov[8 * f + 7]) * inv);
-              *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
+              for (int f = 0; f < 4; ++f)
+                *reinterpret_cast<float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4)) =
+                    make_float4(__uint_as_float(ov[c][4 * f]) * inv, __uint_as_float(ov[c][4 * f + 1]) * inv,
+                                __uint_as_float(ov[c][4 * f + 2]) * inv, __uint_as_float(ov[c][4 * f + 3]) * inv);
+            } else {
+              // 32-byte rows, 32B swizzle: 16-byte chunk f of row r at f ^ ((r >> 2) & 1)
+#pragma unroll
+              for (int f = 0; f < 2; ++f) {
+                uint4 w;
+                w.x = st::pack_bf16x2(__uint_as_float(ov[c][8 * f]) * inv, __uint_as_float(ov[c][8 * f + 1]) * inv);
+                w.y = st::pack_bf16x2(__uint_as_float(ov[c][8 * f + 2]) * inv, __uint_as_float(ov[c][8 * f + 3]) * inv);
+                w.z = st::pack_bf16x2(__uint_as_float(ov[c][8 * f + 4]) * inv, __uint_as_float(ov[c][8 * f + 5]) * inv);
+                w.w = st::pack_bf16x2(__uint_as_float(ov[c][8 * f + 6]) * inv, __uint_as_float(ov[c][8 * f + 7]) * inv);
+                *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
+              }
             }
-          }
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            // a block wholly past the last row stores nothing, but still
-            // commits a (empty) group so the buffer accounting stays in step
-            const int row0 = it.q0 + X * BLOCK_M + qd * 32;
-            if (row0 < g.S) tma_store_5d(&to, buf, c * EPI_COLS, it.h, row0, it.c3, it.c4);
-            bulk_commit();
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              // a block wholly past the last row stores nothing, but still
+              // commits a (empty) group so the buffer accounting stays in step
+              const int row0 = it.q0 + X * BLOCK_M + qd * 32;
+              if (row0 < g.S) tma_store_5d(&to, buf, (c0 + c) * EPI_COLS, it.h, row0, it.c3, it.c4);
+              bulk_commit();
+            }
           }
         }
         if (valid && p.lse) p.lse[lse_idx] = (m + log2f(l)) * 0.6931471805599453f;
@@ -882,6 +913,16 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   auto kern = attn_fwd_sm100<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM) != cudaSuccess)
     return ST_ERR_CUDA;
+  // The register split of the warpgroups (setmaxnreg) assumes the launch
+  // grants 96 registers per thread; with fewer, the warpgroups that ask for
+  // more would wait forever.  Refuse to launch such a build.
+  static int regs_ok = -1;
+  if (regs_ok < 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ST_ERR_CUDA;
+    regs_ok = fa.numRegs * NUM_THREADS >= 256 * REG_SOFTMAX + 128 * REG_EPI + 256 * REG_ISSUE ? 1 : 0;
+  }
+  if (!regs_ok) return ST_ERR_UNSUPPORTED;
   kern<<<ctas, NUM_THREADS, K::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
   return st::launch_status();
 }
