@@ -25,6 +25,7 @@ int num_sms();
 // Reads and clears the device error word of the tensor-core attention kernel
 // (defined next to that kernel).  Returns the word's previous value.
 unsigned int read_and_clear_attn_error(cudaStream_t stream, cudaError_t *err);
+unsigned int read_and_clear_relayout_error(cudaStream_t stream, cudaError_t *err);
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
 

@@ -8,9 +8,10 @@
 // Design.  HBM-bound: every partial element is read once and every output
 // written once.  One thread owns four consecutive channels of one
 // (unit, token, head) row: it reads the R chunk LSEs of the row (the other
-// threads of the row hit the same cache lines), computes the R weights once,
-// then issues all R 16-byte partial loads before the FMAs.  Output is fp32
-// or bf16 (rounded once, to nearest even).
+// threads of the row hit the same cache lines) and the R 16-byte partials,
+// all issued before any arithmetic (and for two elements at a time), then
+// forms the weights and the sum.  Output is fp32 or bf16 (rounded once, to
+// nearest even).
 #include <math.h>
 
 #include "common.cuh"
@@ -24,74 +25,95 @@ struct MergeArgs {
   const float *lse[MAXC];
 };
 
-template <bool BF16, int R>
-__global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, long long n_rows_h, int S,
-                                                    int H, int D4, void *__restrict__ o_out,
-                                                    float *__restrict__ lse_out) {
+// Element f of the output (four channels) -> index of its LSE row.
+template <typename I>
+__device__ __forceinline__ I lse_index(I f, int D4, int H, int S) {
+  const I rh = f / D4;                   // (unit, s, h) row index
+  const I row = rh / H;                  // unit * S + s
+  const int h = int(rh - row * H);
+  const I unit = row / S;
+  const int s = int(row - unit * S);
+  return (unit * H + h) * S + s;
+}
+
+// I is the index type (32-bit when every index fits).  Each thread handles
+// U elements per iteration and issues all their loads (R LSEs and R partial
+// vectors each) before any arithmetic, so U * 2R loads are in flight.
+template <bool BF16, int R, typename I>
+__global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_rows_h, int S, int H, int D4,
+                                                    void *__restrict__ o_out, float *__restrict__ lse_out) {
+  constexpr int NC = R > 0 ? R : MAXC;
+  constexpr int U = R > 0 && R <= 4 ? 2 : 1;
   const int n = R > 0 ? R : nc;
-  const long long total = n_rows_h * D4;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long f = (long long)blockIdx.x * blockDim.x + threadIdx.x; f < total; f += stride) {
-    const long long rh = f / D4;             // (unit, s, h) row index
-    const int d4 = int(f - rh * D4);
-    const long long row = rh / H;            // unit * S + s
-    const int h = int(rh - row * H);
-    const long long unit = row / S;
-    const int s = int(row - unit * S);
-    const long long li = (unit * H + h) * S + s;
-    float l[MAXC];
-    float M = -INFINITY;
+  const I total = n_rows_h * D4;
+  const I stride = (I)gridDim.x * blockDim.x;
+  for (I f0 = (I)blockIdx.x * blockDim.x + threadIdx.x; f0 < total; f0 += stride * U) {
+    float l[U][NC];
+    float4 v[U][NC];
+    I li[U];
 #pragma unroll
-    for (int c = 0; c < (R > 0 ? R : MAXC); ++c) {
-      if (c < n) {
-        l[c] = __ldg(a.lse[c] + li);
-        M = fmaxf(M, l[c]);
+    for (int u = 0; u < U; ++u) {
+      const I f = f0 + (I)u * stride;
+      if (f < total) {
+        li[u] = lse_index<I>(f, D4, H, S);
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+          if (c < n) {
+            l[u][c] = __ldg(a.lse[c] + li[u]);
+            v[u][c] = __ldg(a.o[c] + f);
+          }
       }
     }
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lse = -INFINITY;
-    if (M != -INFINITY) {
-      float sum = 0.f;
-      float4 v[R > 0 ? R : MAXC];
 #pragma unroll
-      for (int c = 0; c < (R > 0 ? R : MAXC); ++c)
-        if (c < n) v[c] = __ldg(a.o[c] + f);
+    for (int u = 0; u < U; ++u) {
+      const I f = f0 + (I)u * stride;
+      if (f >= total) break;
+      float M = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < (R > 0 ? R : MAXC); ++c)
-        if (c < n) sum += expf(l[c] - M);
-      lse = M + logf(sum);
+      for (int c = 0; c < NC; ++c)
+        if (c < n) M = fmaxf(M, l[u][c]);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float lse = -INFINITY;
+      if (M != -INFINITY) {
+        float sum = 0.f;
 #pragma unroll
-      for (int c = 0; c < (R > 0 ? R : MAXC); ++c) {
-        if (c < n) {
-          const float w = expf(l[c] - lse);
-          acc.x = fmaf(w, v[c].x, acc.x);
-          acc.y = fmaf(w, v[c].y, acc.y);
-          acc.z = fmaf(w, v[c].z, acc.z);
-          acc.w = fmaf(w, v[c].w, acc.w);
+        for (int c = 0; c < NC; ++c)
+          if (c < n) sum += expf(l[u][c] - M);
+        lse = M + logf(sum);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          if (c < n) {
+            const float w = expf(l[u][c] - lse);
+            acc.x = fmaf(w, v[u][c].x, acc.x);
+            acc.y = fmaf(w, v[u][c].y, acc.y);
+            acc.z = fmaf(w, v[u][c].z, acc.z);
+            acc.w = fmaf(w, v[u][c].w, acc.w);
+          }
         }
       }
+      if (BF16) {
+        uint2 pk;
+        pk.x = st::pack_bf16x2(acc.x, acc.y);
+        pk.y = st::pack_bf16x2(acc.z, acc.w);
+        reinterpret_cast<uint2 *>(o_out)[f] = pk;
+      } else {
+        reinterpret_cast<float4 *>(o_out)[f] = acc;
+      }
+      if (lse_out && f % D4 == 0) lse_out[li[u]] = lse;
     }
-    if (BF16) {
-      uint2 p;
-      p.x = st::pack_bf16x2(acc.x, acc.y);
-      p.y = st::pack_bf16x2(acc.z, acc.w);
-      reinterpret_cast<uint2 *>(o_out)[f] = p;
-    } else {
-      reinterpret_cast<float4 *>(o_out)[f] = acc;
-    }
-    if (lse_out && d4 == 0) lse_out[li] = lse;
   }
 }
 
-template <bool BF16>
+template <bool BF16, typename I>
 void launch(const MergeArgs &a, int nc, long long rows_h, int S, int H, int D4, void *o, float *lse,
             int grid, cudaStream_t s) {
+  const I rh = (I)rows_h;
   switch (nc) {
-    case 1: merge_kernel<BF16, 1><<<grid, 256, 0, s>>>(a, nc, rows_h, S, H, D4, o, lse); break;
-    case 2: merge_kernel<BF16, 2><<<grid, 256, 0, s>>>(a, nc, rows_h, S, H, D4, o, lse); break;
-    case 4: merge_kernel<BF16, 4><<<grid, 256, 0, s>>>(a, nc, rows_h, S, H, D4, o, lse); break;
-    case 8: merge_kernel<BF16, 8><<<grid, 256, 0, s>>>(a, nc, rows_h, S, H, D4, o, lse); break;
-    default: merge_kernel<BF16, 0><<<grid, 256, 0, s>>>(a, nc, rows_h, S, H, D4, o, lse); break;
+    case 1: merge_kernel<BF16, 1, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
+    case 2: merge_kernel<BF16, 2, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
+    case 4: merge_kernel<BF16, 4, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
+    case 8: merge_kernel<BF16, 8, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
+    default: merge_kernel<BF16, 0, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
   }
 }
 
@@ -118,7 +140,14 @@ ST_API st_status attn_chunk_merge(int n_chunks, const float *const *o_parts, con
   const long long cap = (long long)st::num_sms() * 16;
   const int grid = int(want < cap ? want : cap);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (out_dtype == ST_BF16) launch<true>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
-  else launch<false>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
+  // 32-bit indexing when every element and LSE index (and the loop's overshoot) fits
+  const bool small = total + (long long)grid * 256 * 2 < (1LL << 31);
+  if (out_dtype == ST_BF16) {
+    if (small) launch<true, int>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
+    else launch<true, long long>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
+  } else {
+    if (small) launch<false, int>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
+    else launch<false, long long>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
+  }
   return st::launch_status();
 }

@@ -16,8 +16,8 @@
 // the D channels of one (token, head).  A group of lanes maps one segment with
 // a few integer divisions and then streams it with the widest aligned vector
 // (16 bytes when possible), several vectors in flight per lane, in destination
-// order.  The optional RMSNorm is a second kernel with one thread per head
-// segment (its sum of squares stays in registers).
+// order.  The optional RMSNorm is a second kernel: the bulk copy engine
+// stages 32 heads per warp in shared memory, one lane normalises each head.
 #include "common.cuh"
 
 namespace {
@@ -143,75 +143,228 @@ __global__ void __launch_bounds__(256) relayout_copy(Map m, int G, int log2G,
   }
 }
 
-// RMSNorm flavour: one thread per head segment of D elements.
+// ---------------------------------------------------------------- RMSNorm flavour
 //   y_d = x_d / sqrt(mean_d x_d^2 + eps) * gamma_d   (fp32 math)
+// A warp task is 32 consecutive heads in destination order.  The bulk copy
+// engine brings them into a per-warp shared buffer (one copy when the heads
+// are contiguous in the source, as inside a spatial/temporal segment;
+// otherwise one copy per head, issued by the heads' lanes), each lane
+// normalises one head in place, and one bulk copy writes the 32 heads back.
+// Every warp double-buffers: the next task's load is in flight while the
+// current one is normalised.  Waits on the copies are bounded in time.
+__device__ unsigned int g_relayout_error;
+
+__device__ __forceinline__ uint32_t sh_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(sh_u32(dst)), "l"(src), "r"(bytes), "r"(sh_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(sh_u32(src)),
+               "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sh_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool bar_try(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}\n"
+               : "=r"(ok)
+               : "r"(sh_u32(bar)), "r"(parity)
+               : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+constexpr int RMS_WARPS = 4;
+constexpr unsigned long long RMS_WAIT_NS = 2000000000ull;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256) relayout_rms(Map m, const char *__restrict__ in,
-                                                    char *__restrict__ out,
-                                                    const float *__restrict__ gamma,
-                                                    float eps) {
-  constexpr int VPH = D * int(sizeof(T)) / 16;          // 16-byte vectors per head
-  constexpr int EPV = 16 / int(sizeof(T));               // elements per vector
-  const long long heads_per_seg = m.seg_bytes / (D * (long long)sizeof(T));
-  const long long n_heads = m.n_segs * heads_per_seg;
+__global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char *__restrict__ in,
+                                                               char *__restrict__ out,
+                                                               const float *__restrict__ gamma, float eps) {
+  constexpr int EPV = 16 / int(sizeof(T));               // elements per 16-byte vector
+  constexpr int VPH = D / EPV;                           // vectors per head
+  constexpr int HB = D * int(sizeof(T));                 // bytes per head
+  constexpr int BUF = 32 * HB;                           // bytes per warp buffer
+  constexpr int ROT = VPH % 4 == 0 ? 1 : 0;              // vector rotation per lane: no bank conflicts
+  extern __shared__ __align__(128) uint8_t rms_smem[];
+  __shared__ uint64_t full[RMS_WARPS][2];
   __shared__ float g_s[D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
-  __syncthreads();
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long hi = (long long)blockIdx.x * blockDim.x + threadIdx.x; hi < n_heads; hi += stride) {
-    const long long seg = hi / heads_per_seg;
-    const long long r = hi - seg * heads_per_seg;
-    long long s, d;
-    map_segment(m, seg, s, d);
-    const long long off = r * D * (long long)sizeof(T);
-    const uint4 *src = reinterpret_cast<const uint4 *>(in + s + off);
-    uint4 *dst = reinterpret_cast<uint4 *>(out + d + off);
-    uint4 v[VPH];
-#pragma unroll
-    for (int u = 0; u < VPH; ++u) v[u] = __ldg(src + u);
-    float ss = 0.f;
-#pragma unroll
-    for (int u = 0; u < VPH; ++u) {
-      const T *e = reinterpret_cast<const T *>(&v[u]);
-#pragma unroll
-      for (int k = 0; k < EPV; ++k) {
-        float x;
-        if constexpr (sizeof(T) == 2) x = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(e)[k]);
-        else x = reinterpret_cast<const float *>(e)[k];
-        ss = fmaf(x, x, ss);
-      }
-    }
-    const float inv = 1.0f / sqrtf(ss / float(D) + eps);
-#pragma unroll
-    for (int u = 0; u < VPH; ++u) {
-      if constexpr (sizeof(T) == 2) {
-        uint16_t *e = reinterpret_cast<uint16_t *>(&v[u]);
-#pragma unroll
-        for (int k = 0; k < EPV; ++k)
-          e[k] = st::f32_to_bf16(st::bf16_to_f32(e[k]) * inv * g_s[u * EPV + k]);
-      } else {
-        float *e = reinterpret_cast<float *>(&v[u]);
-#pragma unroll
-        for (int k = 0; k < EPV; ++k) e[k] = e[k] * inv * g_s[u * EPV + k];
-      }
-      dst[u] = v[u];
-    }
+  if (lane == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][1])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  __syncthreads();
+  uint8_t *buf0 = rms_smem + warp * 2 * BUF;
+  const bool one_src = (m.mode == ST_S2T || m.mode == ST_T2S);   // heads of a task contiguous in the source
+  const long long hps = m.seg_bytes / HB;                         // heads per segment
+  const long long tps = one_src ? (hps + 31) / 32 : 1;            // tasks per segment (unused otherwise)
+  const long long n_tasks = one_src ? m.n_segs * tps : (m.n_segs + 31) / 32;
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+
+  // task -> (destination byte offset, number of heads); issues its load into buffer b
+  auto issue = [&](long long task, int b, long long &dst, int &nh) {
+    uint8_t *bufp = buf0 + b * BUF;
+    if (one_src) {
+      const long long seg = task / tps;
+      const long long c = task - seg * tps;
+      nh = int(min(32LL, hps - c * 32));
+      long long so, dof;
+      map_segment(m, seg, so, dof);
+      dst = dof + c * 32 * HB;
+      if (lane == 0) {
+        expect_tx(&full[warp][b], nh * HB);
+        bulk_g2s(bufp, in + so + c * 32 * HB, nh * HB, &full[warp][b]);
+      }
+    } else {
+      const long long g0 = task * 32;
+      nh = int(min(32LL, m.n_segs - g0));
+      long long so, dof;
+      map_segment(m, g0 + (lane < nh ? lane : 0), so, dof);
+      dst = __shfl_sync(0xffffffffu, dof, 0);                     // destination rows are consecutive
+      if (lane == 0) expect_tx(&full[warp][b], nh * HB);
+      __syncwarp();
+      if (lane < nh) bulk_g2s(bufp + lane * HB, in + so, HB, &full[warp][b]);
+    }
+  };
+
+  bool ok = true;
+  long long dst_cur = 0, dst_next = 0;
+  int nh_cur = 0, nh_next = 0;
+  if (gw < n_tasks) issue(gw, 0, dst_cur, nh_cur);
+  int i = 0;
+  for (long long task = gw; task < n_tasks && ok; task += nw, ++i) {
+    const int b = i & 1;
+    const long long next = task + nw;
+    if (next < n_tasks) {
+      // the store of the previous task used the other buffer: it must have read it
+      if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      __syncwarp();
+      issue(next, b ^ 1, dst_next, nh_next);
+    }
+    {
+      const unsigned long long t0 = gtimer();
+      while (!bar_try(&full[warp][b], (i >> 1) & 1)) {
+        if (gtimer() - t0 > RMS_WAIT_NS) {
+          atomicOr(&g_relayout_error, 1u);
+          ok = false;
+          break;
+        }
+      }
+    }
+    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+    uint8_t *bufp = buf0 + b * BUF;
+    if (lane < nh_cur) {
+      uint8_t *h = bufp + lane * HB;
+      const int r0 = (lane * ROT) % VPH;
+      float ss = 0.f;
+#pragma unroll
+      for (int u0 = 0; u0 < VPH; ++u0) {
+        const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
+        const uint4 v = *reinterpret_cast<const uint4 *>(h + u * 16);
+        if constexpr (sizeof(T) == 2) {
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float a = __uint_as_float(w[k] << 16), c = __uint_as_float(w[k] & 0xffff0000u);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(c, c, ss);
+          }
+        } else {
+          ss = fmaf(__uint_as_float(v.x), __uint_as_float(v.x), ss);
+          ss = fmaf(__uint_as_float(v.y), __uint_as_float(v.y), ss);
+          ss = fmaf(__uint_as_float(v.z), __uint_as_float(v.z), ss);
+          ss = fmaf(__uint_as_float(v.w), __uint_as_float(v.w), ss);
+        }
+      }
+      const float inv = rsqrtf(ss * (1.0f / float(D)) + eps);
+#pragma unroll
+      for (int u0 = 0; u0 < VPH; ++u0) {
+        const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
+        uint4 v = *reinterpret_cast<const uint4 *>(h + u * 16);
+        const float *gg = g_s + u * EPV;
+        if constexpr (sizeof(T) == 2) {
+          uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            w[k] = st::pack_bf16x2(__uint_as_float(w[k] << 16) * inv * gg[2 * k],
+                                   __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1]);
+          v = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+          v = make_uint4(__float_as_uint(__uint_as_float(v.x) * inv * gg[0]),
+                         __float_as_uint(__uint_as_float(v.y) * inv * gg[1]),
+                         __float_as_uint(__uint_as_float(v.z) * inv * gg[2]),
+                         __float_as_uint(__uint_as_float(v.w) * inv * gg[3]));
+        }
+        *reinterpret_cast<uint4 *>(h + u * 16) = v;
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) bulk_s2g(out + dst_cur, bufp, nh_cur * HB);
+    dst_cur = dst_next;
+    nh_cur = nh_next;
+  }
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  if (!ok && lane == 0) {
+    // a copy into this warp's buffers may still be in flight: wait for it (bounded) before exiting
+    const unsigned long long t0 = gtimer();
+    for (int it = i; it < i + 2; ++it)   // uses it and it + 1: buffer it & 1, phase (it >> 1) & 1
+      while (!bar_try(&full[warp][it & 1], (it >> 1) & 1) && gtimer() - t0 < RMS_WAIT_NS) {
+      }
+  }
+  __syncwarp();
+}
+
+template <typename T, int D>
+st_status launch_rms_d(const Map &m, const char *in, char *out, const float *gamma, float eps, int sms,
+                       cudaStream_t s) {
+  constexpr int BUF = 32 * D * int(sizeof(T));
+  constexpr int SMEM = RMS_WARPS * 2 * BUF;
+  auto kern = relayout_rms<T, D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+    return ST_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, RMS_WARPS * 32, SMEM) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const bool one_src = (m.mode == ST_S2T || m.mode == ST_T2S);
+  const long long hps = m.seg_bytes / (D * (long long)sizeof(T));
+  const long long n_tasks = one_src ? m.n_segs * ((hps + 31) / 32) : (m.n_segs + 31) / 32;
+  const long long want = (n_tasks + RMS_WARPS - 1) / RMS_WARPS;
+  const long long cap = (long long)sms * per_sm;
+  const int grid = int(want < cap ? want : cap);
+  kern<<<grid, RMS_WARPS * 32, SMEM, s>>>(m, in, out, gamma, eps);
+  return st::launch_status();
 }
 
 template <typename T>
-st_status launch_rms(const Map &m, const char *in, char *out, const float *gamma, int D,
-                     float eps, int grid, cudaStream_t s) {
+st_status launch_rms(const Map &m, const char *in, char *out, const float *gamma, int D, float eps, int sms,
+                     cudaStream_t s) {
   switch (D) {
-    case 32: relayout_rms<T, 32><<<grid, 256, 0, s>>>(m, in, out, gamma, eps); break;
-    case 64: relayout_rms<T, 64><<<grid, 256, 0, s>>>(m, in, out, gamma, eps); break;
-    case 72: relayout_rms<T, 72><<<grid, 256, 0, s>>>(m, in, out, gamma, eps); break;
-    case 80: relayout_rms<T, 80><<<grid, 256, 0, s>>>(m, in, out, gamma, eps); break;
-    case 96: relayout_rms<T, 96><<<grid, 256, 0, s>>>(m, in, out, gamma, eps); break;
-    case 128: relayout_rms<T, 128><<<grid, 256, 0, s>>>(m, in, out, gamma, eps); break;
+    case 32: return launch_rms_d<T, 32>(m, in, out, gamma, eps, sms, s);
+    case 64: return launch_rms_d<T, 64>(m, in, out, gamma, eps, sms, s);
+    case 72: return launch_rms_d<T, 72>(m, in, out, gamma, eps, sms, s);
+    case 80: return launch_rms_d<T, 80>(m, in, out, gamma, eps, sms, s);
+    case 96: return launch_rms_d<T, 96>(m, in, out, gamma, eps, sms, s);
+    case 128: return launch_rms_d<T, 128>(m, in, out, gamma, eps, sms, s);
     default: return ST_ERR_UNSUPPORTED;
   }
-  return st::launch_status();
 }
 
 template <int VEC>
@@ -229,6 +382,18 @@ st_status launch_copy(const Map &m, const char *in, char *out, int grid, cudaStr
 }
 
 }  // namespace
+
+namespace st {
+unsigned int read_and_clear_relayout_error(cudaStream_t stream, cudaError_t *err) {
+  unsigned int word = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&word, g_relayout_error, sizeof(word), 0, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyToSymbolAsync(g_relayout_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (err) *err = e;
+  return word;
+}
+}  // namespace st
 
 ST_API st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *out, int elem_bytes,
                                   int P, int B, int T_or_N, int S_or_H, int C_or_D, int n_t,
@@ -277,11 +442,8 @@ ST_API st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *o
     if ((rms_head_dim * elem_bytes) % 16 || !st::is_aligned(in, 16) || !st::is_aligned(out, 16) ||
         m.row_bytes % 16)
       return ST_ERR_ALIGN;
-    const long long n_heads = m.n_segs * (m.seg_bytes / ((long long)rms_head_dim * elem_bytes));
-    const long long want = (n_heads + 255) / 256;
-    const int grid = int(want < (long long)sms * 16 ? want : (long long)sms * 16);
-    return elem_bytes == 2 ? launch_rms<uint16_t>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, grid, s)
-                           : launch_rms<float>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, grid, s);
+    return elem_bytes == 2 ? launch_rms<uint16_t>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s)
+                           : launch_rms<float>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s);
   }
   // widest vector that divides the row pitch and both base addresses
   int vec = 16;

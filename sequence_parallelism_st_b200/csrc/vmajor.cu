@@ -4,8 +4,8 @@
 //
 // Design.  vmajor_mask_compact is two launches and no atomics, so its output
 // is deterministic:
-//   1. l1_mask: one warp per token streams both [C] rows with 16-byte loads
-//      (all of a lane's loads issued before any arithmetic), accumulates
+//   1. l1_mask: a warp streams the [C] rows of two tokens at a time with
+//      16-byte loads (all of a lane's loads issued before any arithmetic), accumulates
 //      |cur - prev| in fp32, reduces over the warp with a fixed butterfly
 //      order, writes the mask byte, and each CTA writes the number of active
 //      tokens of its tile of TILE tokens to the workspace.
@@ -32,49 +32,66 @@ __global__ void __launch_bounds__(THREADS) l1_mask(const char *__restrict__ cur,
                                                    float *__restrict__ l1_out,
                                                    int *__restrict__ tile_count) {
   constexpr int EPV = 16 / int(sizeof(T));
+  constexpr int TPW = 2;                         // tokens of a warp in flight together
+  constexpr int VM = VMAX / TPW;                 // vectors per lane per token per tensor in flight
   __shared__ int warp_cnt[THREADS / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int active = 0;
-  for (int r = warp; r < TILE; r += THREADS / 32) {
-    const long long tok = (long long)blockIdx.x * TILE + r;
-    if (tok >= n) break;
-    const uint4 *a = reinterpret_cast<const uint4 *>(cur) + tok * row_vecs;
-    const uint4 *b = reinterpret_cast<const uint4 *>(prev) + tok * row_vecs;
-    float acc = 0.f;
-    for (int v0 = 0; v0 < row_vecs; v0 += 32 * VMAX) {
-      uint4 va[VMAX], vb[VMAX];
+  for (int r = warp; r < TILE; r += TPW * (THREADS / 32)) {
+    long long tok[TPW];
+    float acc[TPW];
 #pragma unroll
-      for (int u = 0; u < VMAX; ++u) {
-        const int v = v0 + u * 32 + lane;
-        if (v < row_vecs) { va[u] = __ldg(a + v); vb[u] = __ldg(b + v); }
+    for (int i = 0; i < TPW; ++i) {
+      tok[i] = (long long)blockIdx.x * TILE + r + i * (THREADS / 32);
+      acc[i] = 0.f;
+    }
+    for (int v0 = 0; v0 < row_vecs; v0 += 32 * VM) {
+      uint4 va[TPW][VM], vb[TPW][VM];
+#pragma unroll
+      for (int i = 0; i < TPW; ++i) {
+        const uint4 *a = reinterpret_cast<const uint4 *>(cur) + tok[i] * row_vecs;
+        const uint4 *b = reinterpret_cast<const uint4 *>(prev) + tok[i] * row_vecs;
+#pragma unroll
+        for (int u = 0; u < VM; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (tok[i] < n && v < row_vecs) { va[i][u] = __ldg(a + v); vb[i][u] = __ldg(b + v); }
+        }
       }
 #pragma unroll
-      for (int u = 0; u < VMAX; ++u) {
-        const int v = v0 + u * 32 + lane;
-        if (v < row_vecs) {
+      for (int i = 0; i < TPW; ++i) {
 #pragma unroll
-          for (int k = 0; k < EPV; ++k) {
-            float x, y;
-            if constexpr (sizeof(T) == 2) {
-              x = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(&va[u])[k]);
-              y = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(&vb[u])[k]);
-            } else {
-              x = reinterpret_cast<const float *>(&va[u])[k];
-              y = reinterpret_cast<const float *>(&vb[u])[k];
+        for (int u = 0; u < VM; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (tok[i] < n && v < row_vecs) {
+#pragma unroll
+            for (int k = 0; k < EPV; ++k) {
+              float x, y;
+              if constexpr (sizeof(T) == 2) {
+                x = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(&va[i][u])[k]);
+                y = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(&vb[i][u])[k]);
+              } else {
+                x = reinterpret_cast<const float *>(&va[i][u])[k];
+                y = reinterpret_cast<const float *>(&vb[i][u])[k];
+              }
+              acc[i] += fabsf(x - y);
             }
-            acc += fabsf(x - y);
           }
         }
       }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    const int m = (force_all || acc > tau) ? 1 : 0;
-    if (lane == 0) {
-      mask[tok] = (unsigned char)m;
-      if (l1_out) l1_out[tok] = acc;
+    for (int i = 0; i < TPW; ++i) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+      if (tok[i] < n) {
+        const int m = (force_all || acc[i] > tau) ? 1 : 0;
+        if (lane == 0) {
+          mask[tok[i]] = (unsigned char)m;
+          if (l1_out) l1_out[tok[i]] = acc[i];
+        }
+        active += m;
+      }
     }
-    active += m;
   }
   if (lane == 0) warp_cnt[warp] = active;
   __syncthreads();
@@ -133,7 +150,9 @@ __global__ void __launch_bounds__(THREADS) compact(const unsigned char *__restri
 }
 
 // One warp per active row: copies each tensor's row to its cache (and to the
-// packed message buffer when present).
+// packed message buffer when present).  The (tensor, vector) pairs of a row
+// are enumerated together and a lane loads NB of them before storing any, so
+// the copy of a row costs one memory round trip, not one per vector.
 struct ScatterArgs {
   const char *src[8];
   char *dst[8];
@@ -144,6 +163,7 @@ __global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
                                                     const int *__restrict__ count, long long n,
                                                     long long row_bytes, int vec, int n_tensors,
                                                     ScatterArgs a) {
+  constexpr int NB = 10;
   const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long cnt = *count;
@@ -151,17 +171,31 @@ __global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
   for (long long i = w; i < cnt && i < n; i += n_warps) {
     const long long row = idx[i];
     if (row < 0 || row >= n) continue;
-    for (int t = 0; t < n_tensors; ++t) {
-      if (vec == 16) {
-        const uint4 *s = reinterpret_cast<const uint4 *>(a.src[t] + row * row_bytes);
-        uint4 *d = reinterpret_cast<uint4 *>(a.dst[t] + row * row_bytes);
-        uint4 *p = a.packed[t] ? reinterpret_cast<uint4 *>(a.packed[t] + i * row_bytes) : nullptr;
-        for (long long k = lane; k < row_bytes / 16; k += 32) {
-          const uint4 v = __ldg(s + k);
-          d[k] = v;
-          if (p) p[k] = v;
+    if (vec == 16) {
+      const int rv = int(row_bytes / 16);
+      const int total = rv * n_tensors;
+      for (int j0 = 0; j0 < total; j0 += 32 * NB) {
+        uint4 v[NB];
+#pragma unroll
+        for (int u = 0; u < NB; ++u) {
+          const int j = j0 + u * 32 + lane;
+          if (j < total) {
+            const int t = j / rv, k = j - t * rv;
+            v[u] = __ldg(reinterpret_cast<const uint4 *>(a.src[t] + row * row_bytes) + k);
+          }
         }
-      } else {
+#pragma unroll
+        for (int u = 0; u < NB; ++u) {
+          const int j = j0 + u * 32 + lane;
+          if (j < total) {
+            const int t = j / rv, k = j - t * rv;
+            reinterpret_cast<uint4 *>(a.dst[t] + row * row_bytes)[k] = v[u];
+            if (a.packed[t]) reinterpret_cast<uint4 *>(a.packed[t] + i * row_bytes)[k] = v[u];
+          }
+        }
+      }
+    } else {
+      for (int t = 0; t < n_tensors; ++t) {
         const char *s = a.src[t] + row * row_bytes;
         char *d = a.dst[t] + row * row_bytes;
         char *p = a.packed[t] ? a.packed[t] + i * row_bytes : nullptr;
@@ -232,6 +266,7 @@ ST_API st_status vmajor_scatter_rows(const int *idx, const int *count, long long
     all16 = all16 && st::is_aligned(src[t], 16) && st::is_aligned(dst_cache[t], 16) &&
             (!a.packed[t] || st::is_aligned(a.packed[t], 16));
   }
+  if (all16 && (row_bytes / 16) * n_tensors >= (1LL << 31)) return ST_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const long long want = (n_tokens * 32 + 255) / 256;
   const long long cap = (long long)st::num_sms() * 16;
