@@ -13,8 +13,9 @@
 //     while the current one computes) when two stages fit in 64 KB.  The
 //     group's rows are contiguous in HBM (4*D channels), so every frame row
 //     is streamed with 16-byte cp.async into a padded shared-memory tile (row
-//     pitch 4D+8 elements keeps ldmatrix conflict-free); frames past T are
-//     zero-filled.  Frame offsets come from a per-CTA table in shared memory.
+//     pitch 4D+8 elements keeps ldmatrix conflict-free); rows past T are
+//     zeroed once.  A thread owns one (tensor, 16-byte column) and walks the
+//     frames, whose offsets come from a per-CTA table in shared memory.
 //   * Warp w owns head w of the group: S = Q K^T from ldmatrix fragments,
 //     row max / row sum by quad shuffles (the warp-shuffle softmax), P kept
 //     in registers and re-packed as the A fragment of O = P V (V fragments
@@ -91,6 +92,11 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
   long long *ftab = reinterpret_cast<long long *>(smem + STAGES * 3 * TILE);   // [B * T] frame offsets
   const int T = g.T;
   for (int i = threadIdx.x; i < g.B * T; i += blockDim.x) ftab[i] = g.frame(i / T, i % T);
+  // rows past T are never loaded: zero them once in every tile
+  for (int i = threadIdx.x; i < STAGES * 3 * (TP - T) * RS; i += blockDim.x) {
+    const int tile = i / ((TP - T) * RS), r = i - tile * (TP - T) * RS;
+    smem[tile * TILE + T * RS + r] = 0;
+  }
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -105,15 +111,15 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
     const long long tok = g.token(s) + (long long)hg * G * D;
     const long long *fb = ftab + b * T;
     uint16_t *st_base = smem + stage * 3 * TILE;
-    for (int i = threadIdx.x; i < 3 * TP * CH; i += blockDim.x) {
-      const int x = i / (TP * CH);
-      const int r = i - x * TP * CH;
-      const int t = r / CH;
-      const int c = r - t * CH;
-      const uint16_t *base = x == 0 ? q : (x == 1 ? k : v);
-      const bool ok = t < T && c * 8 < heads_here * D;
-      const uint16_t *src = ok ? base + fb[t] + tok + c * 8 : base;
-      cp_async16(st_base + x * TILE + t * RS + c * 8, src, ok ? 16 : 0);
+    // a thread owns a (tensor, 16-byte column) pair and walks the T frames:
+    // one shared-table read, one add and one copy per 16 bytes
+    const int cols = heads_here * D / 8;
+    for (int pc = threadIdx.x; pc < 3 * CH; pc += blockDim.x) {
+      const int x = pc / CH, c = pc - x * CH;
+      if (c >= cols) continue;
+      const uint16_t *src = (x == 0 ? q : (x == 1 ? k : v)) + tok + c * 8;
+      uint16_t *dst = st_base + x * TILE + c * 8;
+      for (int t = 0; t < T; ++t) cp_async16(dst + t * RS, src + fb[t], 16);
     }
     asm volatile("cp.async.commit_group;\n" ::: "memory");
   };

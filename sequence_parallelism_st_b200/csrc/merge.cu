@@ -10,7 +10,8 @@
 // (unit, token, head) row: it reads the R chunk LSEs of the row (the other
 // threads of the row hit the same cache lines) and the R 16-byte partials,
 // all issued before any arithmetic (and for two elements at a time), then
-// forms the weights and the sum.  Output is fp32 or bf16 (rounded once, to
+// forms the weights as exp(lse_c - M) / sum_c' exp(lse_c' - M): R
+// exponentials and one reciprocal; the log only where the LSE is written.  Output is fp32 or bf16 (rounded once, to
 // nearest even).
 #include <math.h>
 
@@ -73,17 +74,21 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_row
       for (int c = 0; c < NC; ++c)
         if (c < n) M = fmaxf(M, l[u][c]);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      float lse = -INFINITY;
+      float sum = 0.f;
       if (M != -INFINITY) {
-        float sum = 0.f;
+        // w_c = exp(lse_c - lse) = e_c / sum_c' e_c' with e_c = exp(lse_c - M)
+        float e[NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c)
-          if (c < n) sum += expf(l[u][c] - M);
-        lse = M + logf(sum);
+          if (c < n) {
+            e[c] = exp2f((l[u][c] - M) * 1.4426950408889634f);
+            sum += e[c];
+          }
+        const float inv = 1.0f / sum;
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
           if (c < n) {
-            const float w = expf(l[u][c] - lse);
+            const float w = e[c] * inv;
             acc.x = fmaf(w, v[u][c].x, acc.x);
             acc.y = fmaf(w, v[u][c].y, acc.y);
             acc.z = fmaf(w, v[u][c].z, acc.z);
@@ -99,7 +104,7 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_row
       } else {
         reinterpret_cast<float4 *>(o_out)[f] = acc;
       }
-      if (lse_out && f % D4 == 0) lse_out[li[u]] = lse;
+      if (lse_out && f % D4 == 0) lse_out[li[u]] = M != -INFINITY ? M + logf(sum) : -INFINITY;
     }
   }
 }
