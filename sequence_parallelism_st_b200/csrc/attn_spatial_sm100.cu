@@ -50,6 +50,9 @@
 
 namespace {
 
+using st::pdl_trigger;
+using st::pdl_wait;
+
 __device__ unsigned int g_attn_error;        // sites of waits that ran out
 __device__ unsigned int g_attn_abort_epoch;  // launch epoch that must abort
 
@@ -428,6 +431,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t epoch = p.epoch;
+  // barriers and TMEM are set up: let the next kernel of the stream be
+  // scheduled, then wait for the previous one before any global access
+  pdl_trigger();
+  pdl_wait();
 
   if (warp >= W_LOAD) {
     // warpgroups 3 and 4: TMA producer, MMA issuers, idle warps
@@ -923,8 +930,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
     regs_ok = fa.numRegs * NUM_THREADS >= 256 * REG_SOFTMAX + 128 * REG_EPI + 256 * REG_ISSUE ? 1 : 0;
   }
   if (!regs_ok) return ST_ERR_UNSUPPORTED;
-  kern<<<ctas, NUM_THREADS, K::SMEM, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
-  return st::launch_status();
+  return st::launch_pdl(kern, ctas, NUM_THREADS, K::SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
 }
 
 }  // namespace

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
   extern __shared__ __align__(16) uint16_t smem[];
   long long *ftab = reinterpret_cast<long long *>(smem + STAGES * 3 * TILE);   // [B * T] frame offsets
   const int T = g.T;
+  st::pdl_trigger();
   for (int i = threadIdx.x; i < g.B * T; i += blockDim.x) ftab[i] = g.frame(i / T, i % T);
   // rows past T are never loaded: zero them once in every tile
   for (int i = threadIdx.x; i < STAGES * 3 * (TP - T) * RS; i += blockDim.x) {
@@ -98,6 +99,7 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
     smem[tile * TILE + T * RS + r] = 0;
   }
   __syncthreads();
+  st::pdl_wait();   // everything above only touched shared memory
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, cq = lane & 3;
@@ -304,10 +306,9 @@ st_status launch_t(const st::Geom &g, int lo, int n_sel, float scale, const void
   const long long cap = (long long)st::num_sms() * per_sm;
   const int grid = int(items < cap ? items : cap);
   const float log2e = 1.4426950408889634f;
-  kern<<<grid, 128, smem, s>>>(g, lo, n_sel, n_hg, int(items), scale * log2e, scale,
-                               static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k),
-                               static_cast<const uint16_t *>(v), o, lse, o_f32);
-  return st::launch_status();
+  return st::launch_pdl(kern, grid, 128, smem, s, g, lo, n_sel, n_hg, int(items), scale * log2e, scale,
+                        static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k),
+                        static_cast<const uint16_t *>(v), o, lse, o_f32);
 }
 
 template <int D>

@@ -19,6 +19,36 @@ inline st_status launch_status() {
   return e == cudaSuccess ? ST_OK : ST_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream is still finishing; it must call
+// pdl_wait() before touching global memory that kernel produces or reads.
+template <typename... Params, typename... Args>
+inline st_status launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<Params>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return ST_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// Device side of the dependent launch: let the next kernel of the stream be
+// scheduled, and wait until the previous one has finished (its writes are
+// visible).  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // SM count of the current device (cached per device ordinal).
 int num_sms();
 

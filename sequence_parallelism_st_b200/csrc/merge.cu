@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_row
   constexpr int NC = R > 0 ? R : MAXC;
   constexpr int U = R > 0 && R <= 4 ? 2 : 1;
   const int n = R > 0 ? R : nc;
+  st::pdl_trigger();
+  st::pdl_wait();
   const I total = n_rows_h * D4;
   const I stride = (I)gridDim.x * blockDim.x;
   for (I f0 = (I)blockIdx.x * blockDim.x + threadIdx.x; f0 < total; f0 += stride * U) {
@@ -110,15 +112,15 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_row
 }
 
 template <bool BF16, typename I>
-void launch(const MergeArgs &a, int nc, long long rows_h, int S, int H, int D4, void *o, float *lse,
-            int grid, cudaStream_t s) {
+st_status launch(const MergeArgs &a, int nc, long long rows_h, int S, int H, int D4, void *o, float *lse,
+                 int grid, cudaStream_t s) {
   const I rh = (I)rows_h;
   switch (nc) {
-    case 1: merge_kernel<BF16, 1, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
-    case 2: merge_kernel<BF16, 2, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
-    case 4: merge_kernel<BF16, 4, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
-    case 8: merge_kernel<BF16, 8, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
-    default: merge_kernel<BF16, 0, I><<<grid, 256, 0, s>>>(a, nc, rh, S, H, D4, o, lse); break;
+    case 1: return st::launch_pdl(merge_kernel<BF16, 1, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
+    case 2: return st::launch_pdl(merge_kernel<BF16, 2, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
+    case 4: return st::launch_pdl(merge_kernel<BF16, 4, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
+    case 8: return st::launch_pdl(merge_kernel<BF16, 8, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
+    default: return st::launch_pdl(merge_kernel<BF16, 0, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
   }
 }
 
@@ -147,12 +149,9 @@ ST_API st_status attn_chunk_merge(int n_chunks, const float *const *o_parts, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // 32-bit indexing when every element and LSE index (and the loop's overshoot) fits
   const bool small = total + (long long)grid * 256 * 2 < (1LL << 31);
-  if (out_dtype == ST_BF16) {
-    if (small) launch<true, int>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
-    else launch<true, long long>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
-  } else {
-    if (small) launch<false, int>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
-    else launch<false, long long>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
-  }
-  return st::launch_status();
+  if (out_dtype == ST_BF16)
+    return small ? launch<true, int>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s)
+                 : launch<true, long long>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
+  return small ? launch<false, int>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s)
+               : launch<false, long long>(a, n_chunks, rows_h, S, H, D / 4, o_out, lse_out, grid, s);
 }

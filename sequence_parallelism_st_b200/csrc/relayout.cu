@@ -99,6 +99,8 @@ __global__ void __launch_bounds__(256) relayout_copy(Map m, int G, int log2G,
                                                      const char *__restrict__ in,
                                                      char *__restrict__ out) {
   using V = typename VecT<VEC>::t;
+  st::pdl_trigger();
+  st::pdl_wait();
   const long long seg_vecs = m.seg_bytes / VEC;
   const long long chunk = (long long)G * U;
   const long long n_chunks = (seg_vecs + chunk - 1) / chunk;
@@ -202,6 +204,8 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
   __shared__ uint64_t full[RMS_WARPS][2];
   __shared__ float g_s[D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  st::pdl_trigger();
+  st::pdl_wait();
   for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
   if (lane == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");
@@ -349,8 +353,7 @@ st_status launch_rms_d(const Map &m, const char *in, char *out, const float *gam
   const long long want = (n_tasks + RMS_WARPS - 1) / RMS_WARPS;
   const long long cap = (long long)sms * per_sm;
   const int grid = int(want < cap ? want : cap);
-  kern<<<grid, RMS_WARPS * 32, SMEM, s>>>(m, in, out, gamma, eps);
-  return st::launch_status();
+  return st::launch_pdl(kern, grid, RMS_WARPS * 32, SMEM, s, m, in, out, gamma, eps);
 }
 
 template <typename T>
@@ -370,15 +373,11 @@ st_status launch_rms(const Map &m, const char *in, char *out, const float *gamma
 template <int VEC>
 st_status launch_copy(const Map &m, const char *in, char *out, int grid, cudaStream_t s) {
   const long long seg_vecs = m.seg_bytes / VEC;
-  if (seg_vecs >= 256) {
-    relayout_copy<VEC, 8, 1><<<grid, 256, 0, s>>>(m, 32, 5, in, out);
-  } else {
-    int G = 1, lg = 0;
-    while (G < seg_vecs && G < 32) { G <<= 1; ++lg; }
-    if (seg_vecs <= G) relayout_copy<VEC, 1, 4><<<grid, 256, 0, s>>>(m, G, lg, in, out);
-    else relayout_copy<VEC, 8, 1><<<grid, 256, 0, s>>>(m, G, lg, in, out);
-  }
-  return st::launch_status();
+  if (seg_vecs >= 256) return st::launch_pdl(relayout_copy<VEC, 8, 1>, grid, 256, 0, s, m, 32, 5, in, out);
+  int G = 1, lg = 0;
+  while (G < seg_vecs && G < 32) { G <<= 1; ++lg; }
+  if (seg_vecs <= G) return st::launch_pdl(relayout_copy<VEC, 1, 4>, grid, 256, 0, s, m, G, lg, in, out);
+  return st::launch_pdl(relayout_copy<VEC, 8, 1>, grid, 256, 0, s, m, G, lg, in, out);
 }
 
 }  // namespace

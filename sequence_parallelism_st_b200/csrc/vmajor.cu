@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(THREADS) l1_mask(const char *__restrict__ cur,
   constexpr int VM = VMAX / TPW;                 // vectors per lane per token per tensor in flight
   __shared__ int warp_cnt[THREADS / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  st::pdl_trigger();
+  st::pdl_wait();
   int active = 0;
   for (int r = warp; r < TILE; r += TPW * (THREADS / 32)) {
     long long tok[TPW];
@@ -111,6 +113,8 @@ __global__ void __launch_bounds__(THREADS) compact(const unsigned char *__restri
   __shared__ int red[THREADS / 32];
   __shared__ int warp_tot[THREADS / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  st::pdl_trigger();
+  st::pdl_wait();
   const long long first_tile = (long long)blockIdx.x * (CTILE / TILE);
   int part = 0;
   for (long long t = threadIdx.x; t < first_tile; t += THREADS) part += tile_count[t];
@@ -164,6 +168,8 @@ __global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
                                                     long long row_bytes, int vec, int n_tensors,
                                                     ScatterArgs a) {
   constexpr int NB = 10;
+  st::pdl_trigger();
+  st::pdl_wait();
   const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long cnt = *count;
@@ -234,19 +240,16 @@ ST_API st_status vmajor_mask_compact(const void *v_cur, const void *v_prev, long
   if (tiles > 0x7fffffffLL) return ST_ERR_SHAPE;
   const int row_vecs = C * esize / 16;
   int *tile_count = static_cast<int *>(workspace);
-  if (dtype == ST_BF16)
-    l1_mask<uint16_t><<<int(tiles), THREADS, 0, s>>>(static_cast<const char *>(v_cur),
-                                                     static_cast<const char *>(v_prev), n_tokens,
-                                                     row_vecs, tau, force_all, mask, l1_out, tile_count);
-  else
-    l1_mask<float><<<int(tiles), THREADS, 0, s>>>(static_cast<const char *>(v_cur),
-                                                  static_cast<const char *>(v_prev), n_tokens,
-                                                  row_vecs, tau, force_all, mask, l1_out, tile_count);
-  st_status st = st::launch_status();
+  const char *cur = static_cast<const char *>(v_cur), *prev = static_cast<const char *>(v_prev);
+  st_status st = dtype == ST_BF16
+                     ? st::launch_pdl(l1_mask<uint16_t>, int(tiles), THREADS, 0, s, cur, prev, n_tokens, row_vecs,
+                                      tau, force_all, mask, l1_out, tile_count)
+                     : st::launch_pdl(l1_mask<float>, int(tiles), THREADS, 0, s, cur, prev, n_tokens, row_vecs, tau,
+                                      force_all, mask, l1_out, tile_count);
   if (st != ST_OK) return st;
   const int ctas = int((n_tokens + CTILE - 1) / CTILE);
-  compact<<<ctas, THREADS, 0, s>>>(mask, n_tokens, ctas, tile_count, idx, count);
-  return st::launch_status();
+  return st::launch_pdl(compact, ctas, THREADS, 0, s, static_cast<const unsigned char *>(mask), n_tokens, ctas,
+                        static_cast<const int *>(tile_count), idx, count);
 }
 
 ST_API st_status vmajor_scatter_rows(const int *idx, const int *count, long long n_tokens, int C,
@@ -271,8 +274,8 @@ ST_API st_status vmajor_scatter_rows(const int *idx, const int *count, long long
   const long long want = (n_tokens * 32 + 255) / 256;
   const long long cap = (long long)st::num_sms() * 16;
   const int grid = int(want < cap ? want : cap);
-  scatter_rows<<<grid, 256, 0, s>>>(idx, count, n_tokens, row_bytes, all16 ? 16 : 1, n_tensors, a);
-  return st::launch_status();
+  return st::launch_pdl(scatter_rows, grid, 256, 0, s, idx, count, n_tokens, row_bytes, all16 ? 16 : 1, n_tensors,
+                        a);
 }
 
 // ---------------------------------------------------------------------------
