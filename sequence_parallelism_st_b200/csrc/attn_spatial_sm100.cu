@@ -64,7 +64,8 @@ constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr int W_EPI = 8;                     // epilogue warpgroup: warps 8-11
 constexpr int W_LOAD = 12;                   // TMA producer
 constexpr int W_S0 = 13;                     // S issuer of tile A (tile B: W_S0 + 1); also allocates TMEM
-constexpr int W_PV0 = 15;                    // PV issuer of tile A (tile B: W_PV0 + 1); warps 17-19 idle
+constexpr int W_PV0 = 15;                    // PV issuer of tile A (tile B: W_PV0 + 1)
+constexpr int W_ONES = 17;                   // writes the ones column into V tiles (padded head dims); 18-19 idle
 // Registers per thread after the split (setmaxnreg): the launch gives every
 // thread 96 (640 x 96 = 61440); the two softmax warpgroups take 128, the
 // epilogue 112, and the issuer / loader warpgroups give back down to 56:
@@ -90,6 +91,11 @@ template <int D> struct Cfg {
   // that O += P V is one instruction with N = DPV per 16 keys.
   static constexpr int VW = (D == 72 || D == 80) ? 16 : ((D == 96 || D == 32) ? 32 : 64);
   static constexpr int DPV = ((D + VW - 1) / VW) * VW; // padded head dim of V and O
+  // When V is padded (D = 72 -> 80), column D of every V tile is set to 1.0:
+  // PV then also yields the row sum of the bf16 P in O's column D, and the
+  // softmax need not add up its exponentials.  (Only when O fits one register
+  // group of the epilogue, which reads the sum before normalising.)
+  static constexpr bool ONES = DPV > D && (D + 15) / 16 <= 5;
   static constexpr int VA = DPV / VW;                  // atoms
   static constexpr int VSW = VW * 2;                   // atom row bytes = swizzle span
   static constexpr int VAT = BLOCK_N * VSW;            // bytes of one atom region
@@ -100,7 +106,7 @@ template <int D> struct Cfg {
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;   // K/V ring depth
   // epilogue: two staging buffers per epilogue warp, then the row statistics (m, l) of both tiles
   static constexpr int EPI = 4 * 2 * EPI_BUF + 2 * 2 * BLOCK_M * 4;
-  static constexpr int SMEM = 1024 + 2 * QB * QTILE + NS * (KTILE + VTILE) + EPI + 512;
+  static constexpr int SMEM = 1024 + 2 * QB * QTILE + NS * (KTILE + VTILE) + EPI + 1024;   // + barriers
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(DP <= 128 && DPV <= 128, "head dim too large");
   static_assert(NS >= 4, "ring too shallow");
@@ -388,7 +394,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *mma_done = o_empty + 2;            // 4, one per issuer
   uint64_t *stat_full = mma_done + 4;          // 2, 128 arrivals (softmax threads)
   uint64_t *stat_empty = stat_full + 2;        // 2, 128 arrivals (epilogue threads)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(stat_empty + 2);
+  uint64_t *v_ready = stat_empty + 2;          // NS: ones column written into the V stage
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(v_ready + NS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const st::Geom &g = p.g;
@@ -405,6 +412,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(k_empty + i, 2);
       mbar_init(v_full + i, 1);
       mbar_init(v_empty + i, 2);
+      mbar_init(v_ready + i, 1);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(s_full + i, 1);
@@ -571,7 +579,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t g0 = kv + j;
           const int st = g0 % NS;
           const uint32_t b = step & 1;
-          if (!(ok = mbar_wait(v_full + st, (g0 / NS) & 1, epoch, 6))) break;
+          if (!(ok = mbar_wait((K::ONES ? v_ready : v_full) + st, (g0 / NS) & 1, epoch, 6))) break;
           if (!(ok = mbar_wait(p_full + 2 * X + b, (step >> 1) & 1, epoch, 7 + X))) break;
           if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc & 1) ^ 1, epoch, 9 + X))) break;
           tc_fence_after();
@@ -593,6 +601,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit(mma_done + 2 + X);
       const unsigned long long t0 = globaltimer();
       while (!mbar_try_wait(mma_done + 2 + X, 0) && globaltimer() - t0 < WAIT_NS) {
+      }
+    } else if (K::ONES && warp == W_ONES && n_kv > 0) {
+      // ================= ones column of every V stage =================
+      // Column D lies in atom D / VW at element D % VW of each 64-key row;
+      // the row's 16-byte chunks are permuted by the atom's swizzle.
+      constexpr int A1 = D / K::VW, XB = (D % K::VW) * 2;
+      constexpr int CHK = XB >> 4, WITHIN = XB & 15;
+      bool ok = true;
+      uint32_t kv = 0;
+      for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
+        for (int j = 0; j < n_kv; ++j, ++kv) {
+          const int st = kv % NS;
+          if (lane == 0) ok = mbar_wait(v_full + st, (kv / NS) & 1, epoch, 21);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          __syncwarp();                        // the copy's zero fill of the column is done
+          uint8_t *vt = sV + st * K::VTILE + A1 * K::VAT;
+          for (int r = lane; r < BLOCK_N; r += 32) {
+            const int sw = K::VSW == 128 ? (r & 7) : (K::VSW == 64 ? ((r >> 1) & 3) : ((r >> 2) & 1));
+            *reinterpret_cast<uint16_t *>(vt + r * K::VSW + ((CHK ^ sw) << 4) + WITHIN) = 0x3F80;   // bf16 1.0
+          }
+          fence_async_smem();                  // visible to the tensor core
+          __syncwarp();
+          if (lane == 0) mbar_arrive(v_ready + st);
+        }
       }
     }
   } else if (warp < 8) {
@@ -648,7 +681,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const float corr = need ? ex2_mufu(m - mx) : 1.0f;
             if (need) {
-              l *= corr;
+              if (!K::ONES) l *= corr;         // with the ones column the sum is rescaled with O
               m = mx;
             }
 #pragma unroll 1
@@ -680,14 +713,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               e.x = ex2_mufu(xx.x);
               e.y = ex2_mufu(xx.y);
             }
-            acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], e);
+            if (!K::ONES) acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], e);
             pk[c >> 1] = st::pack_bf16x2(e.x, e.y);
           }
           TMEM_ST16(tS + b * BLOCK_N + (c0 >> 1), pk);
         }
-        const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
-        const float2 a = fadd2(a01, a23);
-        l += a.x + a.y;
+        if (!K::ONES) {
+          const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+          const float2 a = fadd2(a01, a23);
+          l += a.x + a.y;
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + 2 * X + b);
@@ -738,9 +773,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++oc[X];
         tc_fence_after();
         const float m = sStat[(X * 2 + 0) * BLOCK_M + r];
-        const float l = sStat[(X * 2 + 1) * BLOCK_M + r];
+        float l = sStat[(X * 2 + 1) * BLOCK_M + r];   // replaced by O's column D with the ones column
         mbar_arrive(stat_empty + X);
-        const float inv = 1.0f / l;
+        float inv = 1.0f / l;
         const uint32_t tO = tmem + lane_off + TM_O + X * 128;
         constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;    // 16-column chunks holding data
         constexpr int G0 = NCH > 5 ? 4 : NCH;                  // chunks of the first register group
@@ -755,6 +790,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < G0; ++c)
             if (c < nch) TMEM_LD16(tO + (c0 + c) * 16, ov[c]);
           tmem_wait_ld();
+          if (K::ONES) {                       // row sum of the bf16 P, accumulated by PV
+            l = __uint_as_float(ov[D / 16][D % 16]);
+            inv = 1.0f / l;
+          }
           if (c0 + nch == NCH) {
             tc_fence_before();
             mbar_arrive(o_empty + X);          // O of this tile may be overwritten
