@@ -47,7 +47,7 @@ import synth  # noqa: E402
 
 METRIC = "attention TFLOP/s & relayout GB/s on 1 B200, as fraction of bf16/HBM peak"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 11
+LAUNCHES_PER_STEP_BASE = 10           # relayouts 3+1, vmajor 3, merge 1, temporal 1, + R spatial launches
 SPATIAL_SRC = os.path.join(ROOT, "sequence_parallelism_st_b200", "csrc", "attn_spatial_sm100.cu")
 
 
@@ -240,11 +240,10 @@ def kernel_bytes(w, frac_active):
     """Algorithmic HBM bytes per step of each memory-bound kernel group."""
     e = w.elem_bytes
     t = w.B * w.T * w.S * w.C * e               # one [B,T,S,C] tensor
-    rows = w.B * w.T * w.S * w.H
     return {
         "relayout_s2t": 3 * 2 * t,
+        "merge": w.R * (2 * t + w.B * w.T * w.S * w.H * 4) + t,  # fp32 partials + LSE in, bf16 out
         "vmajor": 2 * t + 2 * 2 * frac_active * t,
-        "merge": w.R * (2 * t + rows * 4) + t,  # fp32 partials + LSE in, bf16 out
         "relayout_t2s": 2 * t,
         "temporal": 4 * t,
     }
@@ -390,7 +389,7 @@ def run_ours(args, w, rank, world, dev):
                      "frac": round(achieved / tc_peak, 4), "traffic": kernel_traffic(),
                      "algorithmic_flop_per_launch": w.spatial_flops() / w.R},
         "kernels": kernels,
-        "gpu_launches": LAUNCHES_PER_STEP * n_steps,
+        "gpu_launches": (LAUNCHES_PER_STEP_BASE + w.R) * n_steps,
         "device_status": st.st_status_string(status),
         "clocks": clocks,
         "cpu_baseline": cpu_baseline(w, budget_s=args.cpu_budget) if world == 1 else None,

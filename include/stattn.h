@@ -118,6 +118,27 @@ typedef struct {
 st_status st_attn_spatial(const st_attn_desc *desc, const void *q, const void *k,
                           const void *v, void *o, float *lse, st_stream_t stream);
 
+/* Spatial attention over one KV chunk, merged into the accumulated result of
+ * the chunks before it -- the per-chunk step of ring / Torus attention with
+ * the log-sum-exp merge done in the same kernel [SW Methodology 2]:
+ *     (O_c, lse_c) = the normalised partial and LSE of keys [kv_begin, kv_end)
+ *     M = max(lse_a, lse_c),  w_a = exp(lse_a - M),  w_c = exp(lse_c - M)
+ *     o = (w_a O_a + w_c O_c) / (w_a + w_c),  lse = M + ln(w_a + w_c)
+ * which equals attn_chunk_merge of the two without writing O_c.
+ *   o_acc: fp32 accumulated partial, same element strides as Q (read only).
+ *   lse_acc: fp32 [B, T, H, S] dense LSE of o_acc (-inf: nothing accumulated).
+ *   o: the merged result; fp32 when desc->o_fp32 (or for fp32 Q), and then it
+ *      may be o_acc itself (in place), else Q's dtype (the final output,
+ *      which must not overlap o_acc).
+ *   lse: optional merged LSE, may be lse_acc.
+ * Chain: chunk 0 with st_attn_spatial (o_fp32), chunks 1..R-2 in place with
+ * o_fp32, the last chunk with o in Q's dtype.  Errors as st_attn_spatial;
+ * ST_ERR_NULL for a missing accumulator, ST_ERR_SHAPE for a bf16 o equal to
+ * o_acc.  The pages have no separate API for this fused form. */
+st_status st_attn_spatial_merge(const st_attn_desc *desc, const void *q, const void *k,
+                                const void *v, const float *o_acc, const float *lse_acc,
+                                void *o, float *lse, st_stream_t stream);
+
 /* Temporal attention [SF "三、技术架构"]: for every (b, s, h) in the selected
  * tokens, attention over the T frames of token s.  T <= 64.
  *   lse: optional fp32 [B, S, H, T] dense.

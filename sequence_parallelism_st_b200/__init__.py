@@ -6,7 +6,7 @@ asynchronous on ``torch.cuda.current_stream()`` unless a stream is given.
 Importing this module fails loudly when the library has not been built.
 
 Entry points (same names as the C ABI in include/stattn.h):
-    st_attn_spatial, st_attn_temporal, attn_chunk_merge, ulysses_relayout,
+    st_attn_spatial, st_attn_spatial_merge, st_attn_temporal, attn_chunk_merge, ulysses_relayout,
     vmajor_mask_compact, vmajor_mask_compact_noalloc, vmajor_scatter_rows, vmajor_workspace_bytes,
     st_check_device_status, st_status_string
 """
@@ -58,6 +58,8 @@ _c = {
     "st_abi_version": _proto("st_abi_version", c_int),
     "st_attn_spatial": _proto("st_attn_spatial", c_int, ctypes.POINTER(st_attn_desc), _VP, _VP, _VP, _VP, _VP, _VP),
     "st_attn_temporal": _proto("st_attn_temporal", c_int, ctypes.POINTER(st_attn_desc), _VP, _VP, _VP, _VP, _VP, _VP),
+    "st_attn_spatial_merge": _proto("st_attn_spatial_merge", c_int, ctypes.POINTER(st_attn_desc), _VP, _VP, _VP,
+                                    _VP, _VP, _VP, _VP, _VP),
     "attn_chunk_merge": _proto("attn_chunk_merge", c_int, c_int, ctypes.POINTER(_VP), ctypes.POINTER(_VP), c_ll,
                                c_int, c_int, c_int, _VP, c_int, _VP, _VP),
     "ulysses_relayout": _proto("ulysses_relayout", c_int, c_int, _VP, _VP, c_int, c_int, c_int, c_int, c_int,
@@ -73,7 +75,8 @@ _c = {
     "st_selftest_wait_timeout": _proto("st_selftest_wait_timeout", c_int, _VP),
 }
 
-EXPORTED = ["st_status_string", "st_abi_version", "st_attn_spatial", "st_attn_temporal", "attn_chunk_merge",
+EXPORTED = ["st_status_string", "st_abi_version", "st_attn_spatial", "st_attn_spatial_merge", "st_attn_temporal",
+            "attn_chunk_merge",
             "ulysses_relayout", "vmajor_workspace_bytes", "vmajor_mask_compact", "vmajor_mask_compact_noalloc",
             "vmajor_scatter_rows",
             "st_check_device_status", "st_selftest_wait_timeout"]
@@ -136,6 +139,19 @@ def st_attn_spatial(q, k, v, o, lse=None, *, desc: st_attn_desc | None = None, s
         desc = make_desc(B, T, S, H, D, _dtype_code(q), **kw)
     r = _c["st_attn_spatial"](ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _stream(stream))
     return r if raw else _check(r, "st_attn_spatial")
+
+
+def st_attn_spatial_merge(q, k, v, o_acc, lse_acc, o, lse=None, *, desc: st_attn_desc | None = None, stream=None,
+                          raw=False, **kw):
+    """Spatial attention over one KV chunk merged into the accumulated fp32
+    partial ``o_acc`` and its LSE ``lse_acc``; ``o`` may be ``o_acc`` when the
+    result is fp32 (``o_fp32=1``)."""
+    if desc is None:
+        B, T, S, H, D = q.shape
+        desc = make_desc(B, T, S, H, D, _dtype_code(q), **kw)
+    r = _c["st_attn_spatial_merge"](ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o_acc), _ptr(lse_acc),
+                                    _ptr(o), _ptr(lse), _stream(stream))
+    return r if raw else _check(r, "st_attn_spatial_merge")
 
 
 def st_attn_temporal(q, k, v, o, lse=None, *, desc: st_attn_desc | None = None, stream=None, raw=False, **kw):

@@ -17,8 +17,10 @@ bool strides_aligned(const st::Geom &g, int esize) {
 
 }  // namespace
 
-ST_API st_status st_attn_spatial(const st_attn_desc *desc, const void *q, const void *k, const void *v, void *o,
-                                 float *lse, st_stream_t stream) {
+namespace {
+
+st_status spatial(const st_attn_desc *desc, const void *q, const void *k, const void *v, void *o, float *lse,
+                  const float *o_acc, const float *lse_acc, st_stream_t stream) {
   if (!desc) return ST_ERR_NULL;
   if (!q || !k || !v || !o) return ST_ERR_NULL;
   st::Geom g;
@@ -35,7 +37,7 @@ ST_API st_status st_attn_spatial(const st_attn_desc *desc, const void *q, const 
       return ST_ERR_ALIGN;
     return st::attn_f32(g, false, lo, hi, kv0, kv1, scale, static_cast<const float *>(q),
                         static_cast<const float *>(k), static_cast<const float *>(v), static_cast<float *>(o),
-                        lse, st);
+                        lse, st, o_acc, lse_acc);
   }
   if (!d_supported(g.D)) return ST_ERR_UNSUPPORTED;
   // the tensor-core kernel needs uniformly strided tokens inside a frame
@@ -43,12 +45,30 @@ ST_API st_status st_attn_spatial(const st_attn_desc *desc, const void *q, const 
   if (g.tblk != g.T && g.sb != (long long)(g.T / g.tblk) * g.stb) return ST_ERR_UNSUPPORTED;
   if (!st::is_aligned(q, 16) || !st::is_aligned(k, 16) || !st::is_aligned(v, 16) || !st::is_aligned(o, 16))
     return ST_ERR_ALIGN;
+  if (o_acc && !st::is_aligned(o_acc, 16)) return ST_ERR_ALIGN;
   if (!strides_aligned(g, 2)) return ST_ERR_ALIGN;
   if (g.sblk != g.S) {                       // uniform in fact: collapse to one level
     g.sblk = g.S;
     g.ssb = (long long)g.S * g.ss;
   }
-  return st::attn_spatial_sm100(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, desc->o_fp32, st);
+  return st::attn_spatial_sm100(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, desc->o_fp32, st, o_acc, lse_acc);
+}
+
+}  // namespace
+
+ST_API st_status st_attn_spatial(const st_attn_desc *desc, const void *q, const void *k, const void *v, void *o,
+                                 float *lse, st_stream_t stream) {
+  return spatial(desc, q, k, v, o, lse, nullptr, nullptr, stream);
+}
+
+ST_API st_status st_attn_spatial_merge(const st_attn_desc *desc, const void *q, const void *k, const void *v,
+                                       const float *o_acc, const float *lse_acc, void *o, float *lse,
+                                       st_stream_t stream) {
+  if (!desc || !o_acc || !lse_acc) return ST_ERR_NULL;
+  // in place only for an fp32 result (same element layout as the accumulator)
+  const bool out_f32 = desc->dtype == ST_F32 || desc->o_fp32;
+  if (!out_f32 && static_cast<const void *>(o_acc) == o) return ST_ERR_SHAPE;
+  return spatial(desc, q, k, v, o, lse, o_acc, lse_acc, stream);
 }
 
 ST_API st_status st_attn_temporal(const st_attn_desc *desc, const void *q, const void *k, const void *v, void *o,

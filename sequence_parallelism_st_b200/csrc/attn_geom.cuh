@@ -63,14 +63,16 @@ inline long long geom_extent(const Geom &g) {
 }
 
 // Entry points of the three attention implementations.
+// o_acc / lse_acc (nullable): merge the result with this accumulated partial.
 st_status attn_f32(const Geom &g, bool temporal, int lo, int hi, int kv0, int kv1, float scale,
                    const float *q, const float *k, const float *v, float *o, float *lse,
-                   cudaStream_t s);
+                   cudaStream_t s, const float *o_acc = nullptr, const float *lse_acc = nullptr);
 st_status attn_temporal_bf16(const Geom &g, int lo, int hi, float scale, const void *q,
                              const void *k, const void *v, void *o, float *lse, int o_f32,
                              cudaStream_t s);
 st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, float scale,
                              const void *q, const void *k, const void *v, void *o, float *lse,
-                             int o_f32, cudaStream_t s);
+                             int o_f32, cudaStream_t s, const float *o_acc = nullptr,
+                             const float *lse_acc = nullptr);
 
 }  // namespace st

@@ -18,8 +18,8 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(st::Geom g, int lo, int h
                                                        float scale, const float *__restrict__ q,
                                                        const float *__restrict__ k,
                                                        const float *__restrict__ v,
-                                                       float *__restrict__ o,
-                                                       float *__restrict__ lse) {
+                                                       float *o, float *lse, const float *o_acc,
+                                                       const float *lse_acc) {
   const int L = TEMPORAL ? g.T : g.S;            // query rows per unit
   const int nsel = hi - lo;
   const long long n_units = (long long)g.B * nsel * g.H;
@@ -71,17 +71,27 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(st::Geom g, int lo, int h
       }
       m = mn;
     }
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const long long li = TEMPORAL ? (((long long)b * g.S + sel) * g.H + h) * g.T + row
+                                  : (((long long)b * g.T + sel) * g.H + h) * g.S + row;
+    float val = l > 0.f ? m + logf(l) : -INFINITY;
+    float fa = 0.f, fc = l > 0.f ? 1.f / l : 0.f;
+    if (o_acc) {
+      // merge with the accumulated partial: weights exp(lse - M) of the two
+      const float la = lse_acc[li];
+      const float M = fmaxf(la, val);
+      if (M != -INFINITY) {
+        const float wa = expf(la - M), wc = expf(val - M), sw = wa + wc;
+        fa = wa / sw;
+        fc = l > 0.f ? wc / (sw * l) : 0.f;
+        val = M + logf(sw);
+      }
+    }
 #pragma unroll
     for (int r = 0; r < MAXR; ++r) {
       const int d = lane + 32 * r;
-      if (d < g.D) o[qoff + d] = acc[r] * inv;
+      if (d < g.D) o[qoff + d] = acc[r] * fc + (o_acc && fa != 0.f ? fa * o_acc[qoff + d] : 0.f);
     }
-    if (lse && lane == 0) {
-      const float val = l > 0.f ? m + logf(l) : -INFINITY;
-      if (TEMPORAL) lse[(((long long)b * g.S + sel) * g.H + h) * g.T + row] = val;
-      else lse[(((long long)b * g.T + sel) * g.H + h) * g.S + row] = val;
-    }
+    if (lse && lane == 0) lse[li] = val;
   }
 }
 
@@ -91,15 +101,17 @@ namespace st {
 
 st_status attn_f32(const Geom &g, bool temporal, int lo, int hi, int kv0, int kv1, float scale,
                    const float *q, const float *k, const float *v, float *o, float *lse,
-                   cudaStream_t s) {
+                   cudaStream_t s, const float *o_acc, const float *lse_acc) {
   if (g.D > 32 * MAXR) return ST_ERR_UNSUPPORTED;
   const long long rows = (long long)g.B * (hi - lo) * g.H * (temporal ? g.T : g.S);
   if (rows == 0) return ST_OK;
   const long long want = (rows * 32 + 255) / 256;
   const long long cap = (long long)num_sms() * 32;
   const int grid = int(want < cap ? want : cap);
-  if (temporal) attn_f32_kernel<true><<<grid, 256, 0, s>>>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse);
-  else attn_f32_kernel<false><<<grid, 256, 0, s>>>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse);
+  if (temporal)
+    attn_f32_kernel<true><<<grid, 256, 0, s>>>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_acc, lse_acc);
+  else
+    attn_f32_kernel<false><<<grid, 256, 0, s>>>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_acc, lse_acc);
   return launch_status();
 }
 

@@ -42,6 +42,7 @@
 //     copies and MMAs, frees TMEM and exits; the host reports ST_ERR_TIMEOUT.
 #include <cuda.h>
 #include <math.h>
+#include <string.h>
 
 #include <atomic>
 #include <mutex>
@@ -67,10 +68,10 @@ constexpr int W_S0 = 13;                     // S issuer of tile A (tile B: W_S0
 constexpr int W_PV0 = 15;                    // PV issuer of tile A (tile B: W_PV0 + 1)
 constexpr int W_ONES = 17;                   // writes the ones column into V tiles (padded head dims); 18-19 idle
 // Registers per thread after the split (setmaxnreg): the launch gives every
-// thread 96 (640 x 96 = 61440); the two softmax warpgroups take 128, the
-// epilogue 112, and the issuer / loader warpgroups give back down to 56:
-// 256 x 128 + 128 x 112 + 256 x 56 = 61440.
-constexpr int REG_SOFTMAX = 128, REG_EPI = 112, REG_ISSUE = 56;
+// thread 96 (640 x 96 = 61440); the two softmax warpgroups and the epilogue
+// take 128, and the issuer / loader warpgroups give back down to 48:
+// 256 x 128 + 128 x 128 + 256 x 48 = 61440.
+constexpr int REG_SOFTMAX = 128, REG_EPI = 128, REG_ISSUE = 48;
 static_assert(256 * REG_SOFTMAX + 128 * REG_EPI + 256 * REG_ISSUE <= NUM_THREADS * 96, "register split");
 constexpr int EPI_COLS = 16;                 // O columns per staged store
 constexpr int EPI_BUF = 32 * EPI_COLS * 4;   // bytes of one staging buffer (32 rows, fp32)
@@ -220,6 +221,8 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // at most one committed bulk store may still be reading its shared memory
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// every committed bulk store has finished reading its shared memory
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -295,6 +298,10 @@ struct Params {
   void *o;
   float *lse;
   int o_f32;
+  // merge mode: the result is merged with an accumulated fp32 partial and its
+  // LSE (read per row by the epilogue; o may alias o_acc)
+  const float *o_acc;
+  const float *lse_acc;
   uint32_t epoch;
 };
 
@@ -366,7 +373,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
                    const __grid_constant__ CUtensorMap tk0, const __grid_constant__ CUtensorMap tk1,
                    const __grid_constant__ CUtensorMap tv0, const __grid_constant__ CUtensorMap tv1,
-                   const __grid_constant__ CUtensorMap to, const Params p) {
+                   const __grid_constant__ CUtensorMap to, const __grid_constant__ CUtensorMap tacc,
+                   const Params p) {
   using K = Cfg<D>;
   constexpr int NS = K::NS, QB = K::QB;
   extern __shared__ uint8_t smem_raw[];
@@ -395,7 +403,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *stat_full = mma_done + 4;          // 2, 128 arrivals (softmax threads)
   uint64_t *stat_empty = stat_full + 2;        // 2, 128 arrivals (epilogue threads)
   uint64_t *v_ready = stat_empty + 2;          // NS: ones column written into the V stage
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(v_ready + NS);
+  uint64_t *acc_full = v_ready + NS;           // 4 epilogue warps x 2 staging buffers: o_acc block landed
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const st::Geom &g = p.g;
@@ -426,6 +435,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(stat_full + i, BLOCK_M);
       mbar_init(stat_empty + i, BLOCK_M);
     }
+    for (int i = 0; i < 8; ++i) mbar_init(acc_full + i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == W_S0) {
@@ -747,35 +757,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int qd = warp - W_EPI;               // TMEM lane quadrant
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     uint8_t *stg = sEpi + qd * 2 * EPI_BUF;
-    uint32_t oc[2] = {0, 0}, nst = 0;          // items per tile, bulk stores issued by this warp
+    uint32_t oc0 = 0, oc1 = 0, nst = 0;        // items per tile, bulk stores issued by this warp
+    uint32_t ua = 0;                           // accumulator loads per staging buffer, 16 bits each (merge mode)
     bool ok = true;
     for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
       const Item it = decode(p, x);
+      if (p.o_acc && n_kv > 0) {
+        // the accumulated rows this warp merges at the end of the item: start
+        // moving them into L2 now, while the item's steps run
+        for (int X = 0; X < it.n_qt; ++X) {
+          const int qrow = it.q0 + X * BLOCK_M + qd * 32 + lane;
+          if (qrow < g.S) {
+            const float *src = p.o_acc + g.frame(it.b, it.t) + g.token(qrow) + (long long)it.h * D;
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(uint32_t(D * 4)) : "memory");
+          }
+        }
+      }
       for (int X = 0; X < it.n_qt && ok; ++X) {
         const int r = qd * 32 + lane;
         const int qrow = it.q0 + X * BLOCK_M + r;
         const bool valid = qrow < g.S;
         const long long lse_idx = (((long long)it.b * g.T + it.t) * g.H + it.h) * g.S + qrow;
         if (n_kv == 0) {
-          // empty key range: o = 0, lse = -inf
+          // empty key range: o = 0, lse = -inf (merged: the accumulated result unchanged)
           if (valid) {
             const long long off = g.frame(it.b, it.t) + g.token(qrow) + (long long)it.h * D;
+            const bool acc = p.o_acc && p.lse_acc[lse_idx] != -INFINITY;
             for (int d = 0; d < D; ++d) {
-              if (p.o_f32) static_cast<float *>(p.o)[off + d] = 0.f;
-              else static_cast<uint16_t *>(p.o)[off + d] = 0;
+              const float x = acc ? p.o_acc[off + d] : 0.f;
+              if (p.o_f32) static_cast<float *>(p.o)[off + d] = x;
+              else static_cast<uint16_t *>(p.o)[off + d] = st::f32_to_bf16(x);
             }
-            if (p.lse) p.lse[lse_idx] = -INFINITY;
+            if (p.lse) p.lse[lse_idx] = p.lse_acc ? p.lse_acc[lse_idx] : -INFINITY;
           }
           continue;
         }
-        if (!(ok = mbar_wait(o_full + X, oc[X] & 1, epoch, 17 + X))) break;
-        if (!(ok = mbar_wait(stat_full + X, oc[X] & 1, epoch, 19 + X))) break;
-        ++oc[X];
+        const uint32_t ocx = X ? oc1 : oc0;
+        if (!(ok = mbar_wait(o_full + X, ocx & 1, epoch, 17 + X))) break;
+        if (!(ok = mbar_wait(stat_full + X, ocx & 1, epoch, 19 + X))) break;
+        if (X) ++oc1;
+        else ++oc0;
         tc_fence_after();
         const float m = sStat[(X * 2 + 0) * BLOCK_M + r];
         float l = sStat[(X * 2 + 1) * BLOCK_M + r];   // replaced by O's column D with the ones column
         mbar_arrive(stat_empty + X);
         float inv = 1.0f / l;
+        float fa = 0.f, lse_row = 0.f;         // weight of the accumulated partial; LSE of the row
+        const long long off = valid ? g.frame(it.b, it.t) + g.token(qrow) + (long long)it.h * D : 0;
         const uint32_t tO = tmem + lane_off + TM_O + X * 128;
         constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;    // 16-column chunks holding data
         constexpr int G0 = NCH > 5 ? 4 : NCH;                  // chunks of the first register group
@@ -790,18 +818,104 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < G0; ++c)
             if (c < nch) TMEM_LD16(tO + (c0 + c) * 16, ov[c]);
           tmem_wait_ld();
-          if (K::ONES) {                       // row sum of the bf16 P, accumulated by PV
+          if (K::ONES && grp == 0) {           // row sum of the bf16 P, accumulated by PV
             l = __uint_as_float(ov[D / 16][D % 16]);
             inv = 1.0f / l;
+          }
+          if (grp == 0) {
+            // this chunk's natural-log LSE; merged with the accumulated one when asked:
+            //   w_a = exp(lse_a - M), w_c = exp(lse_c - M), o = (w_a o_a + w_c O / l) / (w_a + w_c)
+            lse_row = (m + log2f(l)) * 0.6931471805599453f;
+            if (p.o_acc) {
+              const float la = valid ? p.lse_acc[lse_idx] : -INFINITY;
+              const float M = fmaxf(la, lse_row);
+              const float wa = expf(la - M), wc = expf(lse_row - M);
+              const float sw = wa + wc;
+              fa = wa / sw;
+              inv = wc / (sw * l);
+              lse_row = M + logf(sw);
+            }
           }
           if (c0 + nch == NCH) {
             tc_fence_before();
             mbar_arrive(o_empty + X);          // O of this tile may be overwritten
           }
+          const int row0 = it.q0 + X * BLOCK_M + qd * 32;
+          if (p.o_acc) {
+            // merge flow: the copy engine brings each 32 x 16 block of o_acc into a
+            // staging buffer (the next block's load overlaps this block's merge),
+            // each lane merges its row there, and the block goes back out with a
+            // bulk tensor store (in place when o is o_acc)
+            const int nb = int(nst & 1);
+            if (lane == 0) {
+              bulk_wait_read0();               // the store that last used a buffer has read it
+              mbar_expect_tx(acc_full + qd * 2 + nb, EPI_BUF);
+              tma_load_5d(stg + nb * EPI_BUF, &tacc, acc_full + qd * 2 + nb, c0 * EPI_COLS, it.h, row0, it.c3, it.c4);
+            }
+#pragma unroll
+            for (int c = 0; c < G0; ++c) {
+              if (c >= nch) break;
+              const int bb = (nb + c) & 1;
+              if (c + 1 < nch && lane == 0) {  // the next block's load overlaps this block's merge
+                bulk_wait_read0();
+                mbar_expect_tx(acc_full + qd * 2 + (bb ^ 1), EPI_BUF);
+                tma_load_5d(stg + (bb ^ 1) * EPI_BUF, &tacc, acc_full + qd * 2 + (bb ^ 1), (c0 + c + 1) * EPI_COLS,
+                            it.h, row0, it.c3, it.c4);
+              }
+              bool got = true;
+              if (lane == 0) got = mbar_wait(acc_full + qd * 2 + bb, (ua >> (16 * bb)) & 1, epoch, 23);
+              ua += 1u << (16 * bb);
+              if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
+                ok = false;
+                break;
+              }
+              __syncwarp();                    // lane 0 saw the block land: order the other lanes after it
+              uint8_t *buf = stg + bb * EPI_BUF;
+              const bool use_acc = fa != 0.f;  // nothing accumulated: the block is not read
+              float *y = reinterpret_cast<float *>(ov[c]);
+#pragma unroll
+              for (int f = 0; f < 4; ++f) {
+                float4 a4 = *reinterpret_cast<const float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4));
+                if (!use_acc) a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                y[4 * f] = fmaf(fa, a4.x, __uint_as_float(ov[c][4 * f]) * inv);
+                y[4 * f + 1] = fmaf(fa, a4.y, __uint_as_float(ov[c][4 * f + 1]) * inv);
+                y[4 * f + 2] = fmaf(fa, a4.z, __uint_as_float(ov[c][4 * f + 2]) * inv);
+                y[4 * f + 3] = fmaf(fa, a4.w, __uint_as_float(ov[c][4 * f + 3]) * inv);
+              }
+              __syncwarp();                    // every row of the block is read before any is overwritten
+              if (p.o_f32) {
+#pragma unroll
+                for (int f = 0; f < 4; ++f)
+                  *reinterpret_cast<float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4)) =
+                      make_float4(y[4 * f], y[4 * f + 1], y[4 * f + 2], y[4 * f + 3]);
+              } else {
+#pragma unroll
+                for (int f = 0; f < 2; ++f) {
+                  uint4 w;
+                  w.x = st::pack_bf16x2(y[8 * f], y[8 * f + 1]);
+                  w.y = st::pack_bf16x2(y[8 * f + 2], y[8 * f + 3]);
+                  w.z = st::pack_bf16x2(y[8 * f + 4], y[8 * f + 5]);
+                  w.w = st::pack_bf16x2(y[8 * f + 6], y[8 * f + 7]);
+                  *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
+                }
+              }
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                if (row0 < g.S) tma_store_5d(&to, buf, (c0 + c) * EPI_COLS, it.h, row0, it.c3, it.c4);
+                bulk_commit();
+              }
+            }
+            nst += nch;
+            if (!ok) break;
+          } else {
 #pragma unroll
           for (int c = 0; c < G0; ++c, ++nst) {
             if (c >= nch) break;
             uint8_t *buf = stg + (nst & 1) * EPI_BUF;
+            float *y = reinterpret_cast<float *>(ov[c]);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(ov[c][e]) * inv;
             if (lane == 0) bulk_wait_read1();  // the store that used this buffer has read it
             __syncwarp();
             if (p.o_f32) {
@@ -809,17 +923,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int f = 0; f < 4; ++f)
                 *reinterpret_cast<float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4)) =
-                    make_float4(__uint_as_float(ov[c][4 * f]) * inv, __uint_as_float(ov[c][4 * f + 1]) * inv,
-                                __uint_as_float(ov[c][4 * f + 2]) * inv, __uint_as_float(ov[c][4 * f + 3]) * inv);
+                    make_float4(y[4 * f], y[4 * f + 1], y[4 * f + 2], y[4 * f + 3]);
             } else {
               // 32-byte rows, 32B swizzle: 16-byte chunk f of row r at f ^ ((r >> 2) & 1)
 #pragma unroll
               for (int f = 0; f < 2; ++f) {
                 uint4 w;
-                w.x = st::pack_bf16x2(__uint_as_float(ov[c][8 * f]) * inv, __uint_as_float(ov[c][8 * f + 1]) * inv);
-                w.y = st::pack_bf16x2(__uint_as_float(ov[c][8 * f + 2]) * inv, __uint_as_float(ov[c][8 * f + 3]) * inv);
-                w.z = st::pack_bf16x2(__uint_as_float(ov[c][8 * f + 4]) * inv, __uint_as_float(ov[c][8 * f + 5]) * inv);
-                w.w = st::pack_bf16x2(__uint_as_float(ov[c][8 * f + 6]) * inv, __uint_as_float(ov[c][8 * f + 7]) * inv);
+                w.x = st::pack_bf16x2(y[8 * f], y[8 * f + 1]);
+                w.y = st::pack_bf16x2(y[8 * f + 2], y[8 * f + 3]);
+                w.z = st::pack_bf16x2(y[8 * f + 4], y[8 * f + 5]);
+                w.w = st::pack_bf16x2(y[8 * f + 6], y[8 * f + 7]);
                 *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
               }
             }
@@ -828,13 +941,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (lane == 0) {
               // a block wholly past the last row stores nothing, but still
               // commits a (empty) group so the buffer accounting stays in step
-              const int row0 = it.q0 + X * BLOCK_M + qd * 32;
               if (row0 < g.S) tma_store_5d(&to, buf, (c0 + c) * EPI_COLS, it.h, row0, it.c3, it.c4);
               bulk_commit();
             }
           }
+          }
         }
-        if (valid && p.lse) p.lse[lse_idx] = (m + log2f(l)) * 0.6931471805599453f;
+        if (!ok) break;
+        if (valid && p.lse) p.lse[lse_idx] = lse_row;
       }
     }
     if (lane == 0) bulk_wait_all();
@@ -928,16 +1042,23 @@ std::atomic<uint32_t> g_epoch{0};
 
 template <int D>
 st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, float scale, const void *q,
-                         const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s) {
+                         const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
+                         const float *o_acc, const float *lse_acc) {
   using K = Cfg<D>;
   const int tmode = g.tblk != g.T ? 1 : 0;
-  CUtensorMap m[7];
+  CUtensorMap m[8];
   const int c1 = K::C1 ? K::C1 : 16;
   if (!make_map(&m[0], q, g, tmode, K::C0, K::SW0, BLOCK_M) || !make_map(&m[1], q, g, tmode, c1, c1 * 2, BLOCK_M) ||
       !make_map(&m[2], k, g, tmode, K::C0, K::SW0, BLOCK_N) || !make_map(&m[3], k, g, tmode, c1, c1 * 2, BLOCK_N) ||
       !make_map(&m[4], v, g, tmode, K::VW, K::VSW, BLOCK_N) || !make_map(&m[5], v, g, tmode, K::VW, K::VSW, BLOCK_N) ||
       !make_map(&m[6], o, g, tmode, EPI_COLS, EPI_COLS * (o_f32 ? 4 : 2), 32, o_f32))
     return ST_ERR_CUDA;
+  // fp32 accumulator blocks of the merge mode (unused otherwise)
+  if (o_acc) {
+    if (!make_map(&m[7], o_acc, g, tmode, EPI_COLS, EPI_COLS * 4, 32, 1)) return ST_ERR_CUDA;
+  } else {
+    memset(&m[7], 0, sizeof(m[7]));
+  }
   Params p;
   p.g = g;
   p.lo = lo;
@@ -951,6 +1072,8 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   p.o = o;
   p.lse = lse;
   p.o_f32 = o_f32;
+  p.o_acc = o_acc;
+  p.lse_acc = lse_acc;
   p.epoch = g_epoch.fetch_add(1) + 1;
   const long long items = (long long)p.q_blocks * g.H * g.B * p.n_frames;
   if (items <= 0) return ST_OK;
@@ -969,7 +1092,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
     regs_ok = fa.numRegs * NUM_THREADS >= 256 * REG_SOFTMAX + 128 * REG_EPI + 256 * REG_ISSUE ? 1 : 0;
   }
   if (!regs_ok) return ST_ERR_UNSUPPORTED;
-  return st::launch_pdl(kern, ctas, NUM_THREADS, K::SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], p);
+  return st::launch_pdl(kern, ctas, NUM_THREADS, K::SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], p);
 }
 
 }  // namespace
@@ -987,15 +1110,16 @@ unsigned int read_and_clear_attn_error(cudaStream_t stream, cudaError_t *err) {
 }
 
 st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, float scale, const void *q,
-                             const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s) {
+                             const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
+                             const float *o_acc, const float *lse_acc) {
   if (hi <= lo) return ST_OK;
   switch (g.D) {
-    case 32: return launch_spatial<32>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s);
-    case 64: return launch_spatial<64>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s);
-    case 72: return launch_spatial<72>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s);
-    case 80: return launch_spatial<80>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s);
-    case 96: return launch_spatial<96>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s);
-    case 128: return launch_spatial<128>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s);
+    case 32: return launch_spatial<32>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
+    case 64: return launch_spatial<64>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
+    case 72: return launch_spatial<72>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
+    case 80: return launch_spatial<80>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
+    case 96: return launch_spatial<96>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
+    case 128: return launch_spatial<128>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
   }
   return ST_ERR_UNSUPPORTED;
 }
