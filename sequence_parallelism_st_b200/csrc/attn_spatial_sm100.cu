@@ -33,6 +33,13 @@
 //     softmax, round once to bf16 (or keep fp32 partials), stage 32 x 16
 //     blocks in shared memory and write them with bulk tensor stores, plus the
 //     natural-log LSE.  The softmax warps go straight on to the next item.
+//   * Merge mode (st_attn_spatial_merge): for head dims up to 80 the epilogue
+//     seeds O in TMEM with the accumulated fp32 partial of the tile's next
+//     item right after reading this item's O, PV accumulates onto it, and the
+//     softmax starts from the partial's LSE (as running max) with row sum 1,
+//     so the online softmax simply continues; the first item of each tile is
+//     seeded before anything else.  Larger head dims merge in the epilogue,
+//     loading 32 x 16 accumulator blocks with TMA into the staging buffers.
 //   * Head dims 32..128: Q and K split D into a 64-wide 128B-swizzled chunk and
 //     a remainder chunk padded to 16/32/64 (zero-filled by TMA beyond D); V is
 //     stored as column atoms so that PV is one instruction of N = padded D.
@@ -97,6 +104,10 @@ template <int D> struct Cfg {
   // softmax need not add up its exponentials.  (Only when O fits one register
   // group of the epilogue, which reads the sum before normalising.)
   static constexpr bool ONES = DPV > D && (D + 15) / 16 <= 5;
+  // Merge mode seeds the TMEM accumulator O with the accumulated partial when
+  // the epilogue can hold a row of it in registers (at most 5 column chunks);
+  // larger head dims merge in the epilogue instead.
+  static constexpr bool MINIT = (D + 15) / 16 <= 5;
   static constexpr int VA = DPV / VW;                  // atoms
   static constexpr int VSW = VW * 2;                   // atom row bytes = swizzle span
   static constexpr int VAT = BLOCK_N * VSW;            // bytes of one atom region
@@ -449,6 +460,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t epoch = p.epoch;
+  const bool minit = K::MINIT && p.o_acc != nullptr;   // merge by seeding O (see the epilogue)
   // barriers and TMEM are set up: let the next kernel of the stream be
   // scheduled, then wait for the previous one before any global access
   pdl_trigger();
@@ -591,7 +603,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b = step & 1;
           if (!(ok = mbar_wait((K::ONES ? v_ready : v_full) + st, (g0 / NS) & 1, epoch, 6))) break;
           if (!(ok = mbar_wait(p_full + 2 * X + b, (step >> 1) & 1, epoch, 7 + X))) break;
-          if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc & 1) ^ 1, epoch, 9 + X))) break;
+          // O free (plain) or O seeded with the accumulated partial (merge mode)
+          if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc & 1) ^ (minit ? 0u : 1u), epoch, 9 + X))) break;
           tc_fence_after();
           const uint32_t d = tmem + TM_O + X * 128;
           const uint32_t pa = tmem + X * 2 * BLOCK_N + b * BLOCK_N;   // P (bf16 pairs) over the S columns
@@ -599,7 +612,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   #pragma unroll
           for (int kk = 0; kk < BLOCK_N / 16; ++kk)
             mma_ts(d, pa + kk * 8, sdesc_c<K::VAT, 8 * K::VSW, layout_of(K::VSW)>(va + kk * 16 * K::VSW), IDPV,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+                   (j > 0 || kk > 0 || minit) ? 1u : 0u);
           tc_commit(pv_done + 2 * X + b);
           tc_commit(v_empty + st);
         }
@@ -654,6 +667,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Item it = decode(p, x);
       if (X >= it.n_qt) continue;
       float m = -INFINITY, l = 0.f;
+      if (minit) {
+        // continue the online softmax from the accumulated partial: its LSE in
+        // log2 units is the running max, and its normalised O (seeded into
+        // TMEM by the epilogue) has row sum 1
+        const int qrow = it.q0 + X * BLOCK_M + r;
+        const float la = qrow < g.S ? p.lse_acc[(((long long)it.b * g.T + it.t) * g.H + it.h) * g.S + qrow] : -INFINITY;
+        if (la != -INFINITY) {
+          m = la * 1.4426950408889634f;
+          l = 1.f;
+        }
+      }
       for (int j = 0; j < n_kv; ++j, ++gs) {
         const uint32_t b = gs & 1;
         if (!(ok = mbar_wait(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
@@ -681,13 +705,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         const float mx = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]), mxp[3]) * sl2;
-        if (j == 0) {
+        if (j == 0 && !minit) {
           m = mx;
         } else {
           const bool need = mx > m + 8.0f;
           if (__any_sync(0xffffffffu, need)) {
-            // O holds PV up to step gs-1: wait for that PV, then rescale in TMEM
-            if (!(ok = mbar_wait(pv_done + 2 * X + ((gs - 1) & 1), ((gs - 1) >> 1) & 1, epoch, 15 + X))) break;
+            // O holds PV up to step gs-1 (or, at the first step of a merge, the
+            // seeded partial): wait for it, then rescale in TMEM
+            if (j == 0) {
+              if (!(ok = mbar_wait(o_empty + X, oc & 1, epoch, 25 + X))) break;
+            } else if (!(ok = mbar_wait(pv_done + 2 * X + ((gs - 1) & 1), ((gs - 1) >> 1) & 1, epoch, 15 + X))) {
+              break;
+            }
             tc_fence_after();
             const float corr = need ? ex2_mufu(m - mx) : 1.0f;
             if (need) {
@@ -760,6 +789,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t oc0 = 0, oc1 = 0, nst = 0;        // items per tile, bulk stores issued by this warp
     uint32_t ua = 0;                           // accumulator loads per staging buffer, 16 bits each (merge mode)
     bool ok = true;
+    if (K::MINIT && minit && n_kv > 0) {
+      // seed O of each tile's first item before waiting on anything: a tile
+      // whose first PV cannot start would stall the shared K/V ring and with
+      // it the other tile
+      constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;
+      constexpr int LC = K::ONES ? D / 16 : 0;
+      for (int X = 0; X < 2; ++X) {
+        int x0 = blockIdx.x;
+        while (x0 < n_items && X >= decode(p, x0).n_qt) x0 += gridDim.x;
+        if (x0 >= n_items) continue;
+        const Item jt = decode(p, x0);
+        const int jrow = jt.q0 + X * BLOCK_M + qd * 32 + lane;
+        const bool jv = jrow < g.S;
+        const bool has = jv && p.lse_acc[(((long long)jt.b * g.T + jt.t) * g.H + jt.h) * g.S + jrow] != -INFINITY;
+        const float *ap = p.o_acc + (jv ? g.frame(jt.b, jt.t) + g.token(jrow) + (long long)jt.h * D : 0);
+        const uint32_t tO = tmem + lane_off + TM_O + X * 128;
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          uint32_t a[16];
+#pragma unroll
+          for (int f = 0; f < 4; ++f) {
+            float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (has && k * 16 + 4 * f < D) a4 = *reinterpret_cast<const float4 *>(ap + k * 16 + 4 * f);
+            a[4 * f] = __float_as_uint(a4.x);
+            a[4 * f + 1] = __float_as_uint(a4.y);
+            a[4 * f + 2] = __float_as_uint(a4.z);
+            a[4 * f + 3] = __float_as_uint(a4.w);
+          }
+          if (K::ONES && k == LC) a[D % 16] = __float_as_uint(has ? 1.f : 0.f);
+          TMEM_ST16(tO + k * 16, a);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(o_empty + X);
+      }
+    }
     for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
       const Item it = decode(p, x);
       if (p.o_acc && n_kv > 0) {
@@ -793,6 +858,108 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           continue;
         }
         const uint32_t ocx = X ? oc1 : oc0;
+        if (K::MINIT && minit) {
+          // ---- merge by seeding O: after reading O of this item, write the
+          // accumulated partial of this tile's next item into the same TMEM
+          // columns (its row sum 1 in the ones column), so that item's PV
+          // accumulates onto it and its softmax continues from the partial's LSE
+          constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;
+          constexpr int LC = K::ONES ? D / 16 : 0;            // chunk holding the ones column
+          const uint32_t tO = tmem + lane_off + TM_O + X * 128;
+          // where the accumulated row of item xx lives, and whether it holds anything
+#define ST_ACC_ROW(xx, ap, has)                                                                              \
+  const float *ap;                                                                                           \
+  bool has;                                                                                                  \
+  {                                                                                                          \
+    const Item jt = decode(p, (xx));                                                                         \
+    const int jrow = jt.q0 + X * BLOCK_M + r;                                                                \
+    const bool jv = jrow < g.S;                                                                              \
+    has = jv && p.lse_acc[(((long long)jt.b * g.T + jt.t) * g.H + jt.h) * g.S + jrow] != -INFINITY;          \
+    ap = p.o_acc + (jv ? g.frame(jt.b, jt.t) + g.token(jrow) + (long long)jt.h * D : 0);                     \
+  }
+          // 16 columns of an accumulated row (zero where nothing is accumulated;
+          // the ones column carries its row sum 1)
+#define ST_ACC_CHUNK(ap, has, k, a)                                                                          \
+  _Pragma("unroll") for (int f = 0; f < 4; ++f) {                                                            \
+    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);                                                             \
+    if ((has) && (k) * 16 + 4 * f < D) a4 = *reinterpret_cast<const float4 *>((ap) + (k) * 16 + 4 * f);     \
+    a[4 * f] = __float_as_uint(a4.x);                                                                        \
+    a[4 * f + 1] = __float_as_uint(a4.y);                                                                    \
+    a[4 * f + 2] = __float_as_uint(a4.z);                                                                    \
+    a[4 * f + 3] = __float_as_uint(a4.w);                                                                    \
+  }                                                                                                          \
+  if (K::ONES && (k) == LC) a[D % 16] = __float_as_uint((has) ? 1.f : 0.f);
+          int xn = x + gridDim.x;              // this tile's next item
+          while (xn < n_items && X >= decode(p, xn).n_qt) xn += gridDim.x;
+          const bool has_next = xn < n_items;
+          ST_ACC_ROW(has_next ? xn : x, apn, hasn)
+          hasn = hasn && has_next;
+          if (hasn)                            // bring the row into L2 while this item computes
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(apn), "r"(uint32_t(D * 4)) : "memory");
+          if (!(ok = mbar_wait(o_full + X, ocx & 1, epoch, 17 + X))) break;
+          if (!(ok = mbar_wait(stat_full + X, ocx & 1, epoch, 19 + X))) break;
+          if (X) ++oc1;
+          else ++oc0;
+          tc_fence_after();
+          const float m = sStat[(X * 2 + 0) * BLOCK_M + r];
+          float l = sStat[(X * 2 + 1) * BLOCK_M + r];
+          mbar_arrive(stat_empty + X);
+          if (K::ONES) {                       // the row sum, from the ones column
+            uint32_t lv;
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(lv) : "r"(tO + D));
+            tmem_wait_ld();
+            l = __uint_as_float(lv);
+          }
+          const float inv = 1.0f / l;
+          const int row0 = it.q0 + X * BLOCK_M + qd * 32;
+          uint32_t an[16];                     // seed chunk k, loaded one chunk ahead
+          if (has_next) { ST_ACC_CHUNK(apn, hasn, 0, an) }
+#pragma unroll
+          for (int k = 0; k < NCH; ++k, ++nst) {
+            uint32_t ov[16];
+            TMEM_LD16(tO + k * 16, ov);
+            tmem_wait_ld();
+            if (has_next) {
+              TMEM_ST16(tO + k * 16, an);      // this chunk of O is read: overwrite it with the seed
+              if (k + 1 < NCH) { ST_ACC_CHUNK(apn, hasn, k + 1, an) }
+            }
+            uint8_t *buf = stg + (nst & 1) * EPI_BUF;
+            if (lane == 0) bulk_wait_read1();
+            __syncwarp();
+            if (p.o_f32) {
+#pragma unroll
+              for (int f = 0; f < 4; ++f)
+                *reinterpret_cast<float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4)) =
+                    make_float4(__uint_as_float(ov[4 * f]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
+                                __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
+            } else {
+#pragma unroll
+              for (int f = 0; f < 2; ++f) {
+                uint4 w;
+                w.x = st::pack_bf16x2(__uint_as_float(ov[8 * f]) * inv, __uint_as_float(ov[8 * f + 1]) * inv);
+                w.y = st::pack_bf16x2(__uint_as_float(ov[8 * f + 2]) * inv, __uint_as_float(ov[8 * f + 3]) * inv);
+                w.z = st::pack_bf16x2(__uint_as_float(ov[8 * f + 4]) * inv, __uint_as_float(ov[8 * f + 5]) * inv);
+                w.w = st::pack_bf16x2(__uint_as_float(ov[8 * f + 6]) * inv, __uint_as_float(ov[8 * f + 7]) * inv);
+                *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
+              }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (row0 < g.S) tma_store_5d(&to, buf, k * EPI_COLS, it.h, row0, it.c3, it.c4);
+              bulk_commit();
+            }
+          }
+#undef ST_ACC_ROW
+#undef ST_ACC_CHUNK
+          if (has_next) {                      // the next item's seed is in TMEM
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(o_empty + X);
+          }
+          if (valid && p.lse) p.lse[lse_idx] = (m + log2f(l)) * 0.6931471805599453f;
+          continue;
+        }
         if (!(ok = mbar_wait(o_full + X, ocx & 1, epoch, 17 + X))) break;
         if (!(ok = mbar_wait(stat_full + X, ocx & 1, epoch, 19 + X))) break;
         if (X) ++oc1;
@@ -826,7 +993,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // this chunk's natural-log LSE; merged with the accumulated one when asked:
             //   w_a = exp(lse_a - M), w_c = exp(lse_c - M), o = (w_a o_a + w_c O / l) / (w_a + w_c)
             lse_row = (m + log2f(l)) * 0.6931471805599453f;
-            if (p.o_acc) {
+            if (!K::MINIT && p.o_acc) {
               const float la = valid ? p.lse_acc[lse_idx] : -INFINITY;
               const float M = fmaxf(la, lse_row);
               const float wa = expf(la - M), wc = expf(lse_row - M);
@@ -841,7 +1008,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_arrive(o_empty + X);          // O of this tile may be overwritten
           }
           const int row0 = it.q0 + X * BLOCK_M + qd * 32;
-          if (p.o_acc) {
+          if (!K::MINIT && p.o_acc) {
             // merge flow: the copy engine brings each 32 x 16 block of o_acc into a
             // staging buffer (the next block's load overlaps this block's merge),
             // each lane merges its row there, and the block goes back out with a
