@@ -145,7 +145,7 @@ constexpr float kP2 = 0.2426111251115799f, kP3 = 0.0551716685295105f;
 
 // Of every 8 consecutive score pairs, this many take ex2_poly and the rest the
 // MUFU, so the two pipes share the exponentials of the softmax.
-constexpr int kPolyPairs = 3;
+constexpr int kPolyPairs = 2;
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
