@@ -257,6 +257,20 @@ st_status vmajor_scatter_rows(const int *idx, const int *count, long long n_toke
                               void *const *dst_cache, int n_tensors,
                               void *const *packed, st_stream_t stream);
 
+/* vmajor_mask_compact and vmajor_scatter_rows (without `packed`) in one call
+ * [CC "V-Major" section]: the pass that decides a token is active also copies
+ * its rows of every src tensor into dst_cache, so the cache update reads no
+ * index list and the mask pass's rows are still in cache.  Arguments,
+ * results and errors as the two calls (src[t] and dst_cache[t] are dense
+ * [n_tokens, C] of dtype, 16-byte aligned; src may include v_cur).  Same
+ * mask, idx, count and caches as the two calls, bit for bit. */
+st_status vmajor_mask_compact_scatter(const void *v_cur, const void *v_prev,
+                                      long long n_tokens, int C, st_dtype dtype, float tau,
+                                      int force_all, unsigned char *mask, int *idx, int *count,
+                                      float *l1_out, void *workspace, size_t workspace_bytes,
+                                      const void *const *src, void *const *dst_cache,
+                                      int n_tensors, st_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that
  * bounded waits set.  Returns ST_ERR_TIMEOUT if a wait ran out since the last
  * call, ST_ERR_CUDA if the stream reports an error, else ST_OK. */

@@ -7,7 +7,8 @@ Importing this module fails loudly when the library has not been built.
 
 Entry points (same names as the C ABI in include/stattn.h):
     st_attn_spatial, st_attn_spatial_merge, st_attn_temporal, attn_chunk_merge, ulysses_relayout,
-    vmajor_mask_compact, vmajor_mask_compact_noalloc, vmajor_scatter_rows, vmajor_workspace_bytes,
+    vmajor_mask_compact, vmajor_mask_compact_noalloc, vmajor_mask_compact_scatter, vmajor_scatter_rows,
+    vmajor_workspace_bytes,
     st_check_device_status, st_status_string
 """
 from __future__ import annotations
@@ -69,6 +70,9 @@ _c = {
                                   _VP, _VP, _VP, _VP, _VP, c_size_t, _VP),
     "vmajor_mask_compact_noalloc": _proto("vmajor_mask_compact_noalloc", c_int, _VP, _VP, c_ll, c_int, c_int,
                                           c_float, c_int, _VP, _VP, _VP, _VP, _VP),
+    "vmajor_mask_compact_scatter": _proto("vmajor_mask_compact_scatter", c_int, _VP, _VP, c_ll, c_int, c_int,
+                                          c_float, c_int, _VP, _VP, _VP, _VP, _VP, c_size_t,
+                                          ctypes.POINTER(_VP), ctypes.POINTER(_VP), c_int, _VP),
     "vmajor_scatter_rows": _proto("vmajor_scatter_rows", c_int, _VP, _VP, c_ll, c_int, c_int,
                                   ctypes.POINTER(_VP), ctypes.POINTER(_VP), c_int, ctypes.POINTER(_VP), _VP),
     "st_check_device_status": _proto("st_check_device_status", c_int, _VP),
@@ -78,7 +82,7 @@ _c = {
 EXPORTED = ["st_status_string", "st_abi_version", "st_attn_spatial", "st_attn_spatial_merge", "st_attn_temporal",
             "attn_chunk_merge",
             "ulysses_relayout", "vmajor_workspace_bytes", "vmajor_mask_compact", "vmajor_mask_compact_noalloc",
-            "vmajor_scatter_rows",
+            "vmajor_scatter_rows", "vmajor_mask_compact_scatter",
             "st_check_device_status", "st_selftest_wait_timeout"]
 
 
@@ -208,6 +212,20 @@ def vmajor_mask_compact_noalloc(v_cur, v_prev, tau, mask, idx, count, force_all=
                                           1 if force_all else 0, _ptr(mask), _ptr(idx), _ptr(count),
                                           _ptr(l1_out), _stream(stream))
     return r if raw else _check(r, "vmajor_mask_compact_noalloc")
+
+
+def vmajor_mask_compact_scatter(v_cur, v_prev, tau, mask, idx, count, workspace, src, dst_cache, force_all=False,
+                                l1_out=None, *, stream=None, raw=False):
+    """vmajor_mask_compact and the cache update of the active tokens' rows in one call."""
+    n, C = v_cur.shape[0], v_cur[0].numel()
+    nt = len(src)
+    sp = (c_void_p * nt)(*[t.data_ptr() for t in src])
+    dp = (c_void_p * nt)(*[t.data_ptr() for t in dst_cache])
+    r = _c["vmajor_mask_compact_scatter"](_ptr(v_cur), _ptr(v_prev), n, C, _dtype_code(v_cur), float(tau),
+                                          1 if force_all else 0, _ptr(mask), _ptr(idx), _ptr(count), _ptr(l1_out),
+                                          _ptr(workspace), workspace.numel() * workspace.element_size(), sp, dp, nt,
+                                          _stream(stream))
+    return r if raw else _check(r, "vmajor_mask_compact_scatter")
 
 
 def vmajor_scatter_rows(idx, count, src, dst_cache, packed=None, *, stream=None, raw=False):

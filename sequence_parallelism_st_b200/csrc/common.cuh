@@ -49,6 +49,16 @@ inline st_status launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// A pointer the compiler cannot see through: loads through the result depend
+// on this point of the program.  Every input read after pdl_wait() goes
+// through it, since loads through const __restrict__ pointers (and __ldg) are
+// taken as invariant and could otherwise be scheduled before the wait.
+template <typename T>
+__device__ __forceinline__ T *after_wait(T *p) {
+  asm volatile("" : "+l"(p));
+  return p;
+}
+
 // SM count of the current device (cached per device ordinal).
 int num_sms();
 

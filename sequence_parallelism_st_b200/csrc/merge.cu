@@ -48,6 +48,12 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_row
   const int n = R > 0 ? R : nc;
   st::pdl_trigger();
   st::pdl_wait();
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if (c < n) {
+      a.o[c] = st::after_wait(a.o[c]);
+      a.lse[c] = st::after_wait(a.lse[c]);
+    }
   const I total = n_rows_h * D4;
   const I stride = (I)gridDim.x * blockDim.x;
   for (I f0 = (I)blockIdx.x * blockDim.x + threadIdx.x; f0 < total; f0 += stride * U) {

@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(256) relayout_copy(Map m, int G, int log2G,
   using V = typename VecT<VEC>::t;
   st::pdl_trigger();
   st::pdl_wait();
+  in = st::after_wait(in);
   const long long seg_vecs = m.seg_bytes / VEC;
   const long long chunk = (long long)G * U;
   const long long n_chunks = (seg_vecs + chunk - 1) / chunk;
@@ -206,6 +207,8 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   st::pdl_trigger();
   st::pdl_wait();
+  in = st::after_wait(in);
+  gamma = st::after_wait(gamma);
   for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
   if (lane == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");

@@ -3,7 +3,8 @@
 // ascending list of active tokens, and the cache update for active tokens.
 //
 // Design.  vmajor_mask_compact is two launches and no atomics, so its output
-// is deterministic:
+// is deterministic (vmajor_mask_compact_scatter is the same two launches, the
+// first also copying the rows of every active token into the caches):
 //   1. l1_mask: a warp streams the [C] rows of two tokens at a time with
 //      16-byte loads (all of a lane's loads issued before any arithmetic), accumulates
 //      |cur - prev| in fp32, reduces over the warp with a fixed butterfly
@@ -24,20 +25,66 @@ constexpr int VMAX = 12;          // 16-byte vectors per lane per tensor in flig
 constexpr int CTILE = 2048;       // tokens per CTA of the compaction pass
 constexpr int ROUNDS = CTILE / THREADS;  // 32-token ballots per warp
 
-template <typename T>
-__global__ void __launch_bounds__(THREADS) l1_mask(const char *__restrict__ cur,
+// One warp per active row: copies each tensor's row to its cache (and to the
+// packed message buffer when present).  The (tensor, vector) pairs of a row
+// are enumerated together and a lane loads NB of them before storing any, so
+// the copy of a row costs one memory round trip, not one per vector.
+struct ScatterArgs {
+  const char *src[8];
+  char *dst[8];
+  char *packed[8];
+};
+
+// The warp copies row `row` of every tensor (16-byte vectors, rv per row):
+// the (tensor, vector) pairs are enumerated together and a lane loads NB of
+// them before storing any, so a row costs one memory round trip.
+__device__ __forceinline__ void copy_row_warp(const ScatterArgs &a, int n_tensors, long long row, int rv,
+                                              long long packed_row, int lane) {
+  constexpr int NB = 10;
+  const long long row_bytes = (long long)rv * 16;
+  const int total = rv * n_tensors;
+  for (int j0 = 0; j0 < total; j0 += 32 * NB) {
+    uint4 v[NB];
+#pragma unroll
+    for (int u = 0; u < NB; ++u) {
+      const int j = j0 + u * 32 + lane;
+      if (j < total) {
+        const int t = j / rv, k = j - t * rv;
+        // after_wait: this kernel may start before the one that wrote src has finished
+        v[u] = __ldg(reinterpret_cast<const uint4 *>(st::after_wait(a.src[t]) + row * row_bytes) + k);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < NB; ++u) {
+      const int j = j0 + u * 32 + lane;
+      if (j < total) {
+        const int t = j / rv, k = j - t * rv;
+        reinterpret_cast<uint4 *>(a.dst[t] + row * row_bytes)[k] = v[u];
+        if (packed_row >= 0 && a.packed[t]) reinterpret_cast<uint4 *>(a.packed[t] + packed_row * row_bytes)[k] = v[u];
+      }
+    }
+  }
+}
+
+// SCATTER: the warp that decides a token is active also copies its rows of
+// the scatter tensors into their caches (the fused mask + cache update).
+template <typename T, bool SCATTER = false>
+__global__ void __launch_bounds__(THREADS, 2) l1_mask(const char *__restrict__ cur,
                                                    const char *__restrict__ prev, long long n,
                                                    int row_vecs, float tau, int force_all,
                                                    unsigned char *__restrict__ mask,
                                                    float *__restrict__ l1_out,
-                                                   int *__restrict__ tile_count) {
+                                                   int *__restrict__ tile_count, ScatterArgs sa = ScatterArgs{},
+                                                   int n_tensors = 0, int scatter_vecs = 0) {
   constexpr int EPV = 16 / int(sizeof(T));
-  constexpr int TPW = 2;                         // tokens of a warp in flight together
-  constexpr int VM = VMAX / TPW;                 // vectors per lane per token per tensor in flight
+  constexpr int TPW = SCATTER ? 1 : 2;           // tokens of a warp in flight together
+  constexpr int VM = VMAX / 2;                   // vectors per lane per token per tensor in flight
   __shared__ int warp_cnt[THREADS / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   st::pdl_trigger();
   st::pdl_wait();
+  cur = st::after_wait(cur);
+  prev = st::after_wait(prev);
   int active = 0;
   for (int r = warp; r < TILE; r += TPW * (THREADS / 32)) {
     long long tok[TPW];
@@ -86,12 +133,13 @@ __global__ void __launch_bounds__(THREADS) l1_mask(const char *__restrict__ cur,
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
       if (tok[i] < n) {
-        const int m = (force_all || acc[i] > tau) ? 1 : 0;
+        const int m = (force_all || acc[i] > tau) ? 1 : 0;   // the same on every lane (butterfly sum)
         if (lane == 0) {
           mask[tok[i]] = (unsigned char)m;
           if (l1_out) l1_out[tok[i]] = acc[i];
         }
         active += m;
+        if (SCATTER && m) copy_row_warp(sa, n_tensors, tok[i], scatter_vecs, -1, lane);
       }
     }
   }
@@ -115,6 +163,8 @@ __global__ void __launch_bounds__(THREADS) compact(const unsigned char *__restri
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   st::pdl_trigger();
   st::pdl_wait();
+  mask = st::after_wait(mask);
+  tile_count = st::after_wait(tile_count);
   const long long first_tile = (long long)blockIdx.x * (CTILE / TILE);
   int part = 0;
   for (long long t = threadIdx.x; t < first_tile; t += THREADS) part += tile_count[t];
@@ -153,23 +203,14 @@ __global__ void __launch_bounds__(THREADS) compact(const unsigned char *__restri
   }
 }
 
-// One warp per active row: copies each tensor's row to its cache (and to the
-// packed message buffer when present).  The (tensor, vector) pairs of a row
-// are enumerated together and a lane loads NB of them before storing any, so
-// the copy of a row costs one memory round trip, not one per vector.
-struct ScatterArgs {
-  const char *src[8];
-  char *dst[8];
-  char *packed[8];
-};
-
 __global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
                                                     const int *__restrict__ count, long long n,
                                                     long long row_bytes, int vec, int n_tensors,
                                                     ScatterArgs a) {
-  constexpr int NB = 10;
   st::pdl_trigger();
   st::pdl_wait();
+  idx = st::after_wait(idx);
+  count = st::after_wait(count);
   const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long cnt = *count;
@@ -178,28 +219,7 @@ __global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
     const long long row = idx[i];
     if (row < 0 || row >= n) continue;
     if (vec == 16) {
-      const int rv = int(row_bytes / 16);
-      const int total = rv * n_tensors;
-      for (int j0 = 0; j0 < total; j0 += 32 * NB) {
-        uint4 v[NB];
-#pragma unroll
-        for (int u = 0; u < NB; ++u) {
-          const int j = j0 + u * 32 + lane;
-          if (j < total) {
-            const int t = j / rv, k = j - t * rv;
-            v[u] = __ldg(reinterpret_cast<const uint4 *>(a.src[t] + row * row_bytes) + k);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < NB; ++u) {
-          const int j = j0 + u * 32 + lane;
-          if (j < total) {
-            const int t = j / rv, k = j - t * rv;
-            reinterpret_cast<uint4 *>(a.dst[t] + row * row_bytes)[k] = v[u];
-            if (a.packed[t]) reinterpret_cast<uint4 *>(a.packed[t] + i * row_bytes)[k] = v[u];
-          }
-        }
-      }
+      copy_row_warp(a, n_tensors, row, int(row_bytes / 16), i, lane);
     } else {
       for (int t = 0; t < n_tensors; ++t) {
         const char *s = a.src[t] + row * row_bytes;
@@ -243,9 +263,47 @@ ST_API st_status vmajor_mask_compact(const void *v_cur, const void *v_prev, long
   const char *cur = static_cast<const char *>(v_cur), *prev = static_cast<const char *>(v_prev);
   st_status st = dtype == ST_BF16
                      ? st::launch_pdl(l1_mask<uint16_t>, int(tiles), THREADS, 0, s, cur, prev, n_tokens, row_vecs,
-                                      tau, force_all, mask, l1_out, tile_count)
+                                      tau, force_all, mask, l1_out, tile_count, ScatterArgs{}, 0, 0)
                      : st::launch_pdl(l1_mask<float>, int(tiles), THREADS, 0, s, cur, prev, n_tokens, row_vecs, tau,
-                                      force_all, mask, l1_out, tile_count);
+                                      force_all, mask, l1_out, tile_count, ScatterArgs{}, 0, 0);
+  if (st != ST_OK) return st;
+  const int ctas = int((n_tokens + CTILE - 1) / CTILE);
+  return st::launch_pdl(compact, ctas, THREADS, 0, s, static_cast<const unsigned char *>(mask), n_tokens, ctas,
+                        static_cast<const int *>(tile_count), idx, count);
+}
+
+ST_API st_status vmajor_mask_compact_scatter(const void *v_cur, const void *v_prev, long long n_tokens, int C,
+                                             st_dtype dtype, float tau, int force_all, unsigned char *mask, int *idx,
+                                             int *count, float *l1_out, void *workspace, size_t workspace_bytes,
+                                             const void *const *src, void *const *dst_cache, int n_tensors,
+                                             st_stream_t stream) {
+  if (!v_cur || !v_prev || !mask || !idx || !count || !src || !dst_cache) return ST_ERR_NULL;
+  if (n_tokens <= 0 || C <= 0 || n_tokens >= (1LL << 31)) return ST_ERR_SHAPE;
+  if (n_tensors < 1 || n_tensors > 8) return ST_ERR_SHAPE;
+  if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_DTYPE;
+  const int esize = dtype == ST_F32 ? 4 : 2;
+  if ((C * esize) % 16 || !st::is_aligned(v_cur, 16) || !st::is_aligned(v_prev, 16)) return ST_ERR_ALIGN;
+  if (!workspace) return ST_ERR_NULL;
+  if (workspace_bytes < vmajor_workspace_bytes(n_tokens)) return ST_ERR_SHAPE;
+  const int row_vecs = C * esize / 16;
+  if ((long long)row_vecs * n_tensors >= (1LL << 31)) return ST_ERR_SHAPE;
+  ScatterArgs a = {};
+  for (int t = 0; t < n_tensors; ++t) {
+    if (!src[t] || !dst_cache[t]) return ST_ERR_NULL;
+    if (!st::is_aligned(src[t], 16) || !st::is_aligned(dst_cache[t], 16)) return ST_ERR_ALIGN;
+    a.src[t] = static_cast<const char *>(src[t]);
+    a.dst[t] = static_cast<char *>(dst_cache[t]);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long tiles = n_tiles_of(n_tokens);
+  if (tiles > 0x7fffffffLL) return ST_ERR_SHAPE;
+  int *tile_count = static_cast<int *>(workspace);
+  const char *cur = static_cast<const char *>(v_cur), *prev = static_cast<const char *>(v_prev);
+  st_status st = dtype == ST_BF16
+                     ? st::launch_pdl(l1_mask<uint16_t, true>, int(tiles), THREADS, 0, s, cur, prev, n_tokens,
+                                      row_vecs, tau, force_all, mask, l1_out, tile_count, a, n_tensors, row_vecs)
+                     : st::launch_pdl(l1_mask<float, true>, int(tiles), THREADS, 0, s, cur, prev, n_tokens, row_vecs,
+                                      tau, force_all, mask, l1_out, tile_count, a, n_tensors, row_vecs);
   if (st != ST_OK) return st;
   const int ctas = int((n_tokens + CTILE - 1) / CTILE);
   return st::launch_pdl(compact, ctas, THREADS, 0, s, static_cast<const unsigned char *>(mask), n_tokens, ctas,

@@ -211,6 +211,43 @@ def test_vmajor_scatter_rows(st):
         assert np.array_equal(f64(packed[:cnt_ref]), oracle.pack_rows(idx_ref, cnt_ref, cur))
 
 
+@pytest.mark.parametrize("name,f", [("vmajor_2304px", 0.5), ("vmajor_2304px", 0.1), ("opensora_low", 0.5),
+                                    ("tiny", 0.5)])
+def test_vmajor_mask_compact_scatter_fused(st, name, f):
+    """The fused call gives the mask, indices, count and caches of the oracle,
+    and the same bits as vmajor_mask_compact + vmajor_scatter_rows."""
+    w = synth.BY_NAME[name]
+    n, C = w.B * w.T * w.S, w.C
+    cur_v, prev_v = synth.vmajor_pair(w, n, C)
+    cur_k, prev_k = synth.vmajor_pair(w, n, C, prev="kprev", noise="knoise")
+    tau = taus()[name][str(f)]["tau"]
+    mask_ref = oracle.change_mask(oracle.l1_change(cur_v, prev_v), tau)
+    idx_ref, cnt_ref = oracle.compact(mask_ref)
+    cv, pvd, ck = cur_v.to(DEV), prev_v.to(DEV), cur_k.to(DEV)
+    ws = torch.zeros(st.vmajor_workspace_bytes(n), dtype=torch.uint8, device=DEV)
+    outs = []
+    for fused in (True, False):
+        mask = torch.full((n,), 7, dtype=torch.uint8, device=DEV)
+        idx = torch.full((n,), -1, dtype=torch.int32, device=DEV)
+        count = torch.zeros(1, dtype=torch.int32, device=DEV)
+        kc, vc = prev_k.to(DEV), prev_v.to(DEV)
+        if fused:
+            st.vmajor_mask_compact_scatter(cv, pvd, tau, mask, idx, count, ws, [ck, cv], [kc, vc])
+        else:
+            st.vmajor_mask_compact(cv, pvd, tau, mask, idx, count, ws)
+            st.vmajor_scatter_rows(idx, count, [ck, cv], [kc, vc])
+        torch.cuda.synchronize()
+        outs.append((mask.cpu(), idx.cpu(), count.cpu(), kc.cpu(), vc.cpu()))
+    mask, idx, count, kc, vc = outs[0]
+    assert count.item() == cnt_ref
+    assert np.array_equal(mask.numpy(), mask_ref)
+    assert np.array_equal(idx.numpy()[:cnt_ref], idx_ref)
+    assert np.array_equal(f64(kc), oracle.scatter_rows(idx_ref, cnt_ref, cur_k, prev_k))
+    assert np.array_equal(f64(vc), oracle.scatter_rows(idx_ref, cnt_ref, cur_v, prev_v))
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+
+
 # ------------------------------------------------------------------ merge
 @pytest.mark.parametrize("R,out_dtype", [(1, torch.float32), (2, torch.bfloat16), (3, torch.float32),
                                          (8, torch.bfloat16), (16, torch.float32)])
