@@ -1,0 +1,66 @@
+"""The bench step's kernels launched back to back (each may start while the
+previous one finishes, through programmatic dependent launch) must give the
+same bits as the same step with a device synchronisation after every call.
+Catches reads that run ahead of a producer kernel; the per-kernel parity tests
+synchronise after each call and cannot see them."""
+import os
+import sys
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def st():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    import sequence_parallelism_st_b200 as st
+    return st
+
+
+class _Synced:
+    """The binding with a device synchronisation after every call."""
+
+    def __init__(self, mod):
+        self._m = mod
+
+    def __getattr__(self, name):
+        f = getattr(self._m, name)
+        if not callable(f) or name in ("make_desc", "vmajor_workspace_bytes"):
+            return f
+
+        def call(*a, **k):
+            r = f(*a, **k)
+            torch.cuda.synchronize()
+            return r
+        return call
+
+
+def outputs(stp):
+    return [t.detach().clone() for t in (stp.ox, stp.ot, stp.kc, stp.vc, stp.mask, stp.idx, stp.count, stp.oy)]
+
+
+@pytest.mark.parametrize("name", ["opensora_low"])
+def test_step_chain_matches_synchronised(st, name):
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    w = synth.BY_NAME[name]
+    stp = bench.Step(st, w, "cuda")
+    stp.reset_caches()
+    stp.st = _Synced(st)
+    stp.run()
+    torch.cuda.synchronize()
+    ref = outputs(stp)
+    stp.st = st
+    for rep in range(10):
+        stp.reset_caches()
+        stp.run()
+        torch.cuda.synchronize()
+        got = outputs(stp)
+        for i, (a, b) in enumerate(zip(got, ref)):
+            assert torch.equal(a, b), f"{name}: output {i} differs from the synchronised step (repeat {rep})"
+    assert st.st_check_device_status() == st.ST_OK
