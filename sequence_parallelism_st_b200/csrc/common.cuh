@@ -67,6 +67,26 @@ int num_sms();
 unsigned int read_and_clear_attn_error(cudaStream_t stream, cudaError_t *err);
 unsigned int read_and_clear_relayout_error(cudaStream_t stream, cudaError_t *err);
 
+// Division of 0 <= n < 2^31 by a divisor fixed for the launch, as a multiply
+// and a shift: with l = ceil(log2 d) and m = ceil(2^(31+l) / d) (< 2^32),
+// floor(n / d) = (n * m) >> (31 + l) exactly (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", theorem 4.2: the
+// error m d - 2^(31+l) is below 2^l).  Integer division by a runtime value
+// would otherwise take a reciprocal on the special-function pipe and about a
+// dozen more instructions.
+struct FastDiv {
+  uint32_t d, m, shift;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  const unsigned long long num = 1ull << (31 + l);
+  return FastDiv{d, uint32_t((num + d - 1) / d), 31 + l};
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+  return uint32_t((unsigned long long)n * f.m >> f.shift);
+}
+
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
 
 // Round to nearest even; NaN stays NaN.

@@ -26,15 +26,29 @@ struct MergeArgs {
   const float *lse[MAXC];
 };
 
+// Divisors of the row decode, as multiply-shift pairs (32-bit indexing only).
+struct MergeDivs {
+  st::FastDiv d4, h, s;
+};
+
 // Element f of the output (four channels) -> index of its LSE row.
 template <typename I>
-__device__ __forceinline__ I lse_index(I f, int D4, int H, int S) {
-  const I rh = f / D4;                   // (unit, s, h) row index
-  const I row = rh / H;                  // unit * S + s
-  const int h = int(rh - row * H);
-  const I unit = row / S;
-  const int s = int(row - unit * S);
-  return (unit * H + h) * S + s;
+__device__ __forceinline__ I lse_index(I f, int D4, int H, int S, const MergeDivs &dv) {
+  if constexpr (sizeof(I) == 4) {
+    const uint32_t rh = st::fdiv(uint32_t(f), dv.d4);   // (unit, s, h) row index
+    const uint32_t row = st::fdiv(rh, dv.h);            // unit * S + s
+    const uint32_t h = rh - row * uint32_t(H);
+    const uint32_t unit = st::fdiv(row, dv.s);
+    const uint32_t s = row - unit * uint32_t(S);
+    return I((unit * uint32_t(H) + h) * uint32_t(S) + s);
+  } else {
+    const I rh = f / D4;
+    const I row = rh / H;
+    const int h = int(rh - row * H);
+    const I unit = row / S;
+    const int s = int(row - unit * S);
+    return (unit * H + h) * S + s;
+  }
 }
 
 // I is the index type (32-bit when every index fits).  Each thread handles
@@ -42,7 +56,8 @@ __device__ __forceinline__ I lse_index(I f, int D4, int H, int S) {
 // vectors each) before any arithmetic, so U * 2R loads are in flight.
 template <bool BF16, int R, typename I>
 __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_rows_h, int S, int H, int D4,
-                                                    void *__restrict__ o_out, float *__restrict__ lse_out) {
+                                                    void *__restrict__ o_out, float *__restrict__ lse_out,
+                                                    MergeDivs dv) {
   constexpr int NC = R > 0 ? R : MAXC;
   constexpr int U = R > 0 && R <= 4 ? 2 : 1;
   const int n = R > 0 ? R : nc;
@@ -64,7 +79,7 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_row
     for (int u = 0; u < U; ++u) {
       const I f = f0 + (I)u * stride;
       if (f < total) {
-        li[u] = lse_index<I>(f, D4, H, S);
+        li[u] = lse_index<I>(f, D4, H, S, dv);
 #pragma unroll
         for (int c = 0; c < NC; ++c)
           if (c < n) {
@@ -112,7 +127,11 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeArgs a, int nc, I n_row
       } else {
         reinterpret_cast<float4 *>(o_out)[f] = acc;
       }
-      if (lse_out && f % D4 == 0) lse_out[li[u]] = M != -INFINITY ? M + logf(sum) : -INFINITY;
+      if (lse_out) {
+        const bool first = sizeof(I) == 4 ? uint32_t(f) - st::fdiv(uint32_t(f), dv.d4) * uint32_t(D4) == 0
+                                          : f % D4 == 0;
+        if (first) lse_out[li[u]] = M != -INFINITY ? M + logf(sum) : -INFINITY;
+      }
     }
   }
 }
@@ -121,12 +140,13 @@ template <bool BF16, typename I>
 st_status launch(const MergeArgs &a, int nc, long long rows_h, int S, int H, int D4, void *o, float *lse,
                  int grid, cudaStream_t s) {
   const I rh = (I)rows_h;
+  const MergeDivs dv{st::make_fastdiv(uint32_t(D4)), st::make_fastdiv(uint32_t(H)), st::make_fastdiv(uint32_t(S))};
   switch (nc) {
-    case 1: return st::launch_pdl(merge_kernel<BF16, 1, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
-    case 2: return st::launch_pdl(merge_kernel<BF16, 2, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
-    case 4: return st::launch_pdl(merge_kernel<BF16, 4, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
-    case 8: return st::launch_pdl(merge_kernel<BF16, 8, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
-    default: return st::launch_pdl(merge_kernel<BF16, 0, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse);
+    case 1: return st::launch_pdl(merge_kernel<BF16, 1, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse, dv);
+    case 2: return st::launch_pdl(merge_kernel<BF16, 2, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse, dv);
+    case 4: return st::launch_pdl(merge_kernel<BF16, 4, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse, dv);
+    case 8: return st::launch_pdl(merge_kernel<BF16, 8, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse, dv);
+    default: return st::launch_pdl(merge_kernel<BF16, 0, I>, grid, 256, 0, s, a, nc, rh, S, H, D4, o, lse, dv);
   }
 }
 

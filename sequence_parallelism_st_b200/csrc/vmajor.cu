@@ -39,7 +39,7 @@ struct ScatterArgs {
 // the (tensor, vector) pairs are enumerated together and a lane loads NB of
 // them before storing any, so a row costs one memory round trip.
 __device__ __forceinline__ void copy_row_warp(const ScatterArgs &a, int n_tensors, long long row, int rv,
-                                              long long packed_row, int lane) {
+                                              const st::FastDiv &frv, long long packed_row, int lane) {
   constexpr int NB = 10;
   const long long row_bytes = (long long)rv * 16;
   const int total = rv * n_tensors;
@@ -49,7 +49,7 @@ __device__ __forceinline__ void copy_row_warp(const ScatterArgs &a, int n_tensor
     for (int u = 0; u < NB; ++u) {
       const int j = j0 + u * 32 + lane;
       if (j < total) {
-        const int t = j / rv, k = j - t * rv;
+        const int t = int(st::fdiv(uint32_t(j), frv)), k = j - t * rv;
         // after_wait: this kernel may start before the one that wrote src has finished
         v[u] = __ldg(reinterpret_cast<const uint4 *>(st::after_wait(a.src[t]) + row * row_bytes) + k);
       }
@@ -58,7 +58,7 @@ __device__ __forceinline__ void copy_row_warp(const ScatterArgs &a, int n_tensor
     for (int u = 0; u < NB; ++u) {
       const int j = j0 + u * 32 + lane;
       if (j < total) {
-        const int t = j / rv, k = j - t * rv;
+        const int t = int(st::fdiv(uint32_t(j), frv)), k = j - t * rv;
         reinterpret_cast<uint4 *>(a.dst[t] + row * row_bytes)[k] = v[u];
         if (packed_row >= 0 && a.packed[t]) reinterpret_cast<uint4 *>(a.packed[t] + packed_row * row_bytes)[k] = v[u];
       }
@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(THREADS, 2) l1_mask(const char *__restrict__ c
                                                    unsigned char *__restrict__ mask,
                                                    float *__restrict__ l1_out,
                                                    int *__restrict__ tile_count, ScatterArgs sa = ScatterArgs{},
-                                                   int n_tensors = 0, int scatter_vecs = 0) {
+                                                   int n_tensors = 0, int scatter_vecs = 0,
+                                                   st::FastDiv frv = st::FastDiv{1, 1u << 31, 31}) {
   constexpr int EPV = 16 / int(sizeof(T));
   constexpr int TPW = SCATTER ? 1 : 2;           // tokens of a warp in flight together
   constexpr int VM = VMAX / 2;                   // vectors per lane per token per tensor in flight
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(THREADS, 2) l1_mask(const char *__restrict__ c
           if (l1_out) l1_out[tok[i]] = acc[i];
         }
         active += m;
-        if (SCATTER && m) copy_row_warp(sa, n_tensors, tok[i], scatter_vecs, -1, lane);
+        if (SCATTER && m) copy_row_warp(sa, n_tensors, tok[i], scatter_vecs, frv, -1, lane);
       }
     }
   }
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(THREADS) compact(const unsigned char *__restri
 __global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
                                                     const int *__restrict__ count, long long n,
                                                     long long row_bytes, int vec, int n_tensors,
-                                                    ScatterArgs a) {
+                                                    ScatterArgs a, st::FastDiv frv) {
   st::pdl_trigger();
   st::pdl_wait();
   idx = st::after_wait(idx);
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
     const long long row = idx[i];
     if (row < 0 || row >= n) continue;
     if (vec == 16) {
-      copy_row_warp(a, n_tensors, row, int(row_bytes / 16), i, lane);
+      copy_row_warp(a, n_tensors, row, int(row_bytes / 16), frv, i, lane);
     } else {
       for (int t = 0; t < n_tensors; ++t) {
         const char *s = a.src[t] + row * row_bytes;
@@ -263,9 +264,9 @@ ST_API st_status vmajor_mask_compact(const void *v_cur, const void *v_prev, long
   const char *cur = static_cast<const char *>(v_cur), *prev = static_cast<const char *>(v_prev);
   st_status st = dtype == ST_BF16
                      ? st::launch_pdl(l1_mask<uint16_t>, int(tiles), THREADS, 0, s, cur, prev, n_tokens, row_vecs,
-                                      tau, force_all, mask, l1_out, tile_count, ScatterArgs{}, 0, 0)
+                                      tau, force_all, mask, l1_out, tile_count, ScatterArgs{}, 0, 0, st::make_fastdiv(1))
                      : st::launch_pdl(l1_mask<float>, int(tiles), THREADS, 0, s, cur, prev, n_tokens, row_vecs, tau,
-                                      force_all, mask, l1_out, tile_count, ScatterArgs{}, 0, 0);
+                                      force_all, mask, l1_out, tile_count, ScatterArgs{}, 0, 0, st::make_fastdiv(1));
   if (st != ST_OK) return st;
   const int ctas = int((n_tokens + CTILE - 1) / CTILE);
   return st::launch_pdl(compact, ctas, THREADS, 0, s, static_cast<const unsigned char *>(mask), n_tokens, ctas,
@@ -301,9 +302,11 @@ ST_API st_status vmajor_mask_compact_scatter(const void *v_cur, const void *v_pr
   const char *cur = static_cast<const char *>(v_cur), *prev = static_cast<const char *>(v_prev);
   st_status st = dtype == ST_BF16
                      ? st::launch_pdl(l1_mask<uint16_t, true>, int(tiles), THREADS, 0, s, cur, prev, n_tokens,
-                                      row_vecs, tau, force_all, mask, l1_out, tile_count, a, n_tensors, row_vecs)
+                                      row_vecs, tau, force_all, mask, l1_out, tile_count, a, n_tensors, row_vecs,
+                                      st::make_fastdiv(uint32_t(row_vecs)))
                      : st::launch_pdl(l1_mask<float, true>, int(tiles), THREADS, 0, s, cur, prev, n_tokens, row_vecs,
-                                      tau, force_all, mask, l1_out, tile_count, a, n_tensors, row_vecs);
+                                      tau, force_all, mask, l1_out, tile_count, a, n_tensors, row_vecs,
+                                      st::make_fastdiv(uint32_t(row_vecs)));
   if (st != ST_OK) return st;
   const int ctas = int((n_tokens + CTILE - 1) / CTILE);
   return st::launch_pdl(compact, ctas, THREADS, 0, s, static_cast<const unsigned char *>(mask), n_tokens, ctas,
@@ -333,7 +336,7 @@ ST_API st_status vmajor_scatter_rows(const int *idx, const int *count, long long
   const long long cap = (long long)st::num_sms() * 16;
   const int grid = int(want < cap ? want : cap);
   return st::launch_pdl(scatter_rows, grid, 256, 0, s, idx, count, n_tokens, row_bytes, all16 ? 16 : 1, n_tensors,
-                        a);
+                        a, st::make_fastdiv(uint32_t(all16 ? row_bytes / 16 : 1)));
 }
 
 // ---------------------------------------------------------------------------
