@@ -224,6 +224,105 @@ class Step:
         st.st_attn_temporal(d["q"], d["k"], d["v"], self.ot, None, desc=self.tdesc)
         self._mark("temporal", False)
 
+    # ------------------------------------------------------------ overlapped schedule
+    def setup_overlap(self, n_slices, att_sms):
+        """Buffers and streams of the chunk-and-overlap schedule: the step is cut
+        into n_slices ranges of temporally sharded shards; the attention of one
+        range runs on att_sms SMs (high-priority stream) while the memory-bound
+        steps of the neighbouring ranges run on the others (low-priority stream)."""
+        w = self.w
+        assert w.P % n_slices == 0
+        self.n_sl, self.att_sms = n_slices, att_sms
+        self.s_att = torch.cuda.Stream(priority=-8)     # mapped to the highest priority the device has
+        self.s_mem = torch.cuda.Stream(priority=0)
+        n_sl_tok = self.n // n_slices
+        self.counts = torch.zeros(n_slices, dtype=torch.int32, device=self.dev)
+        T = w.T
+        self.sdesc_sl = [[self.st.make_desc(1, T, w.S, w.H, w.D, self.st.ST_BF16, kv_begin=c * w.S // w.R,
+                                            kv_end=(c + 1) * w.S // w.R, o_fp32=1, n_slices=n_slices, slice=i)
+                          for c in range(w.R)] for i in range(n_slices)]
+        self.n_sl_tok = n_sl_tok
+
+    def _prep(self, i):
+        """S->T relayout of shard range i and the V-Major steps of its tokens."""
+        st, w, d = self.st, self.w, self.d
+        P, B, T, S, C, D = w.P, w.B, w.T, w.S, w.C, w.D
+        per = P // self.n_sl
+        sh = (i * per, (i + 1) * per)
+        st.ulysses_relayout_range("S2T", d["v"], self.vy, P, B, T, S, C, w.n_t, w.n_s, shards=sh)
+        st.ulysses_relayout_range("S2T", d["k"], self.ky, P, B, T, S, C, w.n_t, w.n_s, shards=sh,
+                                  rms_gamma=self.gamma, rms_head_dim=D, rms_eps=w.rms_eps)
+        st.ulysses_relayout_range("S2T", d["q"], self.qy, P, B, T, S, C, w.n_t, w.n_s, shards=sh,
+                                  rms_gamma=self.gamma, rms_head_dim=D, rms_eps=w.rms_eps)
+        t0, t1 = i * self.n_sl_tok, (i + 1) * self.n_sl_tok
+        rows = lambda t: t.view(self.n, C)[t0:t1]
+        cnt = self.counts[i:i + 1]
+        st.vmajor_mask_compact(rows(self.vy), rows(self.vprev_y), self.tau, self.mask[t0:t1],
+                               self.idx[t0:t1], cnt, self.ws)
+        st.vmajor_scatter_rows(self.idx[t0:t1], cnt, [rows(self.ky), rows(self.vy)], [rows(self.kc), rows(self.vc)])
+
+    def _post(self, i):
+        """Merge of the KV-chunk partials of shard range i and its T->S relayout."""
+        st, w = self.st, self.w
+        P, B, T, S, C, D, H = w.P, w.B, w.T, w.S, w.C, w.D, w.H
+        per = P // self.n_sl
+        f0, f1 = i * T // self.n_sl, (i + 1) * T // self.n_sl
+        e0, e1 = f0 * S * C, f1 * S * C
+        l0, l1 = f0 * H * S, f1 * H * S
+        st.attn_chunk_merge([p[e0:e1] for p in self.parts], [x[l0:l1] for x in self.lses], B * (f1 - f0), S, H, D,
+                            self.oy[e0:e1])
+        st.ulysses_relayout_range("T2S", self.oy, self.ox, P, B, T, S, C, w.n_t, w.n_s, shards=(i * per, (i + 1) * per))
+
+    def run_overlap(self):
+        """One step on the overlapped schedule; ordered after, and followed by,
+        the current stream's work."""
+        st, w, d = self.st, self.w, self.d
+        main = torch.cuda.current_stream()
+        n_sl, mem_sms = self.n_sl, self.st_num_sms() - self.att_sms
+        start = torch.cuda.Event()
+        start.record(main)
+        self.s_att.wait_event(start)
+        self.s_mem.wait_event(start)
+        e_prep = [torch.cuda.Event() for _ in range(n_sl)]
+        e_att = [torch.cuda.Event() for _ in range(n_sl)]
+        e_go = [torch.cuda.Event() for _ in range(n_sl)]
+        try:
+            with torch.cuda.stream(self.s_mem):
+                st.st_set_sm_budget(0)                  # nothing else runs yet
+                self._prep(0)
+                e_prep[0].record(self.s_mem)
+            for i in range(n_sl):
+                with torch.cuda.stream(self.s_att):
+                    self.s_att.wait_event(e_prep[i])
+                    e_go[i].record(self.s_att)          # attention of range i may start
+                    st.st_set_sm_budget(self.att_sms)
+                    for c in range(w.R):
+                        st.st_attn_spatial(self.qy, self.kc, self.vc, self.parts[c], self.lses[c],
+                                           desc=self.sdesc_sl[i][c])
+                    e_att[i].record(self.s_att)
+                with torch.cuda.stream(self.s_mem):
+                    self.s_mem.wait_event(e_go[i])      # let the attention take its SMs first
+                    st.st_set_sm_budget(mem_sms)
+                    if i + 1 < n_sl:
+                        self._prep(i + 1)
+                        e_prep[i + 1].record(self.s_mem)
+                    if i == 0:
+                        st.st_attn_temporal(d["q"], d["k"], d["v"], self.ot, None, desc=self.tdesc)
+                    if i >= 1:
+                        self.s_mem.wait_event(e_att[i - 1])
+                        self._post(i - 1)
+            with torch.cuda.stream(self.s_mem):
+                self.s_mem.wait_event(e_att[n_sl - 1])
+                st.st_set_sm_budget(0)
+                self._post(n_sl - 1)
+        finally:
+            st.st_set_sm_budget(0)
+        main.wait_stream(self.s_mem)
+        main.wait_stream(self.s_att)
+
+    def st_num_sms(self):
+        return torch.cuda.get_device_properties(self.dev).multi_processor_count
+
     def kernel_times(self):
         out = {}
         for name, evs in self.ev.items():
@@ -252,14 +351,21 @@ def kernel_bytes(w, frac_active):
 def run_ours(args, w, rank, world, dev):
     import sequence_parallelism_st_b200 as st
     stp = Step(st, w, dev)
+    if args.schedule == "overlap":
+        stp.setup_overlap(args.slices, args.att_sms)
+        step_fn = stp.run_overlap
+        launches = (3 + 2 + w.R + 2) * args.slices + 1
+    else:
+        step_fn = stp.run
+        launches = LAUNCHES_PER_STEP_BASE + w.R
     pk, pk_src = peaks()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
-        stp.run()
+        step_fn()
     torch.cuda.synchronize()
     if st.st_check_device_status() != st.ST_OK:
         raise RuntimeError("device status not OK after warm-up")
-    active = int(stp.count.item())
+    active = int(stp.count.item()) if args.schedule == "serial" else int(stp.counts.sum().item())
     # ---- timed: device time of exactly K steps, L2 flushed between steps outside the events
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -271,7 +377,7 @@ def run_ours(args, w, rank, world, dev):
         for i in range(args.steps):
             flush.zero_()
             starts[i].record()
-            stp.run()
+            step_fn()
             ends[i].record()
         torch.cuda.synchronize()
     if world > 1:
@@ -327,7 +433,7 @@ def run_ours(args, w, rank, world, dev):
                 comp.wait_event(ev_out[i - 2])           # set j's outputs already copied down
             stp.d = d_sets[j]
             stp.ox, stp.ot = o_sets[j]
-            stp.run()
+            step_fn()
             ev_comp[i].record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[i])
@@ -381,7 +487,8 @@ def run_ours(args, w, rank, world, dev):
         "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "H": w.H, "D": w.D, "P": w.P,
                    "N_T": w.n_t, "N_S": w.n_s, "kv_chunks": w.R, "vmajor_active": round(frac_active, 4),
                    "parallelism": f"replicas{world}", "l2": "flushed between timed steps (256 MiB write, "
-                   "outside the step events)"},
+                   "outside the step events)", "schedule": args.schedule if args.schedule == "serial" else
+                   f"overlap: {args.slices} shard ranges, attention on {args.att_sms} SMs"},
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(statistics.mean(e2e_ms), 5)},
         "roofline": {"bound": "tensor", "kernel": "st_attn_spatial", "achieved": round(achieved, 2),
@@ -389,7 +496,7 @@ def run_ours(args, w, rank, world, dev):
                      "frac": round(achieved / tc_peak, 4), "traffic": kernel_traffic(),
                      "algorithmic_flop_per_launch": w.spatial_flops() / w.R},
         "kernels": kernels,
-        "gpu_launches": (LAUNCHES_PER_STEP_BASE + w.R) * n_steps,
+        "gpu_launches": launches * n_steps,
         "device_status": st.st_status_string(status),
         "clocks": clocks,
         "cpu_baseline": cpu_baseline(w, budget_s=args.cpu_budget) if world == 1 else None,
@@ -462,6 +569,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="opensora_low")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--schedule", choices=["serial", "overlap"], default="serial",
+                    help="overlap: shard ranges of the step on two streams (attention / memory-bound steps)")
+    ap.add_argument("--slices", type=int, default=4, help="shard ranges of the overlap schedule")
+    ap.add_argument("--att-sms", type=int, default=120, help="SMs of the attention stream in the overlap schedule")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -197,6 +197,23 @@ st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *out,
                            int j1, const float *rms_gamma, int rms_head_dim,
                            float rms_eps, st_stream_t stream);
 
+/* ulysses_relayout restricted to the temporally sharded shards q0 <= q < q1
+ * of y as well: S2T writes only y shards q0..q1-1 (every row of them inside
+ * the block range), T2S writes only the x rows whose frames come from those
+ * y shards.  Each y shard's frames are contiguous in y, so a shard range is a
+ * contiguous set of frames for the attention, V-Major and merge calls that
+ * follow -- the unit of an intra-GPU chunk-and-overlap schedule in which the
+ * exchange of one shard range runs while another range is attended [SF "四、
+ * 核心创新" intra-layer schedule].  Any partition of (0, P) into ranges gives
+ * the same bytes as one call.  (q0, q1) = (0, P) is ulysses_relayout; the
+ * sequence/head modes accept only that.  ST_ERR_SHAPE for an empty or
+ * out-of-range shard range. */
+st_status ulysses_relayout_range(st_relayout_mode mode, const void *in, void *out,
+                                 int elem_bytes, int P, int B, int T_or_N, int S_or_H,
+                                 int C_or_D, int n_t, int n_s, int i0, int i1, int j0,
+                                 int j1, int q0, int q1, const float *rms_gamma,
+                                 int rms_head_dim, float rms_eps, st_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * V-Major selective communication [CC "V-Major"].
  * ---------------------------------------------------------------------- */
@@ -275,6 +292,16 @@ st_status vmajor_mask_compact_scatter(const void *v_cur, const void *v_prev,
  * bounded waits set.  Returns ST_ERR_TIMEOUT if a wait ran out since the last
  * call, ST_ERR_CUDA if the stream reports an error, else ST_OK. */
 st_status st_check_device_status(st_stream_t stream);
+
+/* SM budget of the calling host thread: the grids of the kernels it launches
+ * afterwards are sized for at most `sms` SMs (persistent kernels start at
+ * most one resident wave of that many SMs; 0 restores the whole device).
+ * Used to share the GPU between two streams, e.g. attention on most SMs while
+ * the memory-bound steps of the next shard range run on the rest; results do
+ * not depend on it.  Host-side only (not stream-ordered); ST_ERR_SHAPE for a
+ * negative count. */
+st_status st_set_sm_budget(int sms);
+int st_get_sm_budget(void);
 
 /* Failure-detection self test: launches a one-thread kernel that waits, with
  * a 20 ms limit, on an mbarrier nothing ever arrives on, through the same

@@ -7,9 +7,9 @@ Importing this module fails loudly when the library has not been built.
 
 Entry points (same names as the C ABI in include/stattn.h):
     st_attn_spatial, st_attn_spatial_merge, st_attn_temporal, attn_chunk_merge, ulysses_relayout,
-    vmajor_mask_compact, vmajor_mask_compact_noalloc, vmajor_mask_compact_scatter, vmajor_scatter_rows,
-    vmajor_workspace_bytes,
-    st_check_device_status, st_status_string
+    ulysses_relayout_range, vmajor_mask_compact, vmajor_mask_compact_noalloc, vmajor_mask_compact_scatter,
+    vmajor_scatter_rows, vmajor_workspace_bytes,
+    st_check_device_status, st_status_string, st_set_sm_budget, st_get_sm_budget
 """
 from __future__ import annotations
 
@@ -65,6 +65,9 @@ _c = {
                                c_int, c_int, c_int, _VP, c_int, _VP, _VP),
     "ulysses_relayout": _proto("ulysses_relayout", c_int, c_int, _VP, _VP, c_int, c_int, c_int, c_int, c_int,
                                c_int, c_int, c_int, c_int, c_int, c_int, c_int, _VP, c_int, c_float, _VP),
+    "ulysses_relayout_range": _proto("ulysses_relayout_range", c_int, c_int, _VP, _VP, c_int, c_int, c_int, c_int,
+                                     c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, _VP,
+                                     c_int, c_float, _VP),
     "vmajor_workspace_bytes": _proto("vmajor_workspace_bytes", c_size_t, c_ll),
     "vmajor_mask_compact": _proto("vmajor_mask_compact", c_int, _VP, _VP, c_ll, c_int, c_int, c_float, c_int,
                                   _VP, _VP, _VP, _VP, _VP, c_size_t, _VP),
@@ -77,13 +80,16 @@ _c = {
                                   ctypes.POINTER(_VP), ctypes.POINTER(_VP), c_int, ctypes.POINTER(_VP), _VP),
     "st_check_device_status": _proto("st_check_device_status", c_int, _VP),
     "st_selftest_wait_timeout": _proto("st_selftest_wait_timeout", c_int, _VP),
+    "st_set_sm_budget": _proto("st_set_sm_budget", c_int, c_int),
+    "st_get_sm_budget": _proto("st_get_sm_budget", c_int),
 }
 
 EXPORTED = ["st_status_string", "st_abi_version", "st_attn_spatial", "st_attn_spatial_merge", "st_attn_temporal",
             "attn_chunk_merge",
             "ulysses_relayout", "vmajor_workspace_bytes", "vmajor_mask_compact", "vmajor_mask_compact_noalloc",
             "vmajor_scatter_rows", "vmajor_mask_compact_scatter",
-            "st_check_device_status", "st_selftest_wait_timeout"]
+            "st_check_device_status", "st_selftest_wait_timeout", "ulysses_relayout_range", "st_set_sm_budget",
+            "st_get_sm_budget"]
 
 
 class StattnError(RuntimeError):
@@ -189,6 +195,18 @@ def ulysses_relayout(mode, inp, out, P, B, T_or_N, S_or_H, C_or_D, n_t=1, n_s=1,
     return r if raw else _check(r, "ulysses_relayout")
 
 
+def ulysses_relayout_range(mode, inp, out, P, B, T_or_N, S_or_H, C_or_D, n_t=1, n_s=1, blocks=None, shards=None,
+                           rms_gamma=None, rms_head_dim=0, rms_eps=1e-6, *, stream=None, raw=False):
+    """ulysses_relayout restricted to the temporally sharded shards ``shards`` = (q0, q1)."""
+    m = MODES[mode] if isinstance(mode, str) else int(mode)
+    i0, i1, j0, j1 = blocks if blocks is not None else (0, n_t, 0, n_s)
+    q0, q1 = shards if shards is not None else (0, P)
+    r = _c["ulysses_relayout_range"](m, _ptr(inp), _ptr(out), inp.element_size(), P, B, T_or_N, S_or_H, C_or_D,
+                                     n_t, n_s, i0, i1, j0, j1, q0, q1, _ptr(rms_gamma), int(rms_head_dim),
+                                     float(rms_eps), _stream(stream))
+    return r if raw else _check(r, "ulysses_relayout_range")
+
+
 # ---------------------------------------------------------------- V-Major
 def vmajor_workspace_bytes(n_tokens: int) -> int:
     return int(_c["vmajor_workspace_bytes"](int(n_tokens)))
@@ -242,6 +260,15 @@ def vmajor_scatter_rows(idx, count, src, dst_cache, packed=None, *, stream=None,
 
 def st_check_device_status(stream=None) -> int:
     return int(_c["st_check_device_status"](_stream(stream)))
+
+
+def st_set_sm_budget(sms: int) -> None:
+    """Size the grids of this thread's later launches for at most ``sms`` SMs (0: all)."""
+    _check(_c["st_set_sm_budget"](int(sms)), "st_set_sm_budget")
+
+
+def st_get_sm_budget() -> int:
+    return int(_c["st_get_sm_budget"]())
 
 
 def st_selftest_wait_timeout(stream=None) -> int:

@@ -26,6 +26,7 @@ struct Map {
   int mode;
   int P, B;
   int n_t, n_s, i0, n_i, j0, n_j;
+  int q0, n_q;             // temporally sharded side: shards q0 <= q < q0 + n_q
   int Tn, Tq, Sp, Ss;      // T/N_T, T/(N_T*P), S/(N_S*P), S/N_S
   int N, H, Np, Hp;        // sequence/head exchange
   long long row_bytes;     // bytes per row (C or D elements)
@@ -44,14 +45,16 @@ __device__ __forceinline__ void map_segment(const Map &m, long long g, long long
     int j = m.j0 + int(g % m.n_j); g /= m.n_j;
     int i = m.i0 + int(g % m.n_i); g /= m.n_i;
     int b = int(g % m.B);
-    int q = int(g / m.B);
+    int q = m.q0 + int(g / m.B);
     long long blk_y = (((long long)q * m.B + b) * m.n_t + i) * m.n_s + j;
     long long blk_x = (((long long)p * m.B + b) * m.n_t + i) * m.n_s + j;
     dst_row = (blk_y * m.Tq + t2) * m.Ss + (long long)p * m.Sp;
     src_row = (blk_x * m.Tn + (long long)q * m.Tq + t2) * m.Sp;
   } else if (m.mode == ST_T2S) {
-    // segments enumerate destination rows (p, b, i, j, t1)
-    int t1 = int(g % m.Tn); g /= m.Tn;
+    // segments enumerate destination rows (p, b, i, j, t1) whose frame comes
+    // from the selected y shards: t1 in [q0 * Tq, (q0 + n_q) * Tq)
+    const int nt1 = m.n_q * m.Tq;
+    int t1 = m.q0 * m.Tq + int(g % nt1); g /= nt1;
     int j = m.j0 + int(g % m.n_j); g /= m.n_j;
     int i = m.i0 + int(g % m.n_i); g /= m.n_i;
     int b = int(g % m.B);
@@ -397,10 +400,11 @@ unsigned int read_and_clear_relayout_error(cudaStream_t stream, cudaError_t *err
 }
 }  // namespace st
 
-ST_API st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *out, int elem_bytes,
-                                  int P, int B, int T_or_N, int S_or_H, int C_or_D, int n_t,
-                                  int n_s, int i0, int i1, int j0, int j1, const float *rms_gamma,
-                                  int rms_head_dim, float rms_eps, st_stream_t stream) {
+ST_API st_status ulysses_relayout_range(st_relayout_mode mode, const void *in, void *out, int elem_bytes,
+                                        int P, int B, int T_or_N, int S_or_H, int C_or_D, int n_t, int n_s,
+                                        int i0, int i1, int j0, int j1, int q0, int q1,
+                                        const float *rms_gamma, int rms_head_dim, float rms_eps,
+                                        st_stream_t stream) {
   if (!in || !out) return ST_ERR_NULL;
   if (!(elem_bytes == 1 || elem_bytes == 2 || elem_bytes == 4 || elem_bytes == 8)) return ST_ERR_DTYPE;
   if (P <= 0 || B <= 0 || T_or_N <= 0 || S_or_H <= 0 || C_or_D <= 0 || n_t <= 0 || n_s <= 0)
@@ -414,15 +418,18 @@ ST_API st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *o
     const int T = T_or_N, S = S_or_H, C = C_or_D;
     if (T % (n_t * P) || S % (n_s * P)) return ST_ERR_DIVISIBILITY;
     if (i0 < 0 || i1 > n_t || i0 >= i1 || j0 < 0 || j1 > n_s || j0 >= j1) return ST_ERR_SHAPE;
+    if (q0 < 0 || q1 > P || q0 >= q1) return ST_ERR_SHAPE;
     m.n_t = n_t; m.n_s = n_s; m.i0 = i0; m.n_i = i1 - i0; m.j0 = j0; m.n_j = j1 - j0;
+    m.q0 = q0; m.n_q = q1 - q0;
     m.Tn = T / n_t; m.Tq = T / (n_t * P); m.Sp = S / (n_s * P); m.Ss = S / n_s;
     m.row_bytes = (long long)C * elem_bytes;
     m.seg_bytes = m.Sp * m.row_bytes;
-    m.n_segs = (long long)P * B * m.n_i * m.n_j * m.Tn;
+    m.n_segs = (long long)m.n_q * B * m.n_i * m.n_j * m.Tq * P;
     if (rms_gamma && (rms_head_dim <= 0 || C % rms_head_dim)) return ST_ERR_SHAPE;
   } else if (mode == ST_SEQ2HEAD || mode == ST_HEAD2SEQ) {
     const int N = T_or_N, H = S_or_H, D = C_or_D;
     if (n_t != 1 || n_s != 1 || i0 != 0 || i1 != 1 || j0 != 0 || j1 != 1) return ST_ERR_SHAPE;
+    if (q0 != 0 || q1 != P) return ST_ERR_SHAPE;
     if (N % P || H % P) return ST_ERR_DIVISIBILITY;
     m.N = N; m.H = H; m.Np = N / P; m.Hp = H / P;
     m.row_bytes = (long long)D * elem_bytes;
@@ -460,4 +467,12 @@ ST_API st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *o
     case 2: return launch_copy<2>(m, src, dst, grid, s);
     default: return launch_copy<1>(m, src, dst, grid, s);
   }
+}
+
+ST_API st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *out, int elem_bytes,
+                                  int P, int B, int T_or_N, int S_or_H, int C_or_D, int n_t,
+                                  int n_s, int i0, int i1, int j0, int j1, const float *rms_gamma,
+                                  int rms_head_dim, float rms_eps, st_stream_t stream) {
+  return ulysses_relayout_range(mode, in, out, elem_bytes, P, B, T_or_N, S_or_H, C_or_D, n_t, n_s, i0, i1, j0,
+                                j1, 0, P, rms_gamma, rms_head_dim, rms_eps, stream);
 }

@@ -5,19 +5,33 @@
 
 namespace st {
 
+// SM budget of the launches this host thread issues (0: the whole device).
+thread_local int t_sm_budget = 0;
+
 int num_sms() {
   static int cache[64] = {0};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
+  int n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+    if (cache[dev] == 0) {
+      int a = 0;
+      if (cudaDeviceGetAttribute(&a, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || a <= 0) a = 148;
+      cache[dev] = a;
+    }
+    n = cache[dev];
   }
-  return cache[dev];
+  return t_sm_budget > 0 && t_sm_budget < n ? t_sm_budget : n;
 }
 
 }  // namespace st
+
+ST_API st_status st_set_sm_budget(int sms) {
+  if (sms < 0) return ST_ERR_SHAPE;
+  st::t_sm_budget = sms;
+  return ST_OK;
+}
+
+ST_API int st_get_sm_budget(void) { return st::t_sm_budget; }
 
 ST_API const char *st_status_string(st_status s) {
   switch (s) {

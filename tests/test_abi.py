@@ -78,6 +78,31 @@ def test_relayout_rejects(st):
     assert relayout(st, st.ST_S2T, out=ctypes.c_void_p(0x100000 + 64)) == st.ST_ERR_SHAPE   # overlap
 
 
+def relayout_range(st, mode, q0, q1, P=2, n_t=1, n_s=1):
+    return st._c["ulysses_relayout_range"](mode, FAKE_IN, FAKE_OUT, 2, P, 1, 8, 16, 64, n_t, n_s, 0, n_t, 0, n_s,
+                                           q0, q1, None, 0, 1e-6, None)
+
+
+def test_relayout_range_rejects(st):
+    """Shard ranges are validated before any launch: empty, reversed or out of range."""
+    for q0, q1 in ((0, 0), (1, 0), (-1, 1), (0, 3), (2, 2)):
+        assert relayout_range(st, st.ST_S2T, q0, q1) == st.ST_ERR_SHAPE, (q0, q1)
+        assert relayout_range(st, st.ST_T2S, q0, q1) == st.ST_ERR_SHAPE, (q0, q1)
+    # the sequence/head exchange has no shard range
+    assert relayout_range(st, st.ST_SEQ2HEAD, 0, 1) == st.ST_ERR_SHAPE
+
+
+def test_sm_budget_setting(st):
+    assert st.st_get_sm_budget() == 0
+    assert st._c["st_set_sm_budget"](-1) == st.ST_ERR_SHAPE
+    st.st_set_sm_budget(32)
+    try:
+        assert st.st_get_sm_budget() == 32
+    finally:
+        st.st_set_sm_budget(0)
+    assert st.st_get_sm_budget() == 0
+
+
 def spatial(st, fn="st_attn_spatial", q=FAKE_IN, **kw):
     d = dict(B=1, T=2, S=64, H=2, D=72, dtype=st.ST_BF16)
     d.update(kw)
