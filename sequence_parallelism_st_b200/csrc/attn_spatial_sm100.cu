@@ -85,7 +85,7 @@ constexpr int EPI_BUF = 32 * EPI_COLS * 4;   // bytes of one staging buffer (32 
 // TMEM columns: per tile two S buffers of BLOCK_N fp32 columns, then O.
 constexpr int TM_O = 256;                    // O(tile X) at TM_O + X * 128
 
-template <int D> struct Cfg {
+template <int D, bool MERGE = false> struct Cfg {
   static constexpr int C0 = D >= 64 ? 64 : 32;
   static constexpr int R1 = D > 64 ? D - 64 : 0;
   static constexpr int C1 = R1 == 0 ? 0 : (R1 <= 16 ? 16 : (R1 <= 32 ? 32 : 64));
@@ -104,21 +104,26 @@ template <int D> struct Cfg {
   // softmax need not add up its exponentials.  (Only when O fits one register
   // group of the epilogue, which reads the sum before normalising.)
   static constexpr bool ONES = DPV > D && (D + 15) / 16 <= 5;
-  // Merge mode seeds the TMEM accumulator O with the accumulated partial when
-  // the epilogue can hold a row of it in registers (at most 5 column chunks);
-  // larger head dims merge in the epilogue instead.
-  static constexpr bool MINIT = (D + 15) / 16 <= 5;
+  // Merge mode (the accumulated partial of earlier KV chunks is merged into
+  // the result in the epilogue): for head dims up to 80 the epilogue stages
+  // the accumulated rows of an item in shared memory while the item runs
+  // (one 32 x 16 fp32 block per warp, tile and 16-column chunk), paid for
+  // with a single Q buffer and a shallower K/V ring; larger head dims load
+  // them from global memory one chunk ahead.
+  static constexpr int NCH = (D + 15) / 16;            // 16-column chunks of O holding data
+  static_assert(!MERGE || NCH <= 5, "staged merge only for head dims up to 80");
+  static constexpr int ACCS = MERGE ? 8 * NCH * EPI_BUF : 0;
   static constexpr int VA = DPV / VW;                  // atoms
   static constexpr int VSW = VW * 2;                   // atom row bytes = swizzle span
   static constexpr int VAT = BLOCK_N * VSW;            // bytes of one atom region
   static constexpr int VTILE = VA * VAT;               // bytes of one V tile
-  static constexpr int BUDGET = 204800;
-  static constexpr int QB = (4 * QTILE + 4 * (KTILE + VTILE) <= BUDGET) ? 2 : 1;   // Q double buffer if 4 stages fit
+  static constexpr int EPI = 4 * 2 * EPI_BUF + 2 * 2 * BLOCK_M * 4;
+  static constexpr int BUDGET = MERGE ? 232448 - 4096 - EPI - ACCS : 204800;   // bytes for Q and the K/V ring
+  static constexpr int QB = (!MERGE && 4 * QTILE + 4 * (KTILE + VTILE) <= BUDGET) ? 2 : 1;   // Q double buffer if 4 stages fit
   static constexpr int NS_RAW = (BUDGET - 2 * QB * QTILE) / (KTILE + VTILE);
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;   // K/V ring depth
-  // epilogue: two staging buffers per epilogue warp, then the row statistics (m, l) of both tiles
-  static constexpr int EPI = 4 * 2 * EPI_BUF + 2 * 2 * BLOCK_M * 4;
-  static constexpr int SMEM = 1024 + 2 * QB * QTILE + NS * (KTILE + VTILE) + EPI + 1024;   // + barriers
+  // epilogue: two staging buffers per epilogue warp, then the row statistics (m, l) of both tiles (EPI above)
+  static constexpr int SMEM = 1024 + 2 * QB * QTILE + NS * (KTILE + VTILE) + ACCS + EPI + 1024;   // + barriers
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(DP <= 128 && DPV <= 128, "head dim too large");
   static_assert(NS >= 4, "ring too shallow");
@@ -379,21 +384,22 @@ __device__ __forceinline__ Item decode(const Params &p, int x) {
   return it;
 }
 
-template <int D>
+template <int D, bool MERGE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
                    const __grid_constant__ CUtensorMap tk0, const __grid_constant__ CUtensorMap tk1,
                    const __grid_constant__ CUtensorMap tv0, const __grid_constant__ CUtensorMap tv1,
                    const __grid_constant__ CUtensorMap to, const __grid_constant__ CUtensorMap tacc,
                    const Params p) {
-  using K = Cfg<D>;
+  using K = Cfg<D, MERGE>;
   constexpr int NS = K::NS, QB = K::QB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = base;                          // QB x 2 Q tiles
   uint8_t *sK = sQ + QB * 2 * K::QTILE;        // NS K tiles
   uint8_t *sV = sK + NS * K::KTILE;            // NS V tiles
-  uint8_t *sEpi = sV + NS * K::VTILE;          // 4 warps x 2 staging buffers
+  uint8_t *sAcc = sV + NS * K::VTILE;          // merge mode: [tile][epilogue warp][chunk] 32 x 16 fp32 blocks
+  uint8_t *sEpi = sAcc + K::ACCS;              // 4 warps x 2 staging buffers
   float *sStat = reinterpret_cast<float *>(sEpi + 4 * 2 * EPI_BUF);   // [tile][m | l][row]
   uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + K::EPI);
   uint64_t *q_full = bars;                     // QB
@@ -414,7 +420,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *stat_full = mma_done + 4;          // 2, 128 arrivals (softmax threads)
   uint64_t *stat_empty = stat_full + 2;        // 2, 128 arrivals (epilogue threads)
   uint64_t *v_ready = stat_empty + 2;          // NS: ones column written into the V stage
-  uint64_t *acc_full = v_ready + NS;           // 4 epilogue warps x 2 staging buffers: o_acc block landed
+  uint64_t *acc_full = v_ready + NS;           // [epilogue warp][tile]: the item's accumulated rows landed
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -460,7 +466,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t epoch = p.epoch;
-  const bool minit = K::MINIT && p.o_acc != nullptr;   // merge by seeding O (see the epilogue)
   // barriers and TMEM are set up: let the next kernel of the stream be
   // scheduled, then wait for the previous one before any global access
   pdl_trigger();
@@ -603,8 +608,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b = step & 1;
           if (!(ok = mbar_wait((K::ONES ? v_ready : v_full) + st, (g0 / NS) & 1, epoch, 6))) break;
           if (!(ok = mbar_wait(p_full + 2 * X + b, (step >> 1) & 1, epoch, 7 + X))) break;
-          // O free (plain) or O seeded with the accumulated partial (merge mode)
-          if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc & 1) ^ (minit ? 0u : 1u), epoch, 9 + X))) break;
+          // O of the tile's previous item read out by the epilogue
+          if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc & 1) ^ 1u, epoch, 9 + X))) break;
           tc_fence_after();
           const uint32_t d = tmem + TM_O + X * 128;
           const uint32_t pa = tmem + X * 2 * BLOCK_N + b * BLOCK_N;   // P (bf16 pairs) over the S columns
@@ -612,7 +617,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   #pragma unroll
           for (int kk = 0; kk < BLOCK_N / 16; ++kk)
             mma_ts(d, pa + kk * 8, sdesc_c<K::VAT, 8 * K::VSW, layout_of(K::VSW)>(va + kk * 16 * K::VSW), IDPV,
-                   (j > 0 || kk > 0 || minit) ? 1u : 0u);
+                   (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(pv_done + 2 * X + b);
           tc_commit(v_empty + st);
         }
@@ -667,17 +672,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Item it = decode(p, x);
       if (X >= it.n_qt) continue;
       float m = -INFINITY, l = 0.f;
-      if (minit) {
-        // continue the online softmax from the accumulated partial: its LSE in
-        // log2 units is the running max, and its normalised O (seeded into
-        // TMEM by the epilogue) has row sum 1
-        const int qrow = it.q0 + X * BLOCK_M + r;
-        const float la = qrow < g.S ? p.lse_acc[(((long long)it.b * g.T + it.t) * g.H + it.h) * g.S + qrow] : -INFINITY;
-        if (la != -INFINITY) {
-          m = la * 1.4426950408889634f;
-          l = 1.f;
-        }
-      }
       for (int j = 0; j < n_kv; ++j, ++gs) {
         const uint32_t b = gs & 1;
         if (!(ok = mbar_wait(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
@@ -705,18 +699,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         const float mx = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]), mxp[3]) * sl2;
-        if (j == 0 && !minit) {
+        if (j == 0) {
           m = mx;
         } else {
           const bool need = mx > m + 8.0f;
           if (__any_sync(0xffffffffu, need)) {
-            // O holds PV up to step gs-1 (or, at the first step of a merge, the
-            // seeded partial): wait for it, then rescale in TMEM
-            if (j == 0) {
-              if (!(ok = mbar_wait(o_empty + X, oc & 1, epoch, 25 + X))) break;
-            } else if (!(ok = mbar_wait(pv_done + 2 * X + ((gs - 1) & 1), ((gs - 1) >> 1) & 1, epoch, 15 + X))) {
-              break;
-            }
+            // O holds PV up to step gs-1: wait for it, then rescale in TMEM
+            if (!(ok = mbar_wait(pv_done + 2 * X + ((gs - 1) & 1), ((gs - 1) >> 1) & 1, epoch, 15 + X))) break;
             tc_fence_after();
             const float corr = need ? ex2_mufu(m - mx) : 1.0f;
             if (need) {
@@ -787,52 +776,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     uint8_t *stg = sEpi + qd * 2 * EPI_BUF;
     uint32_t oc0 = 0, oc1 = 0, nst = 0;        // items per tile, bulk stores issued by this warp
-    uint32_t ua = 0;                           // accumulator loads per staging buffer, 16 bits each (merge mode)
     bool ok = true;
-    if (K::MINIT && minit && n_kv > 0) {
-      // seed O of each tile's first item before waiting on anything: a tile
-      // whose first PV cannot start would stall the shared K/V ring and with
-      // it the other tile
-      constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;
-      constexpr int LC = K::ONES ? D / 16 : 0;
-      for (int X = 0; X < 2; ++X) {
-        int x0 = blockIdx.x;
-        while (x0 < n_items && X >= decode(p, x0).n_qt) x0 += gridDim.x;
-        if (x0 >= n_items) continue;
-        const Item jt = decode(p, x0);
-        const int jrow = jt.q0 + X * BLOCK_M + qd * 32 + lane;
-        const bool jv = jrow < g.S;
-        const bool has = jv && p.lse_acc[(((long long)jt.b * g.T + jt.t) * g.H + jt.h) * g.S + jrow] != -INFINITY;
-        const float *ap = p.o_acc + (jv ? g.frame(jt.b, jt.t) + g.token(jrow) + (long long)jt.h * D : 0);
-        const uint32_t tO = tmem + lane_off + TM_O + X * 128;
-#pragma unroll
-        for (int k = 0; k < NCH; ++k) {
-          uint32_t a[16];
-#pragma unroll
-          for (int f = 0; f < 4; ++f) {
-            float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (has && k * 16 + 4 * f < D) a4 = *reinterpret_cast<const float4 *>(ap + k * 16 + 4 * f);
-            a[4 * f] = __float_as_uint(a4.x);
-            a[4 * f + 1] = __float_as_uint(a4.y);
-            a[4 * f + 2] = __float_as_uint(a4.z);
-            a[4 * f + 3] = __float_as_uint(a4.w);
-          }
-          if (K::ONES && k == LC) a[D % 16] = __float_as_uint(has ? 1.f : 0.f);
-          TMEM_ST16(tO + k * 16, a);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(o_empty + X);
-      }
-    }
+    bool acc_pending[2] = {false, false};      // merge mode: staged loads issued and not yet waited for
+    uint32_t acc_par[2] = {0u, 0u};            // ... and the barrier phase they complete
     for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
       const Item it = decode(p, x);
-      if (p.o_acc && n_kv > 0) {
-        // the accumulated rows this warp merges at the end of the item: start
-        // moving them into L2 now, while the item's steps run
+      float la_t[2] = {-INFINITY, -INFINITY};  // merge mode: accumulated LSE of this lane's row per tile
+      if ((MERGE || K::NCH > 5) && p.o_acc && n_kv > 0) {
+        // the accumulated rows this warp merges at the end of the item: with a
+        // staging area the copy engine brings them into shared memory now,
+        // otherwise into L2, while the item's steps run
         for (int X = 0; X < it.n_qt; ++X) {
-          const int qrow = it.q0 + X * BLOCK_M + qd * 32 + lane;
-          if (qrow < g.S) {
+          const int row0 = it.q0 + X * BLOCK_M + qd * 32;
+          const int qrow = row0 + lane;
+          if (qrow < g.S) la_t[X] = p.lse_acc[(((long long)it.b * g.T + it.t) * g.H + it.h) * g.S + qrow];
+          if constexpr (MERGE) {
+            __syncwarp();                      // the previous item's reads of the area are done
+            if (lane == 0) {
+              fence_async_smem();              // ... and ordered before the copies that overwrite it
+              mbar_expect_tx(acc_full + qd * 2 + X, K::NCH * EPI_BUF);
+#pragma unroll
+              for (int k = 0; k < K::NCH; ++k)
+                tma_load_5d(sAcc + ((X * 4 + qd) * K::NCH + k) * EPI_BUF, &tacc, acc_full + qd * 2 + X,
+                            k * EPI_COLS, it.h, row0, it.c3, it.c4);
+            }
+            acc_pending[X] = true;
+            acc_par[X] = (X ? oc1 : oc0) & 1;   // items of this tile so far = the phase of these copies
+          } else if (qrow < g.S) {
             const float *src = p.o_acc + g.frame(it.b, it.t) + g.token(qrow) + (long long)it.h * D;
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(uint32_t(D * 4)) : "memory");
           }
@@ -858,108 +828,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           continue;
         }
         const uint32_t ocx = X ? oc1 : oc0;
-        if (K::MINIT && minit) {
-          // ---- merge by seeding O: after reading O of this item, write the
-          // accumulated partial of this tile's next item into the same TMEM
-          // columns (its row sum 1 in the ones column), so that item's PV
-          // accumulates onto it and its softmax continues from the partial's LSE
-          constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;
-          constexpr int LC = K::ONES ? D / 16 : 0;            // chunk holding the ones column
-          const uint32_t tO = tmem + lane_off + TM_O + X * 128;
-          // where the accumulated row of item xx lives, and whether it holds anything
-#define ST_ACC_ROW(xx, ap, has)                                                                              \
-  const float *ap;                                                                                           \
-  bool has;                                                                                                  \
-  {                                                                                                          \
-    const Item jt = decode(p, (xx));                                                                         \
-    const int jrow = jt.q0 + X * BLOCK_M + r;                                                                \
-    const bool jv = jrow < g.S;                                                                              \
-    has = jv && p.lse_acc[(((long long)jt.b * g.T + jt.t) * g.H + jt.h) * g.S + jrow] != -INFINITY;          \
-    ap = p.o_acc + (jv ? g.frame(jt.b, jt.t) + g.token(jrow) + (long long)jt.h * D : 0);                     \
-  }
-          // 16 columns of an accumulated row (zero where nothing is accumulated;
-          // the ones column carries its row sum 1)
-#define ST_ACC_CHUNK(ap, has, k, a)                                                                          \
+        const long long off = valid ? g.frame(it.b, it.t) + g.token(qrow) + (long long)it.h * D : 0;
+        // merge flow: the accumulated LSE of the row was loaded at the start of
+        // the item; the accumulated partial is read from the staging area
+        // (MERGE) or from global memory one 16-column chunk ahead of its use
+        // (head dims up to 80 merge only in the MERGE instantiation)
+        const bool merging = (MERGE || K::NCH > 5) && p.o_acc != nullptr;
+        const float la = la_t[X];
+        const bool use_acc = la != -INFINITY;  // nothing accumulated: the partial is not read
+        const float *arow = p.o_acc + off;
+        float4 an[4];                          // accumulated chunk, one ahead (global flow)
+#define ST_LOAD_ACC(k)                                                                                       \
   _Pragma("unroll") for (int f = 0; f < 4; ++f) {                                                            \
-    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);                                                             \
-    if ((has) && (k) * 16 + 4 * f < D) a4 = *reinterpret_cast<const float4 *>((ap) + (k) * 16 + 4 * f);     \
-    a[4 * f] = __float_as_uint(a4.x);                                                                        \
-    a[4 * f + 1] = __float_as_uint(a4.y);                                                                    \
-    a[4 * f + 2] = __float_as_uint(a4.z);                                                                    \
-    a[4 * f + 3] = __float_as_uint(a4.w);                                                                    \
-  }                                                                                                          \
-  if (K::ONES && (k) == LC) a[D % 16] = __float_as_uint((has) ? 1.f : 0.f);
-          int xn = x + gridDim.x;              // this tile's next item
-          while (xn < n_items && X >= decode(p, xn).n_qt) xn += gridDim.x;
-          const bool has_next = xn < n_items;
-          ST_ACC_ROW(has_next ? xn : x, apn, hasn)
-          hasn = hasn && has_next;
-          if (hasn)                            // bring the row into L2 while this item computes
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(apn), "r"(uint32_t(D * 4)) : "memory");
-          if (!(ok = mbar_wait(o_full + X, ocx & 1, epoch, 17 + X))) break;
-          if (!(ok = mbar_wait(stat_full + X, ocx & 1, epoch, 19 + X))) break;
-          if (X) ++oc1;
-          else ++oc0;
-          tc_fence_after();
-          const float m = sStat[(X * 2 + 0) * BLOCK_M + r];
-          float l = sStat[(X * 2 + 1) * BLOCK_M + r];
-          mbar_arrive(stat_empty + X);
-          if (K::ONES) {                       // the row sum, from the ones column
-            uint32_t lv;
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(lv) : "r"(tO + D));
-            tmem_wait_ld();
-            l = __uint_as_float(lv);
-          }
-          const float inv = 1.0f / l;
-          const int row0 = it.q0 + X * BLOCK_M + qd * 32;
-          uint32_t an[16];                     // seed chunk k, loaded one chunk ahead
-          if (has_next) { ST_ACC_CHUNK(apn, hasn, 0, an) }
-#pragma unroll
-          for (int k = 0; k < NCH; ++k, ++nst) {
-            uint32_t ov[16];
-            TMEM_LD16(tO + k * 16, ov);
-            tmem_wait_ld();
-            if (has_next) {
-              TMEM_ST16(tO + k * 16, an);      // this chunk of O is read: overwrite it with the seed
-              if (k + 1 < NCH) { ST_ACC_CHUNK(apn, hasn, k + 1, an) }
-            }
-            uint8_t *buf = stg + (nst & 1) * EPI_BUF;
-            if (lane == 0) bulk_wait_read1();
-            __syncwarp();
-            if (p.o_f32) {
-#pragma unroll
-              for (int f = 0; f < 4; ++f)
-                *reinterpret_cast<float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4)) =
-                    make_float4(__uint_as_float(ov[4 * f]) * inv, __uint_as_float(ov[4 * f + 1]) * inv,
-                                __uint_as_float(ov[4 * f + 2]) * inv, __uint_as_float(ov[4 * f + 3]) * inv);
-            } else {
-#pragma unroll
-              for (int f = 0; f < 2; ++f) {
-                uint4 w;
-                w.x = st::pack_bf16x2(__uint_as_float(ov[8 * f]) * inv, __uint_as_float(ov[8 * f + 1]) * inv);
-                w.y = st::pack_bf16x2(__uint_as_float(ov[8 * f + 2]) * inv, __uint_as_float(ov[8 * f + 3]) * inv);
-                w.z = st::pack_bf16x2(__uint_as_float(ov[8 * f + 4]) * inv, __uint_as_float(ov[8 * f + 5]) * inv);
-                w.w = st::pack_bf16x2(__uint_as_float(ov[8 * f + 6]) * inv, __uint_as_float(ov[8 * f + 7]) * inv);
-                *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
-              }
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              if (row0 < g.S) tma_store_5d(&to, buf, k * EPI_COLS, it.h, row0, it.c3, it.c4);
-              bulk_commit();
-            }
-          }
-#undef ST_ACC_ROW
-#undef ST_ACC_CHUNK
-          if (has_next) {                      // the next item's seed is in TMEM
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(o_empty + X);
-          }
-          if (valid && p.lse) p.lse[lse_idx] = (m + log2f(l)) * 0.6931471805599453f;
-          continue;
-        }
+    an[f] = make_float4(0.f, 0.f, 0.f, 0.f);                                                                 \
+    if (valid && (k) * 16 + 4 * f < D) an[f] = *reinterpret_cast<const float4 *>(arow + (k) * 16 + 4 * f);   \
+  }
+        if (!MERGE && merging) { ST_LOAD_ACC(0) }
         if (!(ok = mbar_wait(o_full + X, ocx & 1, epoch, 17 + X))) break;
         if (!(ok = mbar_wait(stat_full + X, ocx & 1, epoch, 19 + X))) break;
         if (X) ++oc1;
@@ -970,7 +854,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive(stat_empty + X);
         float inv = 1.0f / l;
         float fa = 0.f, lse_row = 0.f;         // weight of the accumulated partial; LSE of the row
-        const long long off = valid ? g.frame(it.b, it.t) + g.token(qrow) + (long long)it.h * D : 0;
         const uint32_t tO = tmem + lane_off + TM_O + X * 128;
         constexpr int NCH = (D + EPI_COLS - 1) / EPI_COLS;    // 16-column chunks holding data
         constexpr int G0 = NCH > 5 ? 4 : NCH;                  // chunks of the first register group
@@ -993,8 +876,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // this chunk's natural-log LSE; merged with the accumulated one when asked:
             //   w_a = exp(lse_a - M), w_c = exp(lse_c - M), o = (w_a o_a + w_c O / l) / (w_a + w_c)
             lse_row = (m + log2f(l)) * 0.6931471805599453f;
-            if (!K::MINIT && p.o_acc) {
-              const float la = valid ? p.lse_acc[lse_idx] : -INFINITY;
+            if (merging) {
               const float M = fmaxf(la, lse_row);
               const float wa = expf(la - M), wc = expf(lse_row - M);
               const float sw = wa + wc;
@@ -1008,81 +890,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_arrive(o_empty + X);          // O of this tile may be overwritten
           }
           const int row0 = it.q0 + X * BLOCK_M + qd * 32;
-          if (!K::MINIT && p.o_acc) {
-            // merge flow: the copy engine brings each 32 x 16 block of o_acc into a
-            // staging buffer (the next block's load overlaps this block's merge),
-            // each lane merges its row there, and the block goes back out with a
-            // bulk tensor store (in place when o is o_acc)
-            const int nb = int(nst & 1);
-            if (lane == 0) {
-              bulk_wait_read0();               // the store that last used a buffer has read it
-              mbar_expect_tx(acc_full + qd * 2 + nb, EPI_BUF);
-              tma_load_5d(stg + nb * EPI_BUF, &tacc, acc_full + qd * 2 + nb, c0 * EPI_COLS, it.h, row0, it.c3, it.c4);
-            }
-#pragma unroll
-            for (int c = 0; c < G0; ++c) {
-              if (c >= nch) break;
-              const int bb = (nb + c) & 1;
-              if (c + 1 < nch && lane == 0) {  // the next block's load overlaps this block's merge
-                bulk_wait_read0();
-                mbar_expect_tx(acc_full + qd * 2 + (bb ^ 1), EPI_BUF);
-                tma_load_5d(stg + (bb ^ 1) * EPI_BUF, &tacc, acc_full + qd * 2 + (bb ^ 1), (c0 + c + 1) * EPI_COLS,
-                            it.h, row0, it.c3, it.c4);
-              }
-              bool got = true;
-              if (lane == 0) got = mbar_wait(acc_full + qd * 2 + bb, (ua >> (16 * bb)) & 1, epoch, 23);
-              ua += 1u << (16 * bb);
-              if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
-                ok = false;
-                break;
-              }
-              __syncwarp();                    // lane 0 saw the block land: order the other lanes after it
-              uint8_t *buf = stg + bb * EPI_BUF;
-              const bool use_acc = fa != 0.f;  // nothing accumulated: the block is not read
-              float *y = reinterpret_cast<float *>(ov[c]);
-#pragma unroll
-              for (int f = 0; f < 4; ++f) {
-                float4 a4 = *reinterpret_cast<const float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4));
-                if (!use_acc) a4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                y[4 * f] = fmaf(fa, a4.x, __uint_as_float(ov[c][4 * f]) * inv);
-                y[4 * f + 1] = fmaf(fa, a4.y, __uint_as_float(ov[c][4 * f + 1]) * inv);
-                y[4 * f + 2] = fmaf(fa, a4.z, __uint_as_float(ov[c][4 * f + 2]) * inv);
-                y[4 * f + 3] = fmaf(fa, a4.w, __uint_as_float(ov[c][4 * f + 3]) * inv);
-              }
-              __syncwarp();                    // every row of the block is read before any is overwritten
-              if (p.o_f32) {
-#pragma unroll
-                for (int f = 0; f < 4; ++f)
-                  *reinterpret_cast<float4 *>(buf + lane * 64 + ((f ^ ((lane >> 1) & 3)) << 4)) =
-                      make_float4(y[4 * f], y[4 * f + 1], y[4 * f + 2], y[4 * f + 3]);
-              } else {
-#pragma unroll
-                for (int f = 0; f < 2; ++f) {
-                  uint4 w;
-                  w.x = st::pack_bf16x2(y[8 * f], y[8 * f + 1]);
-                  w.y = st::pack_bf16x2(y[8 * f + 2], y[8 * f + 3]);
-                  w.z = st::pack_bf16x2(y[8 * f + 4], y[8 * f + 5]);
-                  w.w = st::pack_bf16x2(y[8 * f + 6], y[8 * f + 7]);
-                  *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
-                }
-              }
-              fence_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                if (row0 < g.S) tma_store_5d(&to, buf, (c0 + c) * EPI_COLS, it.h, row0, it.c3, it.c4);
-                bulk_commit();
-              }
-            }
-            nst += nch;
-            if (!ok) break;
-          } else {
+          {
 #pragma unroll
           for (int c = 0; c < G0; ++c, ++nst) {
             if (c >= nch) break;
             uint8_t *buf = stg + (nst & 1) * EPI_BUF;
             float *y = reinterpret_cast<float *>(ov[c]);
+            if (merging) {
+              // o = fa * o_acc + O * inv, with fa = w_a / (w_a + w_c), inv = w_c / ((w_a + w_c) l)
+              float a[16];
+              if constexpr (MERGE) {
+                if (c0 + c == 0) {             // the item's staged rows of this warp and tile have landed
+                  bool got = true;
+                  if (lane == 0) got = mbar_wait(acc_full + qd * 2 + X, ocx & 1, epoch, 23);
+                  if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) {
+                    ok = false;
+                    break;
+                  }
+                  acc_pending[X] = false;
+                  __syncwarp();
+                }
+                // 64B swizzle of the fp32 block: 16-byte chunk f of row r at f ^ ((r >> 1) & 3)
+                const uint8_t *ab = sAcc + ((X * 4 + qd) * K::NCH + c0 + c) * EPI_BUF + lane * 64;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(ov[c][e]) * inv;
+                for (int f = 0; f < 4; ++f) an[f] = *reinterpret_cast<const float4 *>(ab + ((f ^ ((lane >> 1) & 3)) << 4));
+              }
+#pragma unroll
+              for (int f = 0; f < 4; ++f) {   // a row with nothing accumulated is not used (may hold NaN)
+                a[4 * f] = use_acc ? an[f].x : 0.f;
+                a[4 * f + 1] = use_acc ? an[f].y : 0.f;
+                a[4 * f + 2] = use_acc ? an[f].z : 0.f;
+                a[4 * f + 3] = use_acc ? an[f].w : 0.f;
+              }
+              if (!MERGE && c0 + c + 1 < NCH) { ST_LOAD_ACC(c0 + c + 1) }
+#pragma unroll
+              for (int e = 0; e < 16; ++e) y[e] = fmaf(fa, a[e], __uint_as_float(ov[c][e]) * inv);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(ov[c][e]) * inv;
+            }
             if (lane == 0) bulk_wait_read1();  // the store that used this buffer has read it
             __syncwarp();
             if (p.o_f32) {
@@ -1114,11 +960,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           }
         }
+#undef ST_LOAD_ACC
         if (!ok) break;
         if (valid && p.lse) p.lse[lse_idx] = lse_row;
       }
     }
     if (lane == 0) bulk_wait_all();
+    if (MERGE && lane == 0) {
+      // after an abort: staged copies into this warp's area may still be in
+      // flight; wait for them (bounded, ignoring the abort epoch) before exiting
+      const unsigned long long t0 = globaltimer();
+      for (int X = 0; X < 2; ++X)
+        if (acc_pending[X])
+          while (!mbar_try_wait(acc_full + qd * 2 + X, acc_par[X]) && globaltimer() - t0 < WAIT_NS) {
+          }
+    }
     __syncwarp();
   }
 
@@ -1207,11 +1063,11 @@ bool make_map(CUtensorMap *m, const void *ptr, const st::Geom &g, int tmode, int
 
 std::atomic<uint32_t> g_epoch{0};
 
-template <int D>
+template <int D, bool MERGE>
 st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, float scale, const void *q,
                          const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
                          const float *o_acc, const float *lse_acc) {
-  using K = Cfg<D>;
+  using K = Cfg<D, MERGE>;
   const int tmode = g.tblk != g.T ? 1 : 0;
   CUtensorMap m[8];
   const int c1 = K::C1 ? K::C1 : 16;
@@ -1220,7 +1076,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
       !make_map(&m[4], v, g, tmode, K::VW, K::VSW, BLOCK_N) || !make_map(&m[5], v, g, tmode, K::VW, K::VSW, BLOCK_N) ||
       !make_map(&m[6], o, g, tmode, EPI_COLS, EPI_COLS * (o_f32 ? 4 : 2), 32, o_f32))
     return ST_ERR_CUDA;
-  // fp32 accumulator blocks of the merge mode (unused otherwise)
+  // fp32 accumulator blocks staged by the merge mode (unused otherwise)
   if (o_acc) {
     if (!make_map(&m[7], o_acc, g, tmode, EPI_COLS, EPI_COLS * 4, 32, 1)) return ST_ERR_CUDA;
   } else {
@@ -1246,7 +1102,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   if (items <= 0) return ST_OK;
   if (items > 0x7fffffffLL) return ST_ERR_SHAPE;
   const int ctas = int(items < st::num_sms() ? items : st::num_sms());  // persistent: one CTA per SM
-  auto kern = attn_fwd_sm100<D>;
+  auto kern = attn_fwd_sm100<D, MERGE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM) != cudaSuccess)
     return ST_ERR_CUDA;
   // The register split of the warpgroups (setmaxnreg) assumes the launch
@@ -1280,14 +1136,18 @@ st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, fl
                              const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
                              const float *o_acc, const float *lse_acc) {
   if (hi <= lo) return ST_OK;
+  // merge mode with head dims up to 80 stages the accumulated rows in shared memory
+#define ST_SPATIAL(DD, MM) launch_spatial<DD, MM>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc)
+  const bool staged = o_acc != nullptr;
   switch (g.D) {
-    case 32: return launch_spatial<32>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
-    case 64: return launch_spatial<64>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
-    case 72: return launch_spatial<72>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
-    case 80: return launch_spatial<80>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
-    case 96: return launch_spatial<96>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
-    case 128: return launch_spatial<128>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc);
+    case 32: return staged ? ST_SPATIAL(32, true) : ST_SPATIAL(32, false);
+    case 64: return staged ? ST_SPATIAL(64, true) : ST_SPATIAL(64, false);
+    case 72: return staged ? ST_SPATIAL(72, true) : ST_SPATIAL(72, false);
+    case 80: return staged ? ST_SPATIAL(80, true) : ST_SPATIAL(80, false);
+    case 96: return ST_SPATIAL(96, false);
+    case 128: return ST_SPATIAL(128, false);
   }
+#undef ST_SPATIAL
   return ST_ERR_UNSUPPORTED;
 }
 
