@@ -10,8 +10,11 @@ the OpenSora-like low-resolution workload (B=1, T=16 frames, S=1200 tokens,
      the active tokens (vmajor_mask_compact), cache update of K/V rows of the
      active tokens (vmajor_scatter_rows);
   3. spatial attention of the fresh Q against the cached K/V in R KV chunks
-     (st_attn_spatial, fp32 partials + LSE) and their log-sum-exp merge
-     (attn_chunk_merge);
+     and their log-sum-exp merge: chunk 0 writes the fp32 partial and its LSE
+     (st_attn_spatial), every later chunk merges into it inside the attention
+     kernel and the last one writes the bf16 result (st_attn_spatial_merge);
+     ``--merge separate`` writes R partials and merges them with
+     attn_chunk_merge instead;
   4. all-to-all T->S of the spatial output;
   5. temporal attention over the T frames of every token, read in place from
      the spatially sharded slice layout (st_attn_temporal).
@@ -47,7 +50,8 @@ import synth  # noqa: E402
 
 METRIC = "attention TFLOP/s & relayout GB/s on 1 B200, as fraction of bf16/HBM peak"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP_BASE = 10           # relayouts 3+1, vmajor 3, merge 1, temporal 1, + R spatial launches
+LAUNCHES_PER_STEP_BASE = 9            # relayouts 3+1, vmajor 3 (mask, compaction, scatter), merge 1, temporal 1
+                                      # (+ R spatial launches; the fused merge has no merge launch)
 SPATIAL_SRC = os.path.join(ROOT, "sequence_parallelism_st_b200", "csrc", "attn_spatial_sm100.cu")
 
 
@@ -159,6 +163,11 @@ class Step:
         assert T % (w.n_t * P) == 0 and T // (w.n_t * P) == 1
         self.sdesc = [st.make_desc(1, T, S, H, D, st.ST_BF16, kv_begin=c * S // w.R, kv_end=(c + 1) * S // w.R,
                                    o_fp32=1) for c in range(w.R)]
+        # fused merge: chunk c >= 1 is merged into the accumulated fp32 partial
+        # inside the attention kernel; the last chunk writes the bf16 result
+        self.fused_merge = True
+        self.sdesc_last = st.make_desc(1, T, S, H, D, st.ST_BF16, kv_begin=(w.R - 1) * S // w.R, kv_end=S,
+                                       o_fp32=0)
         Tb, Sb = T // w.n_t, S // (w.n_s * P)
         self.tdesc = st.make_desc(P * B, T, S // P, H, D, st.ST_BF16, stride_b=w.n_t * w.n_s * Tb * Sb * C,
                                   stride_t=Sb * C, stride_s=C, t_block=Tb, stride_tb=w.n_s * Tb * Sb * C,
@@ -210,19 +219,41 @@ class Step:
         st.vmajor_scatter_rows(self.idx, self.count, [self.ky.view(self.n, C), self.vy.view(self.n, C)],
                                [self.kc.view(self.n, C), self.vc.view(self.n, C)])
         self._mark("vmajor", False)
-        self._mark("spatial", True)
-        for c in range(w.R):
-            st.st_attn_spatial(self.qy, self.kc, self.vc, self.parts[c], self.lses[c], desc=self.sdesc[c])
-        self._mark("spatial", False)
-        self._mark("merge", True)
-        st.attn_chunk_merge(self.parts, self.lses, B * T, S, w.H, D, self.oy)
-        self._mark("merge", False)
+        if self.fused_merge:
+            self._spatial_fused(None)
+        else:
+            self._mark("spatial", True)
+            for c in range(w.R):
+                st.st_attn_spatial(self.qy, self.kc, self.vc, self.parts[c], self.lses[c], desc=self.sdesc[c])
+            self._mark("spatial", False)
+            self._mark("merge", True)
+            st.attn_chunk_merge(self.parts, self.lses, B * T, S, w.H, D, self.oy)
+            self._mark("merge", False)
         self._mark("relayout_t2s", True)
         st.ulysses_relayout("T2S", self.oy, self.ox, P, B, T, S, C, w.n_t, w.n_s)
         self._mark("relayout_t2s", False)
         self._mark("temporal", True)
         st.st_attn_temporal(d["q"], d["k"], d["v"], self.ot, None, desc=self.tdesc)
         self._mark("temporal", False)
+
+    def _spatial_fused(self, i):
+        """KV chunks of the spatial attention with the merge fused into the
+        kernel: chunk 0 writes the fp32 partial and its LSE, chunks 1..R-2 merge
+        into it in place, chunk R-1 merges and writes the bf16 result (and the
+        merged LSE).  i: shard range of the overlapped schedule, or None."""
+        st, w = self.st, self.w
+        descs = self.sdesc if i is None else self.sdesc_sl[i]
+        last = self.sdesc_last if i is None else self.sdesc_last_sl[i]
+        self._mark("spatial", True)
+        st.st_attn_spatial(self.qy, self.kc, self.vc, self.parts[0], self.lses[0], desc=descs[0])
+        self._mark("spatial", False)
+        self._mark("spatial_merge", True)
+        for c in range(1, w.R - 1):
+            st.st_attn_spatial_merge(self.qy, self.kc, self.vc, self.parts[0], self.lses[0], self.parts[0],
+                                     self.lses[0], desc=descs[c])
+        st.st_attn_spatial_merge(self.qy, self.kc, self.vc, self.parts[0], self.lses[0], self.oy, self.lses[1],
+                                 desc=last)
+        self._mark("spatial_merge", False)
 
     # ------------------------------------------------------------ overlapped schedule
     def setup_overlap(self, n_slices, att_sms):
@@ -241,6 +272,9 @@ class Step:
         self.sdesc_sl = [[self.st.make_desc(1, T, w.S, w.H, w.D, self.st.ST_BF16, kv_begin=c * w.S // w.R,
                                             kv_end=(c + 1) * w.S // w.R, o_fp32=1, n_slices=n_slices, slice=i)
                           for c in range(w.R)] for i in range(n_slices)]
+        self.sdesc_last_sl = [self.st.make_desc(1, T, w.S, w.H, w.D, self.st.ST_BF16,
+                                                kv_begin=(w.R - 1) * w.S // w.R, kv_end=w.S, o_fp32=0,
+                                                n_slices=n_slices, slice=i) for i in range(n_slices)]
         self.n_sl_tok = n_sl_tok
 
     def _prep(self, i):
@@ -269,8 +303,9 @@ class Step:
         f0, f1 = i * T // self.n_sl, (i + 1) * T // self.n_sl
         e0, e1 = f0 * S * C, f1 * S * C
         l0, l1 = f0 * H * S, f1 * H * S
-        st.attn_chunk_merge([p[e0:e1] for p in self.parts], [x[l0:l1] for x in self.lses], B * (f1 - f0), S, H, D,
-                            self.oy[e0:e1])
+        if not self.fused_merge:
+            st.attn_chunk_merge([p[e0:e1] for p in self.parts], [x[l0:l1] for x in self.lses], B * (f1 - f0), S, H,
+                                D, self.oy[e0:e1])
         st.ulysses_relayout_range("T2S", self.oy, self.ox, P, B, T, S, C, w.n_t, w.n_s, shards=(i * per, (i + 1) * per))
 
     def run_overlap(self):
@@ -296,9 +331,12 @@ class Step:
                     self.s_att.wait_event(e_prep[i])
                     e_go[i].record(self.s_att)          # attention of range i may start
                     st.st_set_sm_budget(self.att_sms)
-                    for c in range(w.R):
-                        st.st_attn_spatial(self.qy, self.kc, self.vc, self.parts[c], self.lses[c],
-                                           desc=self.sdesc_sl[i][c])
+                    if self.fused_merge:
+                        self._spatial_fused(i)
+                    else:
+                        for c in range(w.R):
+                            st.st_attn_spatial(self.qy, self.kc, self.vc, self.parts[c], self.lses[c],
+                                               desc=self.sdesc_sl[i][c])
                     e_att[i].record(self.s_att)
                 with torch.cuda.stream(self.s_mem):
                     self.s_mem.wait_event(e_go[i])      # let the attention take its SMs first
@@ -351,13 +389,14 @@ def kernel_bytes(w, frac_active):
 def run_ours(args, w, rank, world, dev):
     import sequence_parallelism_st_b200 as st
     stp = Step(st, w, dev)
+    stp.fused_merge = args.merge == "fused"
     if args.schedule == "overlap":
         stp.setup_overlap(args.slices, args.att_sms)
         step_fn = stp.run_overlap
-        launches = (3 + 2 + w.R + 2) * args.slices + 1
+        launches = (3 + 3 + w.R + (1 if stp.fused_merge else 2)) * args.slices + 1
     else:
         step_fn = stp.run
-        launches = LAUNCHES_PER_STEP_BASE + w.R
+        launches = LAUNCHES_PER_STEP_BASE + w.R - (1 if stp.fused_merge else 0)
     pk, pk_src = peaks()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
@@ -462,8 +501,10 @@ def run_ours(args, w, rank, world, dev):
     kernels = {}
     for name, t in ktimes.items():
         ent = {"ms": round(t, 5)}
-        if name == "spatial":
-            ent["tflops"] = round(w.spatial_flops() / (t * 1e-3) / 1e12, 2)
+        if name in ("spatial", "spatial_merge"):
+            # fused merge: "spatial" is chunk 0, "spatial_merge" the other R-1 chunks with the merge
+            share = (1.0 if not stp.fused_merge else (1.0 / w.R if name == "spatial" else (w.R - 1.0) / w.R))
+            ent["tflops"] = round(w.spatial_flops() * share / (t * 1e-3) / 1e12, 2)
             ent["frac_of_bf16_peak"] = round(ent["tflops"] / pk["bf16_tflops"], 4)
         else:
             ent["gbs"] = round(kb[name] / (t * 1e-3) / 1e9, 1)
@@ -474,7 +515,7 @@ def run_ours(args, w, rank, world, dev):
     # roofline of the dominant kernel: spatial attention, R launches per step.
     # Peak: the burst GEMM figure while the clocks ran free, the sustained one
     # when the power cap throttled them during the timed region.
-    sp_launch_ms = ktimes["spatial"] / w.R
+    sp_launch_ms = ktimes["spatial"] / (1 if stp.fused_merge else w.R)   # one plain chunk launch
     achieved = (w.spatial_flops() / w.R) / (sp_launch_ms * 1e-3) / 1e12
     clocks = clk.summary()
     capped = "sw_power_cap" in clocks.get("reasons", []) and "bf16_tflops_sustained" in pk
@@ -488,7 +529,8 @@ def run_ours(args, w, rank, world, dev):
                    "N_T": w.n_t, "N_S": w.n_s, "kv_chunks": w.R, "vmajor_active": round(frac_active, 4),
                    "parallelism": f"replicas{world}", "l2": "flushed between timed steps (256 MiB write, "
                    "outside the step events)", "schedule": args.schedule if args.schedule == "serial" else
-                   f"overlap: {args.slices} shard ranges, attention on {args.att_sms} SMs"},
+                   f"overlap: {args.slices} shard ranges, attention on {args.att_sms} SMs",
+                   "chunk_merge": "fused into the attention kernel" if stp.fused_merge else "attn_chunk_merge"},
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(statistics.mean(e2e_ms), 5)},
         "roofline": {"bound": "tensor", "kernel": "st_attn_spatial", "achieved": round(achieved, 2),
@@ -569,6 +611,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="opensora_low")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--merge", choices=["fused", "separate"], default="fused",
+                    help="fused: KV chunks 1..R-1 merged inside the attention kernel; separate: attn_chunk_merge")
     ap.add_argument("--schedule", choices=["serial", "overlap"], default="serial",
                     help="overlap: shard ranges of the step on two streams (attention / memory-bound steps)")
     ap.add_argument("--slices", type=int, default=4, help="shard ranges of the overlap schedule")

@@ -106,20 +106,20 @@ template <int D, bool MERGE = false> struct Cfg {
   static constexpr bool ONES = DPV > D && (D + 15) / 16 <= 5;
   // Merge mode (the accumulated partial of earlier KV chunks is merged into
   // the result in the epilogue): for head dims up to 80 the epilogue stages
-  // the accumulated rows of an item in shared memory while the item runs
-  // (one 32 x 16 fp32 block per warp, tile and 16-column chunk), paid for
-  // with a single Q buffer and a shallower K/V ring; larger head dims load
-  // them from global memory one chunk ahead.
+  // the accumulated rows of one tile in shared memory (one 32 x 16 fp32 block
+  // per warp and 16-column chunk) -- tile A's while the item runs, tile B's
+  // while tile A is merged -- paid for with a shallower K/V ring; larger head
+  // dims load them from global memory one chunk ahead.
   static constexpr int NCH = (D + 15) / 16;            // 16-column chunks of O holding data
   static_assert(!MERGE || NCH <= 5, "staged merge only for head dims up to 80");
-  static constexpr int ACCS = MERGE ? 8 * NCH * EPI_BUF : 0;
+  static constexpr int ACCS = MERGE ? 4 * NCH * EPI_BUF : 0;
   static constexpr int VA = DPV / VW;                  // atoms
   static constexpr int VSW = VW * 2;                   // atom row bytes = swizzle span
   static constexpr int VAT = BLOCK_N * VSW;            // bytes of one atom region
   static constexpr int VTILE = VA * VAT;               // bytes of one V tile
   static constexpr int EPI = 4 * 2 * EPI_BUF + 2 * 2 * BLOCK_M * 4;
   static constexpr int BUDGET = MERGE ? 232448 - 4096 - EPI - ACCS : 204800;   // bytes for Q and the K/V ring
-  static constexpr int QB = (!MERGE && 4 * QTILE + 4 * (KTILE + VTILE) <= BUDGET) ? 2 : 1;   // Q double buffer if 4 stages fit
+  static constexpr int QB = (4 * QTILE + 4 * (KTILE + VTILE) <= BUDGET) ? 2 : 1;   // Q double buffer if 4 stages fit
   static constexpr int NS_RAW = (BUDGET - 2 * QB * QTILE) / (KTILE + VTILE);
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;   // K/V ring depth
   // epilogue: two staging buffers per epilogue warp, then the row statistics (m, l) of both tiles (EPI above)
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *sQ = base;                          // QB x 2 Q tiles
   uint8_t *sK = sQ + QB * 2 * K::QTILE;        // NS K tiles
   uint8_t *sV = sK + NS * K::KTILE;            // NS V tiles
-  uint8_t *sAcc = sV + NS * K::VTILE;          // merge mode: [tile][epilogue warp][chunk] 32 x 16 fp32 blocks
+  uint8_t *sAcc = sV + NS * K::VTILE;          // merge mode: [epilogue warp][chunk] 32 x 16 fp32 blocks
   uint8_t *sEpi = sAcc + K::ACCS;              // 4 warps x 2 staging buffers
   float *sStat = reinterpret_cast<float *>(sEpi + 4 * 2 * EPI_BUF);   // [tile][m | l][row]
   uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + K::EPI);
@@ -779,6 +779,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     bool acc_pending[2] = {false, false};      // merge mode: staged loads issued and not yet waited for
     uint32_t acc_par[2] = {0u, 0u};            // ... and the barrier phase they complete
+    // the copy engine brings the accumulated rows of tile XX of the current
+    // item (this warp's 32 rows, every chunk) into this warp's staging area
+#define STAGE_ACC(XX, ROW0)                                                                                  \
+  {                                                                                                          \
+    __syncwarp(); /* the area's previous contents are read */                                                \
+    if (lane == 0) {                                                                                         \
+      fence_async_smem(); /* ... and ordered before the copies that overwrite them */                        \
+      mbar_expect_tx(acc_full + qd * 2 + (XX), K::NCH * EPI_BUF);                                            \
+      _Pragma("unroll") for (int k = 0; k < K::NCH; ++k)                                                     \
+        tma_load_5d(sAcc + (qd * K::NCH + k) * EPI_BUF, &tacc, acc_full + qd * 2 + (XX), k * EPI_COLS, it.h, \
+                    (ROW0), it.c3, it.c4);                                                                   \
+    }                                                                                                        \
+    acc_pending[XX] = true;                                                                                  \
+    acc_par[XX] = ((XX) ? oc1 : oc0) & 1; /* items of the tile so far = the phase of these copies */        \
+  }
     for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
       const Item it = decode(p, x);
       float la_t[2] = {-INFINITY, -INFINITY};  // merge mode: accumulated LSE of this lane's row per tile
@@ -790,18 +805,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int row0 = it.q0 + X * BLOCK_M + qd * 32;
           const int qrow = row0 + lane;
           if (qrow < g.S) la_t[X] = p.lse_acc[(((long long)it.b * g.T + it.t) * g.H + it.h) * g.S + qrow];
-          if constexpr (MERGE) {
-            __syncwarp();                      // the previous item's reads of the area are done
-            if (lane == 0) {
-              fence_async_smem();              // ... and ordered before the copies that overwrite it
-              mbar_expect_tx(acc_full + qd * 2 + X, K::NCH * EPI_BUF);
-#pragma unroll
-              for (int k = 0; k < K::NCH; ++k)
-                tma_load_5d(sAcc + ((X * 4 + qd) * K::NCH + k) * EPI_BUF, &tacc, acc_full + qd * 2 + X,
-                            k * EPI_COLS, it.h, row0, it.c3, it.c4);
-            }
-            acc_pending[X] = true;
-            acc_par[X] = (X ? oc1 : oc0) & 1;   // items of this tile so far = the phase of these copies
+          if (MERGE && X == 0) {
+            STAGE_ACC(0, row0);                // tile B's rows follow once tile A is merged
           } else if (qrow < g.S) {
             const float *src = p.o_acc + g.frame(it.b, it.t) + g.token(qrow) + (long long)it.h * D;
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(uint32_t(D * 4)) : "memory");
@@ -911,7 +916,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   __syncwarp();
                 }
                 // 64B swizzle of the fp32 block: 16-byte chunk f of row r at f ^ ((r >> 1) & 3)
-                const uint8_t *ab = sAcc + ((X * 4 + qd) * K::NCH + c0 + c) * EPI_BUF + lane * 64;
+                const uint8_t *ab = sAcc + (qd * K::NCH + c0 + c) * EPI_BUF + lane * 64;
 #pragma unroll
                 for (int f = 0; f < 4; ++f) an[f] = *reinterpret_cast<const float4 *>(ab + ((f ^ ((lane >> 1) & 3)) << 4));
               }
@@ -962,10 +967,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
 #undef ST_LOAD_ACC
         if (!ok) break;
+        // tile A is merged: its staging area takes tile B's rows (in L2 since the item started)
+        if (MERGE && merging && X == 0 && it.n_qt == 2) STAGE_ACC(1, it.q0 + BLOCK_M + qd * 32)
         if (valid && p.lse) p.lse[lse_idx] = lse_row;
       }
     }
     if (lane == 0) bulk_wait_all();
+#undef STAGE_ACC
     if (MERGE && lane == 0) {
       // after an abort: staged copies into this warp's area may still be in
       // flight; wait for them (bounded, ignoring the abort epoch) before exiting

@@ -96,3 +96,28 @@ def test_overlap_schedule_matches_serial(st, n_slices, att_sms):
         assert torch.equal(torch.cat(parts), idx_ref)
     assert st.st_get_sm_budget() == 0
     assert st.st_check_device_status() == st.ST_OK
+
+
+def test_fused_merge_step_matches_separate(st):
+    """The bench step with the merge fused into the attention kernel agrees with
+    the step that writes both partials and merges them with attn_chunk_merge
+    (bf16 tolerance on the spatial output; every other output bit for bit)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    w = synth.BY_NAME["opensora_low"]
+    stp = bench.Step(st, w, "cuda")
+    res = {}
+    for fused in (False, True):
+        stp.fused_merge = fused
+        stp.reset_caches()
+        stp.run()
+        torch.cuda.synchronize()
+        res[fused] = outputs(stp)
+    for i in (1, 2, 3, 4, 5, 6):                 # ot, kc, vc, mask, idx, count
+        assert torch.equal(res[True][i], res[False][i]), f"output {i} differs"
+    for i in (0, 7):                             # ox, oy: the spatial result, two merge orders
+        a, b = res[True][i].float(), res[False][i].float()
+        assert (a - b).abs().max().item() <= 2e-2
+        assert ((a - b).norm() / b.norm()).item() <= 5e-3
+    assert st.st_check_device_status() == st.ST_OK
