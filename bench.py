@@ -4,11 +4,16 @@ One step = one pass of every hot-path step over one ST-DiT attention block of
 the OpenSora-like low-resolution workload (B=1, T=16 frames, S=1200 tokens,
 16 heads x 72, bf16, virtual P=4, N_T=N_S=4, KV chunks R=2):
 
-  1. all-to-all S->T of Q and K with the fused per-head RMSNorm, and of V
-     (ulysses_relayout on the [B,N_T,N_S,T/N_T,S/N_S/P,C] slice layouts);
-  2. V-Major change mask of V against the previous step's V, compaction of
-     the active tokens (vmajor_mask_compact), cache update of K/V rows of the
-     active tokens (vmajor_scatter_rows);
+  1. V-Major on the sending side: the L1 change of V against the previous
+     step's V is measured on the spatially sharded layout, and only the
+     active tokens take part in the all-to-all S->T -- their V rows and
+     their per-head RMS-normalised K rows go straight into the K/V caches in
+     the temporally sharded layout (vmajor_relayout_mask, which also writes
+     the mask and the ascending list of active tokens, and
+     vmajor_relayout_rows); ``--vmajor receiver`` moves all of K and V
+     (ulysses_relayout), takes the mask there and scatters the active rows
+     (vmajor_mask_compact, vmajor_scatter_rows) instead;
+  2. all-to-all S->T of Q with the fused per-head RMSNorm (ulysses_relayout);
   3. spatial attention of the fresh Q against the cached K/V in R KV chunks
      and their log-sum-exp merge: chunk 0 writes the fp32 partial and its LSE
      (st_attn_spatial), every later chunk merges into it inside the attention
@@ -143,8 +148,11 @@ class Step:
         v = vcur.reshape(B, T, S, H, D)
         self.host = {"q": self.to_x(q), "k": self.to_x(k), "v": self.to_x(v)}
         self.gamma = synth.rms_gamma(w).to(dev)
-        # previous step's V and K/V caches, already in the temporally sharded (y) layout
-        vprev_y = self.x_to_y_host(self.to_x(vprev.reshape(B, T, S, H, D)))
+        # previous step's V (in both layouts: the sender-side V-Major compares on x)
+        # and the K/V caches, already in the temporally sharded (y) layout
+        vprev_x = self.to_x(vprev.reshape(B, T, S, H, D))
+        self.vprev_x = vprev_x.to(dev)
+        vprev_y = self.x_to_y_host(vprev_x)
         kprev = synth.randn(w, "kprev", (B, T, S, H, D))
         kprev_y = self.x_to_y_host(self.to_x(kprev))
         self.d = {name: t.to(dev) for name, t in self.host.items()}
@@ -163,6 +171,9 @@ class Step:
         assert T % (w.n_t * P) == 0 and T // (w.n_t * P) == 1
         self.sdesc = [st.make_desc(1, T, S, H, D, st.ST_BF16, kv_begin=c * S // w.R, kv_end=(c + 1) * S // w.R,
                                    o_fp32=1) for c in range(w.R)]
+        # sender-side V-Major: the mask is taken on x and only active K/V rows move
+        # (into the caches); receiver side: full relayouts, mask on y, scatter
+        self.sender_vmajor = True
         # fused merge: chunk c >= 1 is merged into the accumulated fp32 partial
         # inside the attention kernel; the last chunk writes the bf16 result
         self.fused_merge = True
@@ -206,19 +217,34 @@ class Step:
         st, w, d = self.st, self.w, self.d
         self.timing = timing
         P, B, T, S, C, D = w.P, w.B, w.T, w.S, w.C, w.D
-        self._mark("relayout_s2t", True)
-        st.ulysses_relayout("S2T", d["q"], self.qy, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
-                            rms_head_dim=D, rms_eps=w.rms_eps)
-        st.ulysses_relayout("S2T", d["k"], self.ky, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
-                            rms_head_dim=D, rms_eps=w.rms_eps)
-        st.ulysses_relayout("S2T", d["v"], self.vy, P, B, T, S, C, w.n_t, w.n_s)
-        self._mark("relayout_s2t", False)
-        self._mark("vmajor", True)
-        st.vmajor_mask_compact(self.vy.view(self.n, C), self.vprev_y.view(self.n, C), self.tau, self.mask,
-                               self.idx, self.count, self.ws)
-        st.vmajor_scatter_rows(self.idx, self.count, [self.ky.view(self.n, C), self.vy.view(self.n, C)],
-                               [self.kc.view(self.n, C), self.vc.view(self.n, C)])
-        self._mark("vmajor", False)
+        if self.sender_vmajor:
+            # V-Major on the sending side: V's change decides which tokens take
+            # part in the exchange; their V and (normalised) K rows go straight
+            # into the caches, Q moves whole
+            self._mark("vmajor", True)
+            st.vmajor_relayout_mask(d["v"], self.vprev_x, self.vc, P, B, T, S, C, w.n_t, w.n_s, self.tau, self.mask,
+                                    self.idx, self.count, self.ws)
+            st.vmajor_relayout_rows(d["k"], self.kc, self.mask, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
+                                    rms_head_dim=D, rms_eps=w.rms_eps)
+            self._mark("vmajor", False)
+            self._mark("relayout_s2t", True)
+            st.ulysses_relayout("S2T", d["q"], self.qy, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
+                                rms_head_dim=D, rms_eps=w.rms_eps)
+            self._mark("relayout_s2t", False)
+        else:
+            self._mark("relayout_s2t", True)
+            st.ulysses_relayout("S2T", d["q"], self.qy, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
+                                rms_head_dim=D, rms_eps=w.rms_eps)
+            st.ulysses_relayout("S2T", d["k"], self.ky, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
+                                rms_head_dim=D, rms_eps=w.rms_eps)
+            st.ulysses_relayout("S2T", d["v"], self.vy, P, B, T, S, C, w.n_t, w.n_s)
+            self._mark("relayout_s2t", False)
+            self._mark("vmajor", True)
+            st.vmajor_mask_compact(self.vy.view(self.n, C), self.vprev_y.view(self.n, C), self.tau, self.mask,
+                                   self.idx, self.count, self.ws)
+            st.vmajor_scatter_rows(self.idx, self.count, [self.ky.view(self.n, C), self.vy.view(self.n, C)],
+                                   [self.kc.view(self.n, C), self.vc.view(self.n, C)])
+            self._mark("vmajor", False)
         if self.fused_merge:
             self._spatial_fused(None)
         else:
@@ -264,6 +290,7 @@ class Step:
         w = self.w
         assert w.P % n_slices == 0
         self.n_sl, self.att_sms = n_slices, att_sms
+        self.sender_vmajor = False          # the shard-range schedule moves whole ranges (receiver side)
         self.s_att = torch.cuda.Stream(priority=-8)     # mapped to the highest priority the device has
         self.s_mem = torch.cuda.Stream(priority=0)
         n_sl_tok = self.n // n_slices
@@ -373,10 +400,15 @@ def flops(w):
     return w.spatial_flops() + w.temporal_flops()
 
 
-def kernel_bytes(w, frac_active):
+def kernel_bytes(w, frac_active, sender=False):
     """Algorithmic HBM bytes per step of each memory-bound kernel group."""
     e = w.elem_bytes
     t = w.B * w.T * w.S * w.C * e               # one [B,T,S,C] tensor
+    if sender:
+        # V and its previous value read once on x, the active rows of V written
+        # and of K read and written; Q moved whole
+        return {"relayout_s2t": 2 * t, "vmajor": 2 * t + 3 * frac_active * t,
+                "merge": w.R * (2 * t + w.B * w.T * w.S * w.H * 4) + t, "relayout_t2s": 2 * t, "temporal": 4 * t}
     return {
         "relayout_s2t": 3 * 2 * t,
         "merge": w.R * (2 * t + w.B * w.T * w.S * w.H * 4) + t,  # fp32 partials + LSE in, bf16 out
@@ -390,13 +422,15 @@ def run_ours(args, w, rank, world, dev):
     import sequence_parallelism_st_b200 as st
     stp = Step(st, w, dev)
     stp.fused_merge = args.merge == "fused"
+    stp.sender_vmajor = args.vmajor == "sender"
     if args.schedule == "overlap":
         stp.setup_overlap(args.slices, args.att_sms)
         step_fn = stp.run_overlap
         launches = (3 + 3 + w.R + (1 if stp.fused_merge else 2)) * args.slices + 1
     else:
         step_fn = stp.run
-        launches = LAUNCHES_PER_STEP_BASE + w.R - (1 if stp.fused_merge else 0)
+        # sender-side V-Major: V mask-relayout, compaction and K rows (3) replace 2 relayouts + 3 V-Major launches
+        launches = LAUNCHES_PER_STEP_BASE + w.R - (1 if stp.fused_merge else 0) - (2 if stp.sender_vmajor else 0)
     pk, pk_src = peaks()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
@@ -497,7 +531,7 @@ def run_ours(args, w, rank, world, dev):
     value = world * f / (ms * 1e-3) / 1e12
     e2e_val = world * f / (statistics.mean(e2e_ms) * 1e-3) / 1e12
     frac_active = active / stp.n
-    kb = kernel_bytes(w, frac_active)
+    kb = kernel_bytes(w, frac_active, stp.sender_vmajor)
     kernels = {}
     for name, t in ktimes.items():
         ent = {"ms": round(t, 5)}
@@ -530,7 +564,9 @@ def run_ours(args, w, rank, world, dev):
                    "parallelism": f"replicas{world}", "l2": "flushed between timed steps (256 MiB write, "
                    "outside the step events)", "schedule": args.schedule if args.schedule == "serial" else
                    f"overlap: {args.slices} shard ranges, attention on {args.att_sms} SMs",
-                   "chunk_merge": "fused into the attention kernel" if stp.fused_merge else "attn_chunk_merge"},
+                   "chunk_merge": "fused into the attention kernel" if stp.fused_merge else "attn_chunk_merge",
+                   "vmajor": "sender side (mask on x, active K/V rows into the caches)" if stp.sender_vmajor else
+                   "receiver side (full relayouts, mask on y, scatter)"},
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(statistics.mean(e2e_ms), 5)},
         "roofline": {"bound": "tensor", "kernel": "st_attn_spatial", "achieved": round(achieved, 2),
@@ -613,6 +649,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--merge", choices=["fused", "separate"], default="fused",
                     help="fused: KV chunks 1..R-1 merged inside the attention kernel; separate: attn_chunk_merge")
+    ap.add_argument("--vmajor", choices=["sender", "receiver"], default="sender",
+                    help="sender: mask on x, only active K/V rows move into the caches; receiver: full relayouts, "
+                         "mask on y, scatter")
     ap.add_argument("--schedule", choices=["serial", "overlap"], default="serial",
                     help="overlap: shard ranges of the step on two streams (attention / memory-bound steps)")
     ap.add_argument("--slices", type=int, default=4, help="shard ranges of the overlap schedule")

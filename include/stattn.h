@@ -274,6 +274,36 @@ st_status vmajor_scatter_rows(const int *idx, const int *count, long long n_toke
                               void *const *dst_cache, int n_tensors,
                               void *const *packed, st_stream_t stream);
 
+/* Sender-side V-Major [CC "V-Major"]: the tokens whose V changed take part
+ * in the all-to-all, the others keep their cached rows.  v_cur_x and v_prev_x
+ * are V of this and of the previous step in the spatially sharded layout x of
+ * ulysses_relayout (ST_S2T shapes P, B, T, S, C, n_t, n_s); the L1 change of
+ * every token is measured there, and the row of every active token moves to
+ * its place in the temporally sharded layout y of v_cache_y (the V cache the
+ * spatial attention reads); rows of inactive tokens are not written.  mask,
+ * l1_out (optional), idx and count are those of vmajor_mask_compact in y
+ * numbering (row r of y = destination row r of the S2T exchange), with the
+ * same threshold rule, precision and determinism; workspace as for
+ * vmajor_mask_compact with n_tokens = B*T*S.  v_cache_y must not overlap the
+ * inputs.  Errors as for ulysses_relayout and vmajor_mask_compact. */
+st_status vmajor_relayout_mask(const void *v_cur_x, const void *v_prev_x, void *v_cache_y,
+                               int P, int B, int T, int S, int C, int n_t, int n_s,
+                               st_dtype dtype, float tau, int force_all,
+                               unsigned char *mask, int *idx, int *count, float *l1_out,
+                               void *workspace, size_t workspace_bytes, st_stream_t stream);
+
+/* The S2T move of ulysses_relayout restricted to the destination rows r
+ * whose mask[r] is nonzero (y numbering, as written by vmajor_relayout_mask):
+ * e.g. K of the active tokens into the K cache.  rms_gamma (optional, fp32
+ * device [rms_head_dim]) applies the per-head RMSNorm of ulysses_relayout on
+ * the way, with the same arithmetic, so a written row holds the same bytes
+ * as in the full relayout.  Rows with mask[r] == 0 are neither read nor
+ * written.  in_x and out_y must not overlap. */
+st_status vmajor_relayout_rows(const void *in_x, void *out_y, const unsigned char *mask,
+                               int P, int B, int T, int S, int C, int n_t, int n_s,
+                               st_dtype dtype, const float *rms_gamma, int rms_head_dim,
+                               float rms_eps, st_stream_t stream);
+
 /* vmajor_mask_compact and vmajor_scatter_rows (without `packed`) in one call
  * [CC "V-Major" section]: the pass that decides a token is active also copies
  * its rows of every src tensor into dst_cache, so the cache update reads no

@@ -8,7 +8,7 @@ Importing this module fails loudly when the library has not been built.
 Entry points (same names as the C ABI in include/stattn.h):
     st_attn_spatial, st_attn_spatial_merge, st_attn_temporal, attn_chunk_merge, ulysses_relayout,
     ulysses_relayout_range, vmajor_mask_compact, vmajor_mask_compact_noalloc, vmajor_mask_compact_scatter,
-    vmajor_scatter_rows, vmajor_workspace_bytes,
+    vmajor_scatter_rows, vmajor_workspace_bytes, vmajor_relayout_mask, vmajor_relayout_rows,
     st_check_device_status, st_status_string, st_set_sm_budget, st_get_sm_budget
 """
 from __future__ import annotations
@@ -81,6 +81,10 @@ _c = {
     "st_check_device_status": _proto("st_check_device_status", c_int, _VP),
     "st_selftest_wait_timeout": _proto("st_selftest_wait_timeout", c_int, _VP),
     "st_set_sm_budget": _proto("st_set_sm_budget", c_int, c_int),
+    "vmajor_relayout_mask": _proto("vmajor_relayout_mask", c_int, _VP, _VP, _VP, c_int, c_int, c_int, c_int, c_int,
+                                   c_int, c_int, c_int, c_float, c_int, _VP, _VP, _VP, _VP, _VP, c_size_t, _VP),
+    "vmajor_relayout_rows": _proto("vmajor_relayout_rows", c_int, _VP, _VP, _VP, c_int, c_int, c_int, c_int, c_int,
+                                   c_int, c_int, c_int, _VP, c_int, c_float, _VP),
     "st_get_sm_budget": _proto("st_get_sm_budget", c_int),
 }
 
@@ -89,7 +93,7 @@ EXPORTED = ["st_status_string", "st_abi_version", "st_attn_spatial", "st_attn_sp
             "ulysses_relayout", "vmajor_workspace_bytes", "vmajor_mask_compact", "vmajor_mask_compact_noalloc",
             "vmajor_scatter_rows", "vmajor_mask_compact_scatter",
             "st_check_device_status", "st_selftest_wait_timeout", "ulysses_relayout_range", "st_set_sm_budget",
-            "st_get_sm_budget"]
+            "st_get_sm_budget", "vmajor_relayout_mask", "vmajor_relayout_rows"]
 
 
 class StattnError(RuntimeError):
@@ -256,6 +260,25 @@ def vmajor_scatter_rows(idx, count, src, dst_cache, packed=None, *, stream=None,
     r = _c["vmajor_scatter_rows"](_ptr(idx), _ptr(count), n_tok, C, src[0].element_size(), sp, dp, n, pp,
                                   _stream(stream))
     return r if raw else _check(r, "vmajor_scatter_rows")
+
+
+def vmajor_relayout_mask(v_cur_x, v_prev_x, v_cache_y, P, B, T, S, C, n_t, n_s, tau, mask, idx, count, workspace,
+                         force_all=False, l1_out=None, *, stream=None, raw=False):
+    """Sender-side V-Major: mask of the L1 change of V on the x layout, rows of active
+    tokens moved S->T into the V cache; mask/idx/count in y numbering."""
+    r = _c["vmajor_relayout_mask"](_ptr(v_cur_x), _ptr(v_prev_x), _ptr(v_cache_y), P, B, T, S, C, n_t, n_s,
+                                   _dtype_code(v_cur_x), float(tau), 1 if force_all else 0, _ptr(mask), _ptr(idx),
+                                   _ptr(count), _ptr(l1_out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    return r if raw else _check(r, "vmajor_relayout_mask")
+
+
+def vmajor_relayout_rows(in_x, out_y, mask, P, B, T, S, C, n_t, n_s, rms_gamma=None, rms_head_dim=0, rms_eps=1e-6,
+                         *, stream=None, raw=False):
+    """S->T move of the destination rows whose mask byte is set (optional per-head RMSNorm)."""
+    r = _c["vmajor_relayout_rows"](_ptr(in_x), _ptr(out_y), _ptr(mask), P, B, T, S, C, n_t, n_s, _dtype_code(in_x),
+                                   _ptr(rms_gamma), int(rms_head_dim), float(rms_eps), _stream(stream))
+    return r if raw else _check(r, "vmajor_relayout_rows")
 
 
 def st_check_device_status(stream=None) -> int:

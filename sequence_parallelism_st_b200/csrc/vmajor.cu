@@ -238,6 +238,250 @@ __global__ void __launch_bounds__(256) scatter_rows(const int *__restrict__ idx,
 
 inline long long n_tiles_of(long long n) { return (n + TILE - 1) / TILE; }
 
+// ---------------------------------------------------------------- sender-side V-Major
+// V-Major decides on the sending side which tokens take part in the
+// all-to-all [CC "V-Major"]: the change of V is measured on the spatially
+// sharded layout x, and only the rows of active tokens move to their place in
+// the temporally sharded layout y -- straight into the K/V caches that the
+// attention reads.  Rows are enumerated in y order, so mask, per-tile counts
+// and the compaction come out in y numbering.
+
+// Destination row r of the S->T exchange -> its source row (the relayout
+// formulas of ulysses_relayout, for one row): r = (q, b, i, j, t2, s2) in y,
+// s2 = p * S/(N_S P) + s1, source (p, b, i, j, q * T/(N_T P) + t2, s1) in x.
+struct RowMap {
+  st::FastDiv fSs, fTq, fns, fnt, fB, fSp;
+  int Ss, Tq, n_s, n_t, B, Sp, Tn;
+};
+
+__device__ __forceinline__ long long y_to_x(const RowMap &m, long long r) {
+  uint32_t g = uint32_t(r);                    // rows < 2^31 (checked on the host)
+  const uint32_t rest = st::fdiv(g, m.fSs), s2 = g - rest * m.Ss;
+  const uint32_t blk = st::fdiv(rest, m.fTq), t2 = rest - blk * m.Tq;
+  const uint32_t b2 = st::fdiv(blk, m.fns), j = blk - b2 * m.n_s;
+  const uint32_t qb = st::fdiv(b2, m.fnt), i = b2 - qb * m.n_t;
+  const uint32_t q = st::fdiv(qb, m.fB), b = qb - q * m.B;
+  const uint32_t p = st::fdiv(s2, m.fSp), s1 = s2 - p * m.Sp;
+  const long long blk_x = (((long long)p * m.B + b) * m.n_t + i) * m.n_s + j;
+  return (blk_x * m.Tn + (long long)q * m.Tq + t2) * m.Sp + s1;
+}
+
+// l1_mask over destination rows: the current and previous V rows are read at
+// the source (x) row, the L1 change decides the mask of the destination row,
+// and an active row is stored into the V cache at the destination -- from the
+// registers that hold it when the row fits one pass of the warp, else read
+// again.
+template <typename T>
+__global__ void __launch_bounds__(THREADS, 2) l1_relayout(const char *__restrict__ cur, const char *__restrict__ prev,
+                                                       char *__restrict__ cache, long long n, int row_vecs,
+                                                       float tau, int force_all, unsigned char *__restrict__ mask,
+                                                       float *__restrict__ l1_out, int *__restrict__ tile_count,
+                                                       RowMap rm) {
+  constexpr int EPV = 16 / int(sizeof(T));
+  constexpr int TPW = 2;
+  constexpr int VM = 5;                          // 160 vectors per pass: a 1152-channel bf16 row in one
+  __shared__ int warp_cnt[THREADS / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  st::pdl_trigger();
+  st::pdl_wait();
+  cur = st::after_wait(cur);
+  prev = st::after_wait(prev);
+  const bool one_pass = row_vecs <= 32 * VM;
+  int active = 0;
+  for (int r = warp; r < TILE; r += TPW * (THREADS / 32)) {
+    long long tok[TPW], src[TPW];
+    float acc[TPW];
+    uint4 va[TPW][VM];
+#pragma unroll
+    for (int i = 0; i < TPW; ++i) {
+      tok[i] = (long long)blockIdx.x * TILE + r + i * (THREADS / 32);
+      src[i] = tok[i] < n ? y_to_x(rm, tok[i]) : 0;
+      acc[i] = 0.f;
+    }
+    for (int v0 = 0; v0 < row_vecs; v0 += 32 * VM) {
+      uint4 vb[TPW][VM];
+#pragma unroll
+      for (int i = 0; i < TPW; ++i) {
+        const uint4 *a = reinterpret_cast<const uint4 *>(cur) + src[i] * row_vecs;
+        const uint4 *b = reinterpret_cast<const uint4 *>(prev) + src[i] * row_vecs;
+#pragma unroll
+        for (int u = 0; u < VM; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (tok[i] < n && v < row_vecs) { va[i][u] = __ldg(a + v); vb[i][u] = __ldg(b + v); }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < TPW; ++i) {
+#pragma unroll
+        for (int u = 0; u < VM; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (tok[i] < n && v < row_vecs) {
+#pragma unroll
+            for (int k = 0; k < EPV; ++k) {
+              float x, y;
+              if constexpr (sizeof(T) == 2) {
+                x = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(&va[i][u])[k]);
+                y = st::bf16_to_f32(reinterpret_cast<const uint16_t *>(&vb[i][u])[k]);
+              } else {
+                x = reinterpret_cast<const float *>(&va[i][u])[k];
+                y = reinterpret_cast<const float *>(&vb[i][u])[k];
+              }
+              acc[i] += fabsf(x - y);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < TPW; ++i) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+      if (tok[i] < n) {
+        const int m = (force_all || acc[i] > tau) ? 1 : 0;   // the same on every lane (butterfly sum)
+        if (lane == 0) {
+          mask[tok[i]] = (unsigned char)m;
+          if (l1_out) l1_out[tok[i]] = acc[i];
+        }
+        active += m;
+        if (m) {
+          uint4 *d = reinterpret_cast<uint4 *>(cache) + tok[i] * row_vecs;
+          if (one_pass) {
+#pragma unroll
+            for (int u = 0; u < VM; ++u) {
+              const int v = u * 32 + lane;
+              if (v < row_vecs) d[v] = va[i][u];
+            }
+          } else {
+            const uint4 *a = reinterpret_cast<const uint4 *>(cur) + src[i] * row_vecs;
+            for (int v = lane; v < row_vecs; v += 32) d[v] = __ldg(a + v);
+          }
+        }
+      }
+    }
+  }
+  if (lane == 0) warp_cnt[warp] = active;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int c = 0;
+    for (int w = 0; w < THREADS / 32; ++w) c += warp_cnt[w];
+    tile_count[blockIdx.x] = c;
+  }
+}
+
+// The S->T move of the rows whose destination mask byte is set (K of the
+// active tokens into the K cache), with the optional per-head RMSNorm
+//   y_d = x_d / sqrt(mean_d x_d^2 + eps) * gamma_d   (fp32 math)
+// of ulysses_relayout, computed in the same order so that the bytes equal
+// the full relayout's.  A warp moves one row: it stages the row in shared
+// memory, one lane per head sums the squares (in the vector order the full
+// relayout's lane for that head would use), then every lane scales and
+// stores its vectors.
+template <typename T>
+__global__ void __launch_bounds__(256) rows_masked(const char *__restrict__ in, char *__restrict__ out,
+                                                   const unsigned char *__restrict__ mask, long long n, int row_vecs,
+                                                   const float *__restrict__ gamma, int D, float eps, RowMap rm) {
+  constexpr int EPV = 16 / int(sizeof(T));
+  extern __shared__ __align__(16) uint8_t rm_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  st::pdl_trigger();
+  st::pdl_wait();
+  in = st::after_wait(in);
+  mask = st::after_wait(mask);
+  const float *g = gamma ? st::after_wait(gamma) : nullptr;
+  const int VPH = g ? D / EPV : 1;                       // vectors per head
+  const int H = g ? row_vecs / VPH : 0;                  // heads per row
+  const int ROT = (g && VPH % 4 == 0) ? 1 : 0;
+  uint4 *buf = reinterpret_cast<uint4 *>(rm_smem) + (size_t)warp * (row_vecs + 8);
+  float *inv_s = reinterpret_cast<float *>(buf + row_vecs);   // up to 32 heads per pass
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n; r += nw) {
+    if (!mask[r]) continue;                              // warp-uniform
+    const long long sr = y_to_x(rm, r);
+    const uint4 *a = reinterpret_cast<const uint4 *>(in) + sr * row_vecs;
+    uint4 *d = reinterpret_cast<uint4 *>(out) + r * row_vecs;
+    if (!g) {
+      for (int v = lane; v < row_vecs; v += 32) d[v] = __ldg(a + v);
+      continue;
+    }
+    for (int v = lane; v < row_vecs; v += 32) buf[v] = __ldg(a + v);
+    __syncwarp();
+    const long long s1 = sr % rm.Sp;                    // the row's place in its segment
+    for (int h0 = 0; h0 < H; h0 += 32) {
+      const int h = h0 + lane;
+      if (h < H) {
+        // the full relayout handles head (s1 * H + h) of the segment on lane (s1 * H + h) % 32
+        const int r0 = int(((s1 * H + h) % 32) * ROT % VPH);
+        float ss = 0.f;
+        for (int u0 = 0; u0 < VPH; ++u0) {
+          const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
+          const uint4 v = buf[h * VPH + u];
+          if constexpr (sizeof(T) == 2) {
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float x0 = __uint_as_float(w[k] << 16), x1 = __uint_as_float(w[k] & 0xffff0000u);
+              ss = fmaf(x0, x0, ss);
+              ss = fmaf(x1, x1, ss);
+            }
+          } else {
+            ss = fmaf(__uint_as_float(v.x), __uint_as_float(v.x), ss);
+            ss = fmaf(__uint_as_float(v.y), __uint_as_float(v.y), ss);
+            ss = fmaf(__uint_as_float(v.z), __uint_as_float(v.z), ss);
+            ss = fmaf(__uint_as_float(v.w), __uint_as_float(v.w), ss);
+          }
+        }
+        inv_s[lane] = rsqrtf(ss * (1.0f / float(D)) + eps);
+      }
+      __syncwarp();
+      const int v_lo = h0 * VPH, v_hi = min(H, h0 + 32) * VPH;
+      for (int v = v_lo + lane; v < v_hi; v += 32) {
+        const int hh = v / VPH, u = v - hh * VPH;
+        const float inv = inv_s[hh - h0];
+        const float *gg = g + u * EPV;
+        uint4 x = buf[v];
+        if constexpr (sizeof(T) == 2) {
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            w[k] = st::pack_bf16x2(__uint_as_float(w[k] << 16) * inv * gg[2 * k],
+                                   __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1]);
+          x = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+          x = make_uint4(__float_as_uint(__uint_as_float(x.x) * inv * gg[0]),
+                         __float_as_uint(__uint_as_float(x.y) * inv * gg[1]),
+                         __float_as_uint(__uint_as_float(x.z) * inv * gg[2]),
+                         __float_as_uint(__uint_as_float(x.w) * inv * gg[3]));
+        }
+        d[v] = x;
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// Host-side check and map of the S->T exchange shape (elem: element bytes).
+st_status make_rowmap(int P, int B, int T, int S, int C, int n_t, int n_s, int elem, RowMap &m, long long &rows) {
+  if (P <= 0 || B <= 0 || T <= 0 || S <= 0 || C <= 0 || n_t <= 0 || n_s <= 0) return ST_ERR_SHAPE;
+  if (T % (n_t * P) || S % (n_s * P)) return ST_ERR_DIVISIBILITY;
+  if (((long long)C * elem) % 16) return ST_ERR_ALIGN;
+  rows = (long long)B * T * S;
+  if (rows >= (1LL << 31)) return ST_ERR_SHAPE;
+  m.Ss = S / n_s;
+  m.Tq = T / (n_t * P);
+  m.n_s = n_s;
+  m.n_t = n_t;
+  m.B = B;
+  m.Sp = S / (n_s * P);
+  m.Tn = T / n_t;
+  m.fSs = st::make_fastdiv(uint32_t(m.Ss));
+  m.fTq = st::make_fastdiv(uint32_t(m.Tq));
+  m.fns = st::make_fastdiv(uint32_t(n_s));
+  m.fnt = st::make_fastdiv(uint32_t(n_t));
+  m.fB = st::make_fastdiv(uint32_t(B));
+  m.fSp = st::make_fastdiv(uint32_t(m.Sp));
+  return ST_OK;
+}
+
 }  // namespace
 
 ST_API size_t vmajor_workspace_bytes(long long n_tokens) {
@@ -404,4 +648,69 @@ ST_API st_status vmajor_mask_compact_noalloc(const void *v_cur, const void *v_pr
   const int ctas = int((n_tokens + CTILE - 1) / CTILE);
   compact<<<ctas, THREADS, 0, s>>>(mask, n_tokens, ctas, tile_count, idx, count);
   return st::launch_status();
+}
+
+ST_API st_status vmajor_relayout_mask(const void *v_cur_x, const void *v_prev_x, void *v_cache_y, int P, int B, int T,
+                                      int S, int C, int n_t, int n_s, st_dtype dtype, float tau, int force_all,
+                                      unsigned char *mask, int *idx, int *count, float *l1_out, void *workspace,
+                                      size_t workspace_bytes, st_stream_t stream) {
+  if (!v_cur_x || !v_prev_x || !v_cache_y || !mask || !idx || !count || !workspace) return ST_ERR_NULL;
+  if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_DTYPE;
+  const int esize = dtype == ST_F32 ? 4 : 2;
+  RowMap rm;
+  long long n = 0;
+  st_status st = make_rowmap(P, B, T, S, C, n_t, n_s, esize, rm, n);
+  if (st != ST_OK) return st;
+  if (!st::is_aligned(v_cur_x, 16) || !st::is_aligned(v_prev_x, 16) || !st::is_aligned(v_cache_y, 16))
+    return ST_ERR_ALIGN;
+  if (workspace_bytes < vmajor_workspace_bytes(n)) return ST_ERR_SHAPE;
+  const long long bytes = n * C * esize;
+  const char *c0 = static_cast<const char *>(v_cur_x), *p0 = static_cast<const char *>(v_prev_x);
+  char *d0 = static_cast<char *>(v_cache_y);
+  if ((d0 < c0 + bytes && c0 < d0 + bytes) || (d0 < p0 + bytes && p0 < d0 + bytes)) return ST_ERR_SHAPE;  // overlap
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long tiles = n_tiles_of(n);
+  const int row_vecs = C * esize / 16;
+  int *tile_count = static_cast<int *>(workspace);
+  st = dtype == ST_BF16
+           ? st::launch_pdl(l1_relayout<uint16_t>, int(tiles), THREADS, 0, s, c0, p0, d0, n, row_vecs, tau,
+                            force_all, mask, l1_out, tile_count, rm)
+           : st::launch_pdl(l1_relayout<float>, int(tiles), THREADS, 0, s, c0, p0, d0, n, row_vecs, tau, force_all,
+                            mask, l1_out, tile_count, rm);
+  if (st != ST_OK) return st;
+  const int ctas = int((n + CTILE - 1) / CTILE);
+  return st::launch_pdl(compact, ctas, THREADS, 0, s, static_cast<const unsigned char *>(mask), n, ctas,
+                        static_cast<const int *>(tile_count), idx, count);
+}
+
+ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const unsigned char *mask, int P, int B, int T,
+                                      int S, int C, int n_t, int n_s, st_dtype dtype, const float *rms_gamma,
+                                      int rms_head_dim, float rms_eps, st_stream_t stream) {
+  if (!in_x || !out_y || !mask) return ST_ERR_NULL;
+  if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_DTYPE;
+  const int esize = dtype == ST_F32 ? 4 : 2;
+  RowMap rm;
+  long long n = 0;
+  st_status st = make_rowmap(P, B, T, S, C, n_t, n_s, esize, rm, n);
+  if (st != ST_OK) return st;
+  if (!st::is_aligned(in_x, 16) || !st::is_aligned(out_y, 16)) return ST_ERR_ALIGN;
+  const int row_vecs = C * esize / 16;
+  if (rms_gamma) {
+    if (rms_head_dim <= 0 || C % rms_head_dim || (rms_head_dim * esize) % 16) return ST_ERR_SHAPE;
+  }
+  const long long bytes = n * C * esize;
+  const char *i0 = static_cast<const char *>(in_x);
+  char *o0 = static_cast<char *>(out_y);
+  if (o0 < i0 + bytes && i0 < o0 + bytes) return ST_ERR_SHAPE;  // overlap
+  const size_t smem = size_t(8) * (row_vecs + 8) * 16;           // 8 warps: a row and the heads' scales each
+  if (smem > 227 * 1024) return ST_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto kern = dtype == ST_BF16 ? rows_masked<uint16_t> : rows_masked<float>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+    return ST_ERR_CUDA;
+  const long long want = (n + 7) / 8;
+  const long long cap = (long long)st::num_sms() * 8;
+  const int grid = int(want < cap ? want : cap);
+  return st::launch_pdl(kern, grid, 256, smem, s, i0, o0, mask, n, row_vecs, rms_gamma, rms_head_dim, rms_eps, rm);
 }

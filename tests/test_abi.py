@@ -150,3 +150,30 @@ def test_merge_and_vmajor_reject(st):
     assert h(FAKE_IN, FAKE_IN, 100, 64, 2, arr, arr, 0, None, None) == st.ST_ERR_SHAPE
     assert h(FAKE_IN, FAKE_IN, 100, 64, 2, arr, arr, 9, None, None) == st.ST_ERR_SHAPE
     assert h(FAKE_IN, FAKE_IN, 100, 64, 3, arr, arr, 2, None, None) == st.ST_ERR_DTYPE
+
+
+def test_sender_vmajor_rejects(st):
+    """vmajor_relayout_mask / vmajor_relayout_rows validate before any launch."""
+    VP = ctypes.c_void_p
+    ws = VP(0x300000)
+    m = st._c["vmajor_relayout_mask"]
+
+    def mask_call(P=2, T=8, S=16, C=64, n_t=1, n_s=1, dtype=st.ST_BF16, cur=FAKE_IN, cache=FAKE_OUT, wsb=1 << 20):
+        return m(cur, VP(0x200000), cache, P, 1, T, S, C, n_t, n_s, dtype, 1.0, 0, VP(0x400000), VP(0x500000),
+                 VP(0x600000), None, ws, wsb, None)
+    assert mask_call(cur=None) == st.ST_ERR_NULL
+    assert mask_call(dtype=7) == st.ST_ERR_DTYPE
+    assert mask_call(T=6, P=4) == st.ST_ERR_DIVISIBILITY
+    assert mask_call(S=16, P=2, n_s=3) == st.ST_ERR_DIVISIBILITY
+    assert mask_call(C=3) == st.ST_ERR_ALIGN
+    assert mask_call(cur=VP(0x100008)) == st.ST_ERR_ALIGN
+    assert mask_call(wsb=0) == st.ST_ERR_SHAPE
+    assert mask_call(cache=VP(0x100000 + 64)) == st.ST_ERR_SHAPE        # overlaps the input
+    r = st._c["vmajor_relayout_rows"]
+
+    def rows_call(gamma=None, hd=0, C=64, out=FAKE_OUT, mask=VP(0x400000)):
+        return r(FAKE_IN, out, mask, 2, 1, 8, 16, C, 1, 1, st.ST_BF16, gamma, hd, 1e-6, None)
+    assert rows_call(mask=None) == st.ST_ERR_NULL
+    assert rows_call(gamma=FAKE_IN, hd=48) == st.ST_ERR_SHAPE
+    assert rows_call(gamma=FAKE_IN, hd=4) == st.ST_ERR_SHAPE            # 8-byte heads: not 16-byte rows
+    assert rows_call(out=VP(0x100000 + 32)) == st.ST_ERR_SHAPE

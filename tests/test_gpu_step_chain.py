@@ -121,3 +121,25 @@ def test_fused_merge_step_matches_separate(st):
         assert (a - b).abs().max().item() <= 2e-2
         assert ((a - b).norm() / b.norm()).item() <= 5e-3
     assert st.st_check_device_status() == st.ST_OK
+
+
+def test_sender_vmajor_step_matches_receiver(st):
+    """Sender-side V-Major (mask on x, only active K/V rows moved into the
+    caches) gives the receiver-side step's bits: mask, compaction, caches,
+    and every attention output."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    w = synth.BY_NAME["opensora_low"]
+    stp = bench.Step(st, w, "cuda")
+    res = {}
+    for sender in (False, True):
+        stp.sender_vmajor = sender
+        stp.reset_caches()
+        stp.idx.fill_(-1)
+        stp.run()
+        torch.cuda.synchronize()
+        res[sender] = outputs(stp) + [stp.qy.clone()]
+    for i, (a, b) in enumerate(zip(res[True], res[False])):
+        assert torch.equal(a, b), f"output {i} differs between sender and receiver V-Major"
+    assert st.st_check_device_status() == st.ST_OK
