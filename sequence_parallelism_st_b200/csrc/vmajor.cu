@@ -368,94 +368,23 @@ __global__ void __launch_bounds__(THREADS, 2) l1_relayout(const char *__restrict
   }
 }
 
-// The S->T move of the rows whose destination mask byte is set (K of the
-// active tokens into the K cache), with the optional per-head RMSNorm
-//   y_d = x_d / sqrt(mean_d x_d^2 + eps) * gamma_d   (fp32 math)
-// of ulysses_relayout, computed in the same order so that the bytes equal
-// the full relayout's.  A warp moves one row: it stages the row in shared
-// memory, one lane per head sums the squares (in the vector order the full
-// relayout's lane for that head would use), then every lane scales and
-// stores its vectors.
-template <typename T>
+// The S->T move of the rows whose destination mask byte is set (without the
+// RMSNorm; with it the bulk-copy RMS kernel of ulysses_relayout does the
+// move): a warp copies one row with 16-byte vectors.
 __global__ void __launch_bounds__(256) rows_masked(const char *__restrict__ in, char *__restrict__ out,
                                                    const unsigned char *__restrict__ mask, long long n, int row_vecs,
-                                                   const float *__restrict__ gamma, int D, float eps, RowMap rm) {
-  constexpr int EPV = 16 / int(sizeof(T));
-  extern __shared__ __align__(16) uint8_t rm_smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                                   RowMap rm) {
+  const int lane = threadIdx.x & 31;
   st::pdl_trigger();
   st::pdl_wait();
   in = st::after_wait(in);
   mask = st::after_wait(mask);
-  const float *g = gamma ? st::after_wait(gamma) : nullptr;
-  const int VPH = g ? D / EPV : 1;                       // vectors per head
-  const int H = g ? row_vecs / VPH : 0;                  // heads per row
-  const int ROT = (g && VPH % 4 == 0) ? 1 : 0;
-  uint4 *buf = reinterpret_cast<uint4 *>(rm_smem) + (size_t)warp * (row_vecs + 8);
-  float *inv_s = reinterpret_cast<float *>(buf + row_vecs);   // up to 32 heads per pass
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
   for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n; r += nw) {
     if (!mask[r]) continue;                              // warp-uniform
-    const long long sr = y_to_x(rm, r);
-    const uint4 *a = reinterpret_cast<const uint4 *>(in) + sr * row_vecs;
+    const uint4 *a = reinterpret_cast<const uint4 *>(in) + y_to_x(rm, r) * row_vecs;
     uint4 *d = reinterpret_cast<uint4 *>(out) + r * row_vecs;
-    if (!g) {
-      for (int v = lane; v < row_vecs; v += 32) d[v] = __ldg(a + v);
-      continue;
-    }
-    for (int v = lane; v < row_vecs; v += 32) buf[v] = __ldg(a + v);
-    __syncwarp();
-    const long long s1 = sr % rm.Sp;                    // the row's place in its segment
-    for (int h0 = 0; h0 < H; h0 += 32) {
-      const int h = h0 + lane;
-      if (h < H) {
-        // the full relayout handles head (s1 * H + h) of the segment on lane (s1 * H + h) % 32
-        const int r0 = int(((s1 * H + h) % 32) * ROT % VPH);
-        float ss = 0.f;
-        for (int u0 = 0; u0 < VPH; ++u0) {
-          const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
-          const uint4 v = buf[h * VPH + u];
-          if constexpr (sizeof(T) == 2) {
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float x0 = __uint_as_float(w[k] << 16), x1 = __uint_as_float(w[k] & 0xffff0000u);
-              ss = fmaf(x0, x0, ss);
-              ss = fmaf(x1, x1, ss);
-            }
-          } else {
-            ss = fmaf(__uint_as_float(v.x), __uint_as_float(v.x), ss);
-            ss = fmaf(__uint_as_float(v.y), __uint_as_float(v.y), ss);
-            ss = fmaf(__uint_as_float(v.z), __uint_as_float(v.z), ss);
-            ss = fmaf(__uint_as_float(v.w), __uint_as_float(v.w), ss);
-          }
-        }
-        inv_s[lane] = rsqrtf(ss * (1.0f / float(D)) + eps);
-      }
-      __syncwarp();
-      const int v_lo = h0 * VPH, v_hi = min(H, h0 + 32) * VPH;
-      for (int v = v_lo + lane; v < v_hi; v += 32) {
-        const int hh = v / VPH, u = v - hh * VPH;
-        const float inv = inv_s[hh - h0];
-        const float *gg = g + u * EPV;
-        uint4 x = buf[v];
-        if constexpr (sizeof(T) == 2) {
-          uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            w[k] = st::pack_bf16x2(__uint_as_float(w[k] << 16) * inv * gg[2 * k],
-                                   __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1]);
-          x = make_uint4(w[0], w[1], w[2], w[3]);
-        } else {
-          x = make_uint4(__float_as_uint(__uint_as_float(x.x) * inv * gg[0]),
-                         __float_as_uint(__uint_as_float(x.y) * inv * gg[1]),
-                         __float_as_uint(__uint_as_float(x.z) * inv * gg[2]),
-                         __float_as_uint(__uint_as_float(x.w) * inv * gg[3]));
-        }
-        d[v] = x;
-      }
-      __syncwarp();
-    }
+    for (int v = lane; v < row_vecs; v += 32) d[v] = __ldg(a + v);
   }
 }
 
@@ -702,15 +631,13 @@ ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const unsig
   const char *i0 = static_cast<const char *>(in_x);
   char *o0 = static_cast<char *>(out_y);
   if (o0 < i0 + bytes && i0 < o0 + bytes) return ST_ERR_SHAPE;  // overlap
-  const size_t smem = size_t(8) * (row_vecs + 8) * 16;           // 8 warps: a row and the heads' scales each
-  if (smem > 227 * 1024) return ST_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  auto kern = dtype == ST_BF16 ? rows_masked<uint16_t> : rows_masked<float>;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-    return ST_ERR_CUDA;
+  // with the RMSNorm: the bulk-copy kernel of ulysses_relayout, restricted to the masked rows
+  if (rms_gamma)
+    return st::relayout_s2t_rms_masked(in_x, out_y, mask, esize, P, B, T, S, C, n_t, n_s, rms_gamma, rms_head_dim,
+                                       rms_eps, s);
   const long long want = (n + 7) / 8;
-  const long long cap = (long long)st::num_sms() * 8;
+  const long long cap = (long long)st::num_sms() * 16;
   const int grid = int(want < cap ? want : cap);
-  return st::launch_pdl(kern, grid, 256, smem, s, i0, o0, mask, n, row_vecs, rms_gamma, rms_head_dim, rms_eps, rm);
+  return st::launch_pdl(rows_masked, grid, 256, 0, s, i0, o0, mask, n, row_vecs, rm);
 }
