@@ -785,6 +785,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   {                                                                                                          \
     __syncwarp(); /* the area's previous contents are read */                                                \
     if (lane == 0) {                                                                                         \
+      bulk_wait_read0(); /* ... also by the stores of merged blocks that went out from it */                 \
       fence_async_smem(); /* ... and ordered before the copies that overwrite them */                        \
       mbar_expect_tx(acc_full + qd * 2 + (XX), K::NCH * EPI_BUF);                                            \
       _Pragma("unroll") for (int k = 0; k < K::NCH; ++k)                                                     \
@@ -934,8 +935,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(ov[c][e]) * inv;
             }
-            if (lane == 0) bulk_wait_read1();  // the store that used this buffer has read it
-            __syncwarp();
+            if constexpr (MERGE) {
+              // the merged block goes out from the slot its accumulated block
+              // came from (every lane has read its row of it); one store per
+              // block once the tile's blocks are all written
+              buf = sAcc + (qd * K::NCH + c0 + c) * EPI_BUF;
+              __syncwarp();
+            } else {
+              if (lane == 0) bulk_wait_read1();  // the store that used this buffer has read it
+              __syncwarp();
+            }
             if (p.o_f32) {
               // 64-byte rows, 64B swizzle: 16-byte chunk f of row r at f ^ ((r >> 1) & 3)
 #pragma unroll
@@ -954,12 +963,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
               }
             }
+            if (!MERGE) {
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                // a block wholly past the last row stores nothing, but still
+                // commits a (empty) group so the buffer accounting stays in step
+                if (row0 < g.S) tma_store_5d(&to, buf, (c0 + c) * EPI_COLS, it.h, row0, it.c3, it.c4);
+                bulk_commit();
+              }
+            }
+          }
+          if (MERGE && ok) {                   // the tile's merged blocks, one bulk store each
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) {
-              // a block wholly past the last row stores nothing, but still
-              // commits a (empty) group so the buffer accounting stays in step
-              if (row0 < g.S) tma_store_5d(&to, buf, (c0 + c) * EPI_COLS, it.h, row0, it.c3, it.c4);
+            if (lane == 0 && row0 < g.S) {
+              for (int c = 0; c < nch; ++c)
+                tma_store_5d(&to, sAcc + (qd * K::NCH + c0 + c) * EPI_BUF, (c0 + c) * EPI_COLS, it.h, row0,
+                             it.c3, it.c4);
               bulk_commit();
             }
           }
