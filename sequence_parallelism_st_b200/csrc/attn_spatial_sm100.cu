@@ -112,13 +112,17 @@ template <int D, bool MERGE = false> struct Cfg {
   // dims load them from global memory one chunk ahead.
   static constexpr int NCH = (D + 15) / 16;            // 16-column chunks of O holding data
   static_assert(!MERGE || NCH <= 5, "staged merge only for head dims up to 80");
-  static constexpr int ACCS = MERGE ? 4 * NCH * EPI_BUF : 0;
+  // Head dims up to 80 write the output of a tile through per-warp slots, one
+  // 32 x 16 block per chunk, and store them once per tile; merge mode first
+  // stages the accumulated blocks in the same slots.
+  static constexpr bool SLOTS = NCH <= 5;
+  static constexpr int ACCS = SLOTS ? 4 * NCH * EPI_BUF : 0;
   static constexpr int VA = DPV / VW;                  // atoms
   static constexpr int VSW = VW * 2;                   // atom row bytes = swizzle span
   static constexpr int VAT = BLOCK_N * VSW;            // bytes of one atom region
   static constexpr int VTILE = VA * VAT;               // bytes of one V tile
   static constexpr int EPI = 4 * 2 * EPI_BUF + 2 * 2 * BLOCK_M * 4;
-  static constexpr int BUDGET = MERGE ? 232448 - 4096 - EPI - ACCS : 204800;   // bytes for Q and the K/V ring
+  static constexpr int BUDGET = SLOTS ? 232448 - 4096 - EPI - ACCS : 204800;   // bytes for Q and the K/V ring
   static constexpr int QB = (4 * QTILE + 4 * (KTILE + VTILE) <= BUDGET) ? 2 : 1;   // Q double buffer if 4 stages fit
   static constexpr int NS_RAW = (BUDGET - 2 * QB * QTILE) / (KTILE + VTILE);
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;   // K/V ring depth
@@ -935,10 +939,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(ov[c][e]) * inv;
             }
-            if constexpr (MERGE) {
-              // the merged block goes out from the slot its accumulated block
-              // came from (every lane has read its row of it); one store per
-              // block once the tile's blocks are all written
+            if constexpr (K::SLOTS) {
+              // the block goes out from its slot (merge mode: the slot its
+              // accumulated block came from, which every lane has read), one
+              // store per block once the tile's blocks are all written; the
+              // stores of the previous tile must have read the slots
+              if (!MERGE && c0 + c == 0 && lane == 0) bulk_wait_read0();
               buf = sAcc + (qd * K::NCH + c0 + c) * EPI_BUF;
               __syncwarp();
             } else {
@@ -963,7 +969,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 *reinterpret_cast<uint4 *>(buf + lane * 32 + ((f ^ ((lane >> 2) & 1)) << 4)) = w;
               }
             }
-            if (!MERGE) {
+            if (!K::SLOTS) {
               fence_async_smem();
               __syncwarp();
               if (lane == 0) {
@@ -974,7 +980,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
           }
-          if (MERGE && ok) {                   // the tile's merged blocks, one bulk store each
+          if (K::SLOTS && ok) {                // the tile's blocks, one bulk store each
             fence_async_smem();
             __syncwarp();
             if (lane == 0 && row0 < g.S) {
