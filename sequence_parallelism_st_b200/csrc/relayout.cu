@@ -244,6 +244,19 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
     }
     return act;
   };
+  // With a row mask, lane k works out up front which heads of the warp's
+  // k-th task move (the mask reads of all its tasks in one round trip).
+  uint32_t pre_act = 0;
+  const bool pre = row_mask && one_src && (n_tasks - gw + nw - 1) / nw <= 32;
+  if (pre) {
+    const long long t = gw + lane * nw;
+    if (t < n_tasks) {
+      const long long seg = t / tps, c = t - seg * tps;
+      long long so, dof;
+      map_segment(m, seg, so, dof);
+      pre_act = active_heads(dof + c * 32 * HB, int(min(32LL, hps - c * 32)));
+    }
+  }
   // task -> (destination byte offset, number of heads, heads to move); issues its load into buffer b
   auto issue = [&](long long task, int b, long long &dst, int &nh, uint32_t &act) {
     uint8_t *bufp = buf0 + b * BUF;
@@ -254,9 +267,9 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
       long long so, dof;
       map_segment(m, seg, so, dof);
       dst = dof + c * 32 * HB;
-      act = 0;
+      act = pre ? __shfl_sync(0xffffffffu, pre_act, int((task - gw) / nw)) : 0u;
       if (lane == 0) {
-        act = active_heads(dst, nh);
+        if (!pre) act = active_heads(dst, nh);
         expect_tx(&full[warp][b], __popc(act) * HB);   // 0 bytes: the phase completes at once
         for (uint32_t rest = act; rest;) {              // one copy per run of heads
           const int lo = __ffs(rest) - 1;
