@@ -224,8 +224,8 @@ class Step:
             self._mark("vmajor", True)
             st.vmajor_relayout_mask(d["v"], self.vprev_x, self.vc, P, B, T, S, C, w.n_t, w.n_s, self.tau, self.mask,
                                     self.idx, self.count, self.ws)
-            st.vmajor_relayout_rows(d["k"], self.kc, self.mask, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
-                                    rms_head_dim=D, rms_eps=w.rms_eps)
+            st.vmajor_relayout_rows(d["k"], self.kc, self.idx, self.count, P, B, T, S, C, w.n_t, w.n_s,
+                                    rms_gamma=self.gamma, rms_head_dim=D, rms_eps=w.rms_eps)
             self._mark("vmajor", False)
             self._mark("relayout_s2t", True)
             st.ulysses_relayout("S2T", d["q"], self.qy, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,

@@ -292,14 +292,15 @@ st_status vmajor_relayout_mask(const void *v_cur_x, const void *v_prev_x, void *
                                unsigned char *mask, int *idx, int *count, float *l1_out,
                                void *workspace, size_t workspace_bytes, st_stream_t stream);
 
-/* The S2T move of ulysses_relayout restricted to the destination rows r
- * whose mask[r] is nonzero (y numbering, as written by vmajor_relayout_mask):
- * e.g. K of the active tokens into the K cache.  rms_gamma (optional, fp32
- * device [rms_head_dim]) applies the per-head RMSNorm of ulysses_relayout on
- * the way, with the same arithmetic, so a written row holds the same bytes
- * as in the full relayout.  Rows with mask[r] == 0 are neither read nor
- * written.  in_x and out_y must not overlap. */
-st_status vmajor_relayout_rows(const void *in_x, void *out_y, const unsigned char *mask,
+/* The S2T move of ulysses_relayout restricted to the destination rows
+ * idx[0], ..., idx[*count - 1] (y numbering, as listed by vmajor_relayout_mask;
+ * idx and count are device memory): e.g. K of the active tokens into the K
+ * cache [CC "V-Major"].  rms_gamma (optional, fp32 device [rms_head_dim])
+ * applies the per-head RMSNorm of ulysses_relayout on the way, with the same
+ * arithmetic, so a written row holds the same bytes as in the full relayout;
+ * with it a row may hold at most 32 heads (else ST_ERR_UNSUPPORTED).  Rows
+ * not listed are neither read nor written.  in_x and out_y must not overlap. */
+st_status vmajor_relayout_rows(const void *in_x, void *out_y, const int *idx, const int *count,
                                int P, int B, int T, int S, int C, int n_t, int n_s,
                                st_dtype dtype, const float *rms_gamma, int rms_head_dim,
                                float rms_eps, st_stream_t stream);

@@ -83,8 +83,8 @@ _c = {
     "st_set_sm_budget": _proto("st_set_sm_budget", c_int, c_int),
     "vmajor_relayout_mask": _proto("vmajor_relayout_mask", c_int, _VP, _VP, _VP, c_int, c_int, c_int, c_int, c_int,
                                    c_int, c_int, c_int, c_float, c_int, _VP, _VP, _VP, _VP, _VP, c_size_t, _VP),
-    "vmajor_relayout_rows": _proto("vmajor_relayout_rows", c_int, _VP, _VP, _VP, c_int, c_int, c_int, c_int, c_int,
-                                   c_int, c_int, c_int, _VP, c_int, c_float, _VP),
+    "vmajor_relayout_rows": _proto("vmajor_relayout_rows", c_int, _VP, _VP, _VP, _VP, c_int, c_int, c_int, c_int,
+                                   c_int, c_int, c_int, c_int, _VP, c_int, c_float, _VP),
     "st_get_sm_budget": _proto("st_get_sm_budget", c_int),
 }
 
@@ -273,11 +273,12 @@ def vmajor_relayout_mask(v_cur_x, v_prev_x, v_cache_y, P, B, T, S, C, n_t, n_s, 
     return r if raw else _check(r, "vmajor_relayout_mask")
 
 
-def vmajor_relayout_rows(in_x, out_y, mask, P, B, T, S, C, n_t, n_s, rms_gamma=None, rms_head_dim=0, rms_eps=1e-6,
-                         *, stream=None, raw=False):
-    """S->T move of the destination rows whose mask byte is set (optional per-head RMSNorm)."""
-    r = _c["vmajor_relayout_rows"](_ptr(in_x), _ptr(out_y), _ptr(mask), P, B, T, S, C, n_t, n_s, _dtype_code(in_x),
-                                   _ptr(rms_gamma), int(rms_head_dim), float(rms_eps), _stream(stream))
+def vmajor_relayout_rows(in_x, out_y, idx, count, P, B, T, S, C, n_t, n_s, rms_gamma=None, rms_head_dim=0,
+                         rms_eps=1e-6, *, stream=None, raw=False):
+    """S->T move of the destination rows idx[:count] (device), with the optional per-head RMSNorm."""
+    r = _c["vmajor_relayout_rows"](_ptr(in_x), _ptr(out_y), _ptr(idx), _ptr(count), P, B, T, S, C, n_t, n_s,
+                                   _dtype_code(in_x), _ptr(rms_gamma), int(rms_head_dim), float(rms_eps),
+                                   _stream(stream))
     return r if raw else _check(r, "vmajor_relayout_rows")
 
 

@@ -69,6 +69,7 @@ st_status relayout_s2t_rms_masked(const void *in, void *out, const unsigned char
 // (defined next to that kernel).  Returns the word's previous value.
 unsigned int read_and_clear_attn_error(cudaStream_t stream, cudaError_t *err);
 unsigned int read_and_clear_relayout_error(cudaStream_t stream, cudaError_t *err);
+unsigned int read_and_clear_vmajor_error(cudaStream_t stream, cudaError_t *err);
 
 // Division of 0 <= n < 2^31 by a divisor fixed for the launch, as a multiply
 // and a shift: with l = ceil(log2 d) and m = ceil(2^(31+l) / d) (< 2^32),

@@ -58,5 +58,7 @@ ST_API st_status st_check_device_status(st_stream_t stream) {
   if (err != cudaSuccess) return ST_ERR_CUDA;
   word |= st::read_and_clear_relayout_error(s, &err);
   if (err != cudaSuccess) return ST_ERR_CUDA;
+  word |= st::read_and_clear_vmajor_error(s, &err);
+  if (err != cudaSuccess) return ST_ERR_CUDA;
   return word ? ST_ERR_TIMEOUT : ST_OK;
 }

@@ -368,24 +368,245 @@ __global__ void __launch_bounds__(THREADS, 2) l1_relayout(const char *__restrict
   }
 }
 
-// The S->T move of the rows whose destination mask byte is set (without the
-// RMSNorm; with it the bulk-copy RMS kernel of ulysses_relayout does the
-// move): a warp copies one row with 16-byte vectors.
-__global__ void __launch_bounds__(256) rows_masked(const char *__restrict__ in, char *__restrict__ out,
-                                                   const unsigned char *__restrict__ mask, long long n, int row_vecs,
-                                                   RowMap rm) {
+// The S->T move of the rows listed in idx[0, *count) without the RMSNorm: a
+// warp copies one listed row with 16-byte vectors.
+__global__ void __launch_bounds__(256) rows_idx(const char *__restrict__ in, char *__restrict__ out,
+                                                const int *__restrict__ idx, const int *__restrict__ count,
+                                                long long n, int row_vecs, RowMap rm) {
   const int lane = threadIdx.x & 31;
   st::pdl_trigger();
   st::pdl_wait();
   in = st::after_wait(in);
-  mask = st::after_wait(mask);
+  idx = st::after_wait(idx);
+  count = st::after_wait(count);
+  const long long n_act = min(max((long long)*count, 0LL), n);   // a listed row outside [0, n) is skipped
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n; r += nw) {
-    if (!mask[r]) continue;                              // warp-uniform
+  for (long long k = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; k < n_act; k += nw) {
+    const long long r = idx[k];
+    if (r < 0 || r >= n) continue;
     const uint4 *a = reinterpret_cast<const uint4 *>(in) + y_to_x(rm, r) * row_vecs;
     uint4 *d = reinterpret_cast<uint4 *>(out) + r * row_vecs;
     for (int v = lane; v < row_vecs; v += 32) d[v] = __ldg(a + v);
   }
+}
+
+__device__ unsigned int g_vmajor_error;      // bounded waits of the gather kernel that ran out
+constexpr unsigned long long VM_WAIT_NS = 2000000000ull;   // 2 s per wait
+constexpr int GATHER_WARPS = 4;
+
+__device__ __forceinline__ uint32_t sh_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// The S->T move of the rows listed in idx[0, *count) (K of the active tokens
+// into the K cache), with the per-head RMSNorm of ulysses_relayout computed in
+// the same order (same bytes).  A warp task is the RPT listed rows whose heads
+// fill a 32-head buffer; the bulk copy engine brings each row in (one copy per
+// row) while the previous task is normalised, one lane normalises one head in
+// shared memory, and one bulk copy per row writes it back.
+template <typename T, int D>
+__global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char *__restrict__ in, char *__restrict__ out,
+                                                                     const int *__restrict__ idx,
+                                                                     const int *__restrict__ count, long long n,
+                                                                     int row_vecs, const float *__restrict__ gamma,
+                                                                     float eps, RowMap rm) {
+  constexpr int EPV = 16 / int(sizeof(T));
+  constexpr int VPH = D / EPV;                 // vectors per head
+  constexpr int HB = D * int(sizeof(T));       // bytes per head
+  constexpr int BUF = 32 * HB;
+  constexpr int ROT = VPH % 4 == 0 ? 1 : 0;    // the full relayout's per-lane rotation of the vector order
+  extern __shared__ __align__(128) uint8_t rg_smem[];
+  __shared__ __align__(8) uint64_t full[GATHER_WARPS][2];
+  __shared__ float g_s[D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  st::pdl_trigger();
+  st::pdl_wait();
+  in = st::after_wait(in);
+  idx = st::after_wait(idx);
+  count = st::after_wait(count);
+  gamma = st::after_wait(gamma);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
+  if (lane == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][1])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const int row_bytes = row_vecs * 16;
+  const int hpr = row_bytes / HB;              // heads per row (<= 32)
+  const int rpt = 32 / hpr;                    // rows per task
+  const long long n_act = min(max((long long)*count, 0LL), n);   // a listed row outside [0, n) is skipped
+  const long long n_tasks = (n_act + rpt - 1) / rpt;
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  uint8_t *buf0 = rg_smem + warp * 2 * BUF;
+  // lane 0: load the rows of task t into buffer b; returns the rows in range as bits
+  auto issue = [&](long long t, int b) -> uint32_t {
+    const int nr = int(min((long long)rpt, n_act - t * rpt));
+    uint32_t vm = 0;
+    for (int j = 0; j < nr; ++j) {
+      const int r = idx[t * rpt + j];
+      if (r >= 0 && r < n) vm |= 1u << j;
+    }
+    uint64_t *bar = &full[warp][b];
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sh_u32(bar)),
+                 "r"(uint32_t(__popc(vm)) * uint32_t(row_bytes))
+                 : "memory");
+    for (int j = 0; j < nr; ++j) {
+      if (!((vm >> j) & 1u)) continue;
+      const long long src = y_to_x(rm, idx[t * rpt + j]);
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                   ::"r"(sh_u32(buf0 + b * BUF + j * row_bytes)), "l"(in + src * row_bytes), "r"(row_bytes),
+                   "r"(sh_u32(bar))
+                   : "memory");
+    }
+    return vm;
+  };
+  bool ok = true;
+  uint32_t vm_cur = 0, vm_next = 0;             // bit j: row j of the task is in range and moves
+  if (lane == 0 && gw < n_tasks) vm_cur = issue(gw, 0);
+  vm_cur = __shfl_sync(0xffffffffu, vm_cur, 0);
+  int i = 0;
+  for (long long t = gw; t < n_tasks && ok; t += nw, ++i) {
+    const int b = i & 1;
+    const long long next = t + nw;
+    if (next < n_tasks) {
+      if (lane == 0) {
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // the other buffer's stores have read it
+        vm_next = issue(next, b ^ 1);
+      }
+      vm_next = __shfl_sync(0xffffffffu, vm_next, 0);
+    }
+    if (lane == 0) {
+      const unsigned long long t0 = gtimer();
+      uint32_t done = 0;
+      while (!done) {
+        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}\n"
+                     : "=r"(done) : "r"(sh_u32(&full[warp][b])), "r"(uint32_t((i >> 1) & 1)) : "memory");
+        if (!done && gtimer() - t0 > VM_WAIT_NS) {
+          atomicOr(&g_vmajor_error, 1u);
+          ok = false;
+          break;
+        }
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (!ok) break;
+    uint8_t *bufp = buf0 + b * BUF;
+    if (lane < rpt * hpr && ((vm_cur >> (lane / hpr)) & 1u)) {
+      const int j = lane / hpr, h = lane - j * hpr;
+      // the full relayout normalises head (s1 * hpr + h) of a segment on lane (s1 * hpr + h) % 32
+      const long long src = y_to_x(rm, idx[t * rpt + j]);
+      const int fl = int(((src % rm.Sp) * hpr + h) % 32);
+      const int r0 = (fl * ROT) % VPH;
+      uint8_t *hp = bufp + j * row_bytes + h * HB;
+      float ss = 0.f;
+#pragma unroll
+      for (int u0 = 0; u0 < VPH; ++u0) {
+        const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
+        const uint4 v = *reinterpret_cast<const uint4 *>(hp + u * 16);
+        if constexpr (sizeof(T) == 2) {
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float a = __uint_as_float(w[k] << 16), c = __uint_as_float(w[k] & 0xffff0000u);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(c, c, ss);
+          }
+        } else {
+          ss = fmaf(__uint_as_float(v.x), __uint_as_float(v.x), ss);
+          ss = fmaf(__uint_as_float(v.y), __uint_as_float(v.y), ss);
+          ss = fmaf(__uint_as_float(v.z), __uint_as_float(v.z), ss);
+          ss = fmaf(__uint_as_float(v.w), __uint_as_float(v.w), ss);
+        }
+      }
+      const float inv = rsqrtf(ss * (1.0f / float(D)) + eps);
+#pragma unroll
+      for (int u0 = 0; u0 < VPH; ++u0) {
+        const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
+        uint4 v = *reinterpret_cast<const uint4 *>(hp + u * 16);
+        const float *gg = g_s + u * EPV;
+        if constexpr (sizeof(T) == 2) {
+          uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            w[k] = st::pack_bf16x2(__uint_as_float(w[k] << 16) * inv * gg[2 * k],
+                                   __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1]);
+          v = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+          v = make_uint4(__float_as_uint(__uint_as_float(v.x) * inv * gg[0]),
+                         __float_as_uint(__uint_as_float(v.y) * inv * gg[1]),
+                         __float_as_uint(__uint_as_float(v.z) * inv * gg[2]),
+                         __float_as_uint(__uint_as_float(v.w) * inv * gg[3]));
+        }
+        *reinterpret_cast<uint4 *>(hp + u * 16) = v;
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) {
+      for (int j = 0; j < rpt; ++j)
+        if ((vm_cur >> j) & 1u)
+          asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                     ::"l"(out + (long long)idx[t * rpt + j] * row_bytes), "r"(sh_u32(bufp + j * row_bytes)),
+                     "r"(row_bytes)
+                     : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    vm_cur = vm_next;
+  }
+  if (lane == 0) {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (!ok) {
+      // the next task's rows may still be landing in the other buffer: wait for them (bounded)
+      const unsigned long long t0 = gtimer();
+      uint32_t done = 0;
+      while (!done && gtimer() - t0 < VM_WAIT_NS)
+        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}\n"
+                     : "=r"(done) : "r"(sh_u32(&full[warp][(i + 1) & 1])), "r"(uint32_t(((i + 1) >> 1) & 1))
+                     : "memory");
+    }
+  }
+  __syncwarp();
+}
+
+template <typename T>
+st_status launch_gather_rms(int D, const char *in, char *out, const int *idx, const int *count, long long n,
+                            int row_vecs, const float *gamma, float eps, RowMap rm, cudaStream_t s) {
+#define ST_GATHER(DD)                                                                                       \
+  {                                                                                                         \
+    auto kern = rows_gather_rms<T, DD>;                                                                     \
+    const int smem = GATHER_WARPS * 2 * 32 * DD * int(sizeof(T));                                           \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)       \
+      return ST_ERR_CUDA;                                                                                   \
+    int per_sm = 0;                                                                                         \
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, GATHER_WARPS * 32, smem) != cudaSuccess || \
+        per_sm < 1)                                                                                         \
+      per_sm = 1;                                                                                           \
+    const int hpr = row_vecs * 16 / (DD * int(sizeof(T)));                                                  \
+    const long long tasks = (n + 32 / hpr - 1) / (32 / hpr); /* at most: every row listed */                \
+    const long long want = (tasks + GATHER_WARPS - 1) / GATHER_WARPS;                                       \
+    const long long cap = (long long)st::num_sms() * per_sm;                                                \
+    const int grid = int(want < cap ? want : cap);                                                          \
+    return st::launch_pdl(kern, grid, GATHER_WARPS * 32, smem, s, in, out, idx, count, n, row_vecs, gamma, eps, rm); \
+  }
+  switch (D) {
+    case 32: ST_GATHER(32)
+    case 64: ST_GATHER(64)
+    case 72: ST_GATHER(72)
+    case 80: ST_GATHER(80)
+    case 96: ST_GATHER(96)
+    case 128: ST_GATHER(128)
+  }
+#undef ST_GATHER
+  return ST_ERR_UNSUPPORTED;
 }
 
 // Host-side check and map of the S->T exchange shape (elem: element bytes).
@@ -612,10 +833,10 @@ ST_API st_status vmajor_relayout_mask(const void *v_cur_x, const void *v_prev_x,
                         static_cast<const int *>(tile_count), idx, count);
 }
 
-ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const unsigned char *mask, int P, int B, int T,
-                                      int S, int C, int n_t, int n_s, st_dtype dtype, const float *rms_gamma,
+ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const int *idx, const int *count, int P, int B,
+                                      int T, int S, int C, int n_t, int n_s, st_dtype dtype, const float *rms_gamma,
                                       int rms_head_dim, float rms_eps, st_stream_t stream) {
-  if (!in_x || !out_y || !mask) return ST_ERR_NULL;
+  if (!in_x || !out_y || !idx || !count) return ST_ERR_NULL;
   if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_DTYPE;
   const int esize = dtype == ST_F32 ? 4 : 2;
   RowMap rm;
@@ -626,18 +847,32 @@ ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const unsig
   const int row_vecs = C * esize / 16;
   if (rms_gamma) {
     if (rms_head_dim <= 0 || C % rms_head_dim || (rms_head_dim * esize) % 16) return ST_ERR_SHAPE;
+    if (C / rms_head_dim > 32) return ST_ERR_UNSUPPORTED;     // a row's heads fill at most one task buffer
   }
   const long long bytes = n * C * esize;
   const char *i0 = static_cast<const char *>(in_x);
   char *o0 = static_cast<char *>(out_y);
   if (o0 < i0 + bytes && i0 < o0 + bytes) return ST_ERR_SHAPE;  // overlap
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // with the RMSNorm: the bulk-copy kernel of ulysses_relayout, restricted to the masked rows
   if (rms_gamma)
-    return st::relayout_s2t_rms_masked(in_x, out_y, mask, esize, P, B, T, S, C, n_t, n_s, rms_gamma, rms_head_dim,
-                                       rms_eps, s);
+    return dtype == ST_BF16 ? launch_gather_rms<uint16_t>(rms_head_dim, i0, o0, idx, count, n, row_vecs, rms_gamma,
+                                                          rms_eps, rm, s)
+                            : launch_gather_rms<float>(rms_head_dim, i0, o0, idx, count, n, row_vecs, rms_gamma,
+                                                       rms_eps, rm, s);
   const long long want = (n + 7) / 8;
   const long long cap = (long long)st::num_sms() * 16;
   const int grid = int(want < cap ? want : cap);
-  return st::launch_pdl(rows_masked, grid, 256, 0, s, i0, o0, mask, n, row_vecs, rm);
+  return st::launch_pdl(rows_idx, grid, 256, 0, s, i0, o0, idx, count, n, row_vecs, rm);
 }
+
+namespace st {
+unsigned int read_and_clear_vmajor_error(cudaStream_t stream, cudaError_t *err) {
+  unsigned int word = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&word, g_vmajor_error, sizeof(word), 0, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyToSymbolAsync(g_vmajor_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (err) *err = e;
+  return word;
+}
+}  // namespace st

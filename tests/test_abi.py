@@ -171,9 +171,9 @@ def test_sender_vmajor_rejects(st):
     assert mask_call(cache=VP(0x100000 + 64)) == st.ST_ERR_SHAPE        # overlaps the input
     r = st._c["vmajor_relayout_rows"]
 
-    def rows_call(gamma=None, hd=0, C=64, out=FAKE_OUT, mask=VP(0x400000)):
-        return r(FAKE_IN, out, mask, 2, 1, 8, 16, C, 1, 1, st.ST_BF16, gamma, hd, 1e-6, None)
-    assert rows_call(mask=None) == st.ST_ERR_NULL
+    def rows_call(gamma=None, hd=0, C=64, out=FAKE_OUT, idx=VP(0x400000)):
+        return r(FAKE_IN, out, idx, VP(0x500000), 2, 1, 8, 16, C, 1, 1, st.ST_BF16, gamma, hd, 1e-6, None)
+    assert rows_call(idx=None) == st.ST_ERR_NULL
     assert rows_call(gamma=FAKE_IN, hd=48) == st.ST_ERR_SHAPE
     assert rows_call(gamma=FAKE_IN, hd=4) == st.ST_ERR_SHAPE            # 8-byte heads: not 16-byte rows
     assert rows_call(out=VP(0x100000 + 32)) == st.ST_ERR_SHAPE

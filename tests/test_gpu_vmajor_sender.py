@@ -106,7 +106,7 @@ def test_vmajor_relayout_mask_force_all_and_unchanged(st):
 @pytest.mark.parametrize("name,rms", [("opensora_low", True), ("opensora_low", False), ("tiny", True),
                                       ("tiny", False)])
 def test_vmajor_relayout_rows(st, name, rms):
-    """Active rows equal the full relayout's (with RMSNorm: the same bytes), the others stay."""
+    """Listed rows equal the full relayout's (with RMSNorm: the same bytes), the others stay."""
     w = synth.BY_NAME[name]
     n, C = w.B * w.T * w.S, w.C
     x = synth.randn(w, "k", (n, C)).to(DEV)
@@ -118,7 +118,11 @@ def test_vmajor_relayout_rows(st, name, rms):
     mask_np = (rng.random(n) < 0.5).astype(np.uint8)
     old = synth.randn(w, "kprev", (n, C))
     out = old.to(DEV)
-    st.vmajor_relayout_rows(x, out, torch.from_numpy(mask_np).to(DEV), w.P, w.B, w.T, w.S, C, w.n_t, w.n_s, **kw)
+    idx_np = np.flatnonzero(mask_np).astype(np.int32)
+    idx = torch.full((n,), -1, dtype=torch.int32)
+    idx[:idx_np.size] = torch.from_numpy(idx_np)
+    count = torch.tensor([idx_np.size], dtype=torch.int32)
+    st.vmajor_relayout_rows(x, out, idx.to(DEV), count.to(DEV), w.P, w.B, w.T, w.S, C, w.n_t, w.n_s, **kw)
     torch.cuda.synchronize()
     on = torch.from_numpy(np.flatnonzero(mask_np))
     off = torch.from_numpy(np.flatnonzero(mask_np == 0))
