@@ -61,9 +61,6 @@ __device__ __forceinline__ T *after_wait(T *p) {
 
 // SM count of the current device (cached per device ordinal).
 int num_sms();
-st_status relayout_s2t_rms_masked(const void *in, void *out, const unsigned char *mask, int elem_bytes, int P, int B,
-                                  int T, int S, int C, int n_t, int n_s, const float *gamma, int D, float eps,
-                                  cudaStream_t s);
 
 // Reads and clears the device error word of the tensor-core attention kernel
 // (defined next to that kernel).  Returns the word's previous value.

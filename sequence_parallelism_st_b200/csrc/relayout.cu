@@ -198,8 +198,7 @@ constexpr unsigned long long RMS_WAIT_NS = 2000000000ull;
 template <typename T, int D>
 __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char *__restrict__ in,
                                                                char *__restrict__ out,
-                                                               const float *__restrict__ gamma, float eps,
-                                                               const unsigned char *__restrict__ row_mask) {
+                                                               const float *__restrict__ gamma, float eps) {
   constexpr int EPV = 16 / int(sizeof(T));               // elements per 16-byte vector
   constexpr int VPH = D / EPV;                           // vectors per head
   constexpr int HB = D * int(sizeof(T));                 // bytes per head
@@ -213,7 +212,6 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
   st::pdl_wait();
   in = st::after_wait(in);
   gamma = st::after_wait(gamma);
-  if (row_mask) row_mask = st::after_wait(row_mask);
   for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
   if (lane == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");
@@ -229,36 +227,8 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
 
-  // With a row mask (destination rows; S->T and T->S only) a task moves only
-  // the heads of the rows whose mask byte is set: runs of whole rows' heads.
-  const long long hpr = m.row_bytes / HB;                        // heads per row
-  // bit k of the result: head k of the task belongs to a masked-in row
-  auto active_heads = [&](long long dst, int nh) -> uint32_t {
-    if (!row_mask) return nh >= 32 ? 0xffffffffu : ((1u << nh) - 1u);
-    const long long h0 = dst / HB;
-    uint32_t act = 0;
-    for (long long r = h0 / hpr; r * hpr < h0 + nh; ++r) {
-      if (!row_mask[r]) continue;
-      const int lo = int(max(0LL, r * hpr - h0)), hi = int(min((long long)nh, (r + 1) * hpr - h0));
-      act |= (hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~((1u << lo) - 1u);
-    }
-    return act;
-  };
-  // With a row mask, lane k works out up front which heads of the warp's
-  // k-th task move (the mask reads of all its tasks in one round trip).
-  uint32_t pre_act = 0;
-  const bool pre = row_mask && one_src && (n_tasks - gw + nw - 1) / nw <= 32;
-  if (pre) {
-    const long long t = gw + lane * nw;
-    if (t < n_tasks) {
-      const long long seg = t / tps, c = t - seg * tps;
-      long long so, dof;
-      map_segment(m, seg, so, dof);
-      pre_act = active_heads(dof + c * 32 * HB, int(min(32LL, hps - c * 32)));
-    }
-  }
-  // task -> (destination byte offset, number of heads, heads to move); issues its load into buffer b
-  auto issue = [&](long long task, int b, long long &dst, int &nh, uint32_t &act) {
+  // task -> (destination byte offset, number of heads); issues its load into buffer b
+  auto issue = [&](long long task, int b, long long &dst, int &nh) {
     uint8_t *bufp = buf0 + b * BUF;
     if (one_src) {
       const long long seg = task / tps;
@@ -267,26 +237,16 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
       long long so, dof;
       map_segment(m, seg, so, dof);
       dst = dof + c * 32 * HB;
-      act = pre ? __shfl_sync(0xffffffffu, pre_act, int((task - gw) / nw)) : 0u;
       if (lane == 0) {
-        if (!pre) act = active_heads(dst, nh);
-        expect_tx(&full[warp][b], __popc(act) * HB);   // 0 bytes: the phase completes at once
-        for (uint32_t rest = act; rest;) {              // one copy per run of heads
-          const int lo = __ffs(rest) - 1;
-          const uint32_t from_lo = rest >> lo;
-          const int len = from_lo == 0xffffffffu ? 32 - lo : __ffs(~from_lo) - 1;
-          bulk_g2s(bufp + lo * HB, in + so + (c * 32 + lo) * HB, len * HB, &full[warp][b]);
-          rest &= len + lo >= 32 ? 0u : ~((1u << (lo + len)) - 1u);
-        }
+        expect_tx(&full[warp][b], nh * HB);
+        bulk_g2s(bufp, in + so + c * 32 * HB, nh * HB, &full[warp][b]);
       }
-      act = __shfl_sync(0xffffffffu, act, 0);
     } else {
       const long long g0 = task * 32;
       nh = int(min(32LL, m.n_segs - g0));
       long long so, dof;
       map_segment(m, g0 + (lane < nh ? lane : 0), so, dof);
       dst = __shfl_sync(0xffffffffu, dof, 0);                     // destination rows are consecutive
-      act = nh >= 32 ? 0xffffffffu : ((1u << nh) - 1u);
       if (lane == 0) expect_tx(&full[warp][b], nh * HB);
       __syncwarp();
       if (lane < nh) bulk_g2s(bufp + lane * HB, in + so, HB, &full[warp][b]);
@@ -296,8 +256,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
   bool ok = true;
   long long dst_cur = 0, dst_next = 0;
   int nh_cur = 0, nh_next = 0;
-  uint32_t act_cur = 0, act_next = 0;
-  if (gw < n_tasks) issue(gw, 0, dst_cur, nh_cur, act_cur);
+  if (gw < n_tasks) issue(gw, 0, dst_cur, nh_cur);
   int i = 0;
   for (long long task = gw; task < n_tasks && ok; task += nw, ++i) {
     const int b = i & 1;
@@ -306,7 +265,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
       // the store of the previous task used the other buffer: it must have read it
       if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       __syncwarp();
-      issue(next, b ^ 1, dst_next, nh_next, act_next);
+      issue(next, b ^ 1, dst_next, nh_next);
     }
     {
       const unsigned long long t0 = gtimer();
@@ -320,7 +279,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
     }
     if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
     uint8_t *bufp = buf0 + b * BUF;
-    if (lane < nh_cur && ((act_cur >> lane) & 1u)) {
+    if (lane < nh_cur) {
       uint8_t *h = bufp + lane * HB;
       const int r0 = (lane * ROT) % VPH;
       float ss = 0.f;
@@ -367,18 +326,9 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    if (lane == 0) {
-      for (uint32_t rest = act_cur; rest;) {            // one store per run of moved heads
-        const int lo = __ffs(rest) - 1;
-        const uint32_t from_lo = rest >> lo;
-        const int len = from_lo == 0xffffffffu ? 32 - lo : __ffs(~from_lo) - 1;
-        bulk_s2g(out + dst_cur + (long long)lo * HB, bufp + lo * HB, len * HB);
-        rest &= len + lo >= 32 ? 0u : ~((1u << (lo + len)) - 1u);
-      }
-    }
+    if (lane == 0) bulk_s2g(out + dst_cur, bufp, nh_cur * HB);
     dst_cur = dst_next;
     nh_cur = nh_next;
-    act_cur = act_next;
   }
   if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   if (!ok && lane == 0) {
@@ -393,7 +343,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
 
 template <typename T, int D>
 st_status launch_rms_d(const Map &m, const char *in, char *out, const float *gamma, float eps, int sms,
-                       cudaStream_t s, const unsigned char *row_mask) {
+                       cudaStream_t s) {
   constexpr int BUF = 32 * D * int(sizeof(T));
   constexpr int SMEM = RMS_WARPS * 2 * BUF;
   auto kern = relayout_rms<T, D>;
@@ -409,19 +359,19 @@ st_status launch_rms_d(const Map &m, const char *in, char *out, const float *gam
   const long long want = (n_tasks + RMS_WARPS - 1) / RMS_WARPS;
   const long long cap = (long long)sms * per_sm;
   const int grid = int(want < cap ? want : cap);
-  return st::launch_pdl(kern, grid, RMS_WARPS * 32, SMEM, s, m, in, out, gamma, eps, row_mask);
+  return st::launch_pdl(kern, grid, RMS_WARPS * 32, SMEM, s, m, in, out, gamma, eps);
 }
 
 template <typename T>
 st_status launch_rms(const Map &m, const char *in, char *out, const float *gamma, int D, float eps, int sms,
-                     cudaStream_t s, const unsigned char *row_mask = nullptr) {
+                     cudaStream_t s) {
   switch (D) {
-    case 32: return launch_rms_d<T, 32>(m, in, out, gamma, eps, sms, s, row_mask);
-    case 64: return launch_rms_d<T, 64>(m, in, out, gamma, eps, sms, s, row_mask);
-    case 72: return launch_rms_d<T, 72>(m, in, out, gamma, eps, sms, s, row_mask);
-    case 80: return launch_rms_d<T, 80>(m, in, out, gamma, eps, sms, s, row_mask);
-    case 96: return launch_rms_d<T, 96>(m, in, out, gamma, eps, sms, s, row_mask);
-    case 128: return launch_rms_d<T, 128>(m, in, out, gamma, eps, sms, s, row_mask);
+    case 32: return launch_rms_d<T, 32>(m, in, out, gamma, eps, sms, s);
+    case 64: return launch_rms_d<T, 64>(m, in, out, gamma, eps, sms, s);
+    case 72: return launch_rms_d<T, 72>(m, in, out, gamma, eps, sms, s);
+    case 80: return launch_rms_d<T, 80>(m, in, out, gamma, eps, sms, s);
+    case 96: return launch_rms_d<T, 96>(m, in, out, gamma, eps, sms, s);
+    case 128: return launch_rms_d<T, 128>(m, in, out, gamma, eps, sms, s);
     default: return ST_ERR_UNSUPPORTED;
   }
 }
@@ -439,29 +389,6 @@ st_status launch_copy(const Map &m, const char *in, char *out, int grid, cudaStr
 }  // namespace
 
 namespace st {
-// The S->T move of the destination rows whose mask byte is set, with the
-// per-head RMSNorm, on the bulk-copy RMS kernel of ulysses_relayout (so the
-// bytes of a moved row equal the full relayout's).  Arguments are checked by
-// the caller.
-st_status relayout_s2t_rms_masked(const void *in, void *out, const unsigned char *mask, int elem_bytes, int P, int B,
-                                  int T, int S, int C, int n_t, int n_s, const float *gamma, int D, float eps,
-                                  cudaStream_t s) {
-  Map m = {};
-  m.mode = ST_S2T;
-  m.P = P;
-  m.B = B;
-  m.n_t = n_t; m.n_s = n_s; m.i0 = 0; m.n_i = n_t; m.j0 = 0; m.n_j = n_s;
-  m.q0 = 0; m.n_q = P;
-  m.Tn = T / n_t; m.Tq = T / (n_t * P); m.Sp = S / (n_s * P); m.Ss = S / n_s;
-  m.row_bytes = (long long)C * elem_bytes;
-  m.seg_bytes = m.Sp * m.row_bytes;
-  m.n_segs = (long long)P * B * n_t * n_s * m.Tq * P;
-  const char *src = static_cast<const char *>(in);
-  char *dst = static_cast<char *>(out);
-  return elem_bytes == 2 ? launch_rms<uint16_t>(m, src, dst, gamma, D, eps, num_sms(), s, mask)
-                         : launch_rms<float>(m, src, dst, gamma, D, eps, num_sms(), s, mask);
-}
-
 unsigned int read_and_clear_relayout_error(cudaStream_t stream, cudaError_t *err) {
   unsigned int word = 0, zero = 0;
   cudaError_t e = cudaMemcpyFromSymbolAsync(&word, g_relayout_error, sizeof(word), 0, cudaMemcpyDeviceToHost, stream);
