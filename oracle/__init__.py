@@ -24,6 +24,8 @@ Every function restates, in float64 numpy, what the pages define:
                  section).
 * rmsnorm     -- per-head RMSNorm on Q and K (CoCoDiff article, "V-First"
                  section).
+* rope        -- rotary position embedding of Q and K after the RMSNorm
+                 (CoCoDiff article, "V-First" section).
 * vmajor      -- per-token L1 change of V against the previous step, the
                  threshold mask, the ascending list of active tokens and the
                  cache update (CoCoDiff article, "V-Major" section).
@@ -34,13 +36,14 @@ from .attention import attention, spatial, temporal, merge_chunks, frames_view
 from .relayout import (st_x_rows, st_y_rows, st_relayout, seq_head_relayout,
                        st_logical_from_x, st_logical_from_y, st_row_pairs, seq_head_row_pairs)
 from .rmsnorm import rmsnorm_heads
+from .rope import rope_angles, rope_table, rope_heads
 from .vmajor import l1_change, change_mask, compact, scatter_rows, pack_rows, tau_for_fraction
 
 __all__ = [
     "attention", "spatial", "temporal", "merge_chunks", "frames_view",
     "st_x_rows", "st_y_rows", "st_relayout", "seq_head_relayout",
     "st_logical_from_x", "st_logical_from_y", "st_row_pairs", "seq_head_row_pairs",
-    "rmsnorm_heads",
+    "rmsnorm_heads", "rope_angles", "rope_table", "rope_heads",
     "l1_change", "change_mask", "compact", "scatter_rows", "pack_rows",
     "tau_for_fraction",
 ]

@@ -44,6 +44,7 @@ from __future__ import annotations
 import numpy as np
 
 from .rmsnorm import rmsnorm_heads
+from .rope import rope_heads
 
 
 def _f64(x):
@@ -78,24 +79,31 @@ def _check_st(P, T, S, n_t, n_s):
         raise ValueError("N_T*P must divide T and N_S*P must divide S")
 
 
-def _move_rows(src, dst, src_log, dst_log, sel, row_len, rms):
+def _move_rows(src, dst, src_log, dst_log, sel, row_len, rms, rope=None, position=None):
     pos = np.empty(src_log.size, dtype=np.int64)
     pos[src_log] = np.arange(src_log.size)              # logical -> source row
     rows = src.reshape(-1, row_len)[pos[dst_log[sel]]]
     if rms is not None:
         gamma, head_dim, eps = rms
         rows = rmsnorm_heads(rows, gamma, head_dim, eps)
+    if rope is not None:                                # after the RMSNorm
+        head_dim, theta = rope
+        rows = rope_heads(rows, position(dst_log[sel]), head_dim, theta)
     dst.reshape(-1, row_len)[sel] = rows
     return dst
 
 
-def st_relayout(mode, buf, P, B, T, S, C, n_t=1, n_s=1, blocks=None, out=None, rms=None):
+def st_relayout(mode, buf, P, B, T, S, C, n_t=1, n_s=1, blocks=None, out=None, rms=None, rope=None):
     """S2T (x -> y) or T2S (y -> x) on a flat buffer of B*T*S*C elements.
 
     blocks = (i0, i1, j0, j1) limits the destination rows written; rows
     outside the range keep the values of ``out`` (NaN when ``out`` is None).
-    rms = (gamma[D], D, eps) applies the per-head RMSNorm to moved rows.
+    rms = (gamma[D], D, eps) applies the per-head RMSNorm to moved rows;
+    rope = (D, theta) then rotates them by their token's index s in its frame
+    (S2T only: the spatial layer's positions).
     """
+    if rope is not None and mode != "S2T":
+        raise ValueError("RoPE applies on the way to the spatial layer (S2T)")
     _check_st(P, T, S, n_t, n_s)
     x_log, xi, xj = st_x_rows(P, B, T, S, n_t, n_s)
     y_log, yi, yj = st_y_rows(P, B, T, S, n_t, n_s)
@@ -109,7 +117,7 @@ def st_relayout(mode, buf, P, B, T, S, C, n_t=1, n_s=1, blocks=None, out=None, r
     sel = np.flatnonzero((di >= i0) & (di < i1) & (dj >= j0) & (dj < j1))
     src = _f64(buf).reshape(-1)
     dst = np.full(src.size, np.nan) if out is None else _f64(out).reshape(-1).copy()
-    return _move_rows(src, dst, src_log, dst_log, sel, C, rms)
+    return _move_rows(src, dst, src_log, dst_log, sel, C, rms, rope, lambda logical: logical % S)
 
 
 def st_row_pairs(mode, P, B, T, S, n_t=1, n_s=1, blocks=None):
@@ -170,8 +178,13 @@ def _head_rows(P, B, N, H):
     return ((b * N + n) * H + h).reshape(-1)
 
 
-def seq_head_relayout(mode, buf, P, B, N, H, D, rms=None):
-    """SEQ2HEAD ([P,B,N/P,H,D] -> [P,B,H/P,N,D]) or HEAD2SEQ (its inverse)."""
+def seq_head_relayout(mode, buf, P, B, N, H, D, rms=None, rope=None):
+    """SEQ2HEAD ([P,B,N/P,H,D] -> [P,B,H/P,N,D]) or HEAD2SEQ (its inverse).
+
+    rope = (D, theta) rotates moved heads by their token's sequence index n
+    after the RMSNorm (SEQ2HEAD only)."""
+    if rope is not None and mode != "SEQ2HEAD":
+        raise ValueError("RoPE applies on the way to the attention (SEQ2HEAD)")
     if N % P or H % P:
         raise ValueError("P must divide N and H")
     seq_log, head_log = _seq_rows(P, B, N, H), _head_rows(P, B, N, H)
@@ -183,4 +196,5 @@ def seq_head_relayout(mode, buf, P, B, N, H, D, rms=None):
         raise ValueError(mode)
     src = _f64(buf).reshape(-1)
     dst = np.full(src.size, np.nan)
-    return _move_rows(src, dst, src_log, dst_log, np.arange(dst_log.size), D, rms)
+    return _move_rows(src, dst, src_log, dst_log, np.arange(dst_log.size), D, rms, rope,
+                      lambda logical: (logical // H) % N)
