@@ -174,6 +174,9 @@ class Step:
         # sender-side V-Major: the mask is taken on x and only active K/V rows move
         # (into the caches); receiver side: full relayouts, mask on y, scatter
         self.sender_vmajor = True
+        # rotary position embedding of Q and K after their RMSNorm (positions: the
+        # token index in the frame); off unless asked for
+        self.rope_table = None
         # fused merge: chunk c >= 1 is merged into the accumulated fp32 partial
         # inside the attention kernel; the last chunk writes the bf16 result
         self.fused_merge = True
@@ -225,19 +228,18 @@ class Step:
             st.vmajor_relayout_mask(d["v"], self.vprev_x, self.vc, P, B, T, S, C, w.n_t, w.n_s, self.tau, self.mask,
                                     self.idx, self.count, self.ws)
             st.vmajor_relayout_rows(d["k"], self.kc, self.idx, self.count, P, B, T, S, C, w.n_t, w.n_s,
-                                    rms_gamma=self.gamma, rms_head_dim=D, rms_eps=w.rms_eps)
+                                    rms_gamma=self.gamma, rms_head_dim=D, rms_eps=w.rms_eps,
+                                    rope_table=self.rope_table)
             self._mark("vmajor", False)
             self._mark("relayout_s2t", True)
-            st.ulysses_relayout("S2T", d["q"], self.qy, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
-                                rms_head_dim=D, rms_eps=w.rms_eps)
+            self._qk_relayout(d["q"], self.qy)
             self._mark("relayout_s2t", False)
         else:
+            # V first: its exchange needs no normalisation ([CC] "V-First")
             self._mark("relayout_s2t", True)
-            st.ulysses_relayout("S2T", d["q"], self.qy, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
-                                rms_head_dim=D, rms_eps=w.rms_eps)
-            st.ulysses_relayout("S2T", d["k"], self.ky, P, B, T, S, C, w.n_t, w.n_s, rms_gamma=self.gamma,
-                                rms_head_dim=D, rms_eps=w.rms_eps)
             st.ulysses_relayout("S2T", d["v"], self.vy, P, B, T, S, C, w.n_t, w.n_s)
+            self._qk_relayout(d["k"], self.ky)
+            self._qk_relayout(d["q"], self.qy)
             self._mark("relayout_s2t", False)
             self._mark("vmajor", True)
             st.vmajor_mask_compact(self.vy.view(self.n, C), self.vprev_y.view(self.n, C), self.tau, self.mask,
@@ -261,6 +263,16 @@ class Step:
         self._mark("temporal", True)
         st.st_attn_temporal(d["q"], d["k"], d["v"], self.ot, None, desc=self.tdesc)
         self._mark("temporal", False)
+
+    def _qk_relayout(self, src, dst):
+        """S->T of Q or K with the per-head RMSNorm (and the rotary embedding when on)."""
+        st, w = self.st, self.w
+        if self.rope_table is not None:
+            st.ulysses_relayout_rope("S2T", src, dst, w.P, w.B, w.T, w.S, w.C, w.n_t, w.n_s, rms_gamma=self.gamma,
+                                     rms_head_dim=w.D, rms_eps=w.rms_eps, rope_table=self.rope_table)
+        else:
+            st.ulysses_relayout("S2T", src, dst, w.P, w.B, w.T, w.S, w.C, w.n_t, w.n_s, rms_gamma=self.gamma,
+                                rms_head_dim=w.D, rms_eps=w.rms_eps)
 
     def _spatial_fused(self, i):
         """KV chunks of the spatial attention with the merge fused into the
@@ -423,6 +435,8 @@ def run_ours(args, w, rank, world, dev):
     stp = Step(st, w, dev)
     stp.fused_merge = args.merge == "fused"
     stp.sender_vmajor = args.vmajor == "sender"
+    if args.rope:
+        stp.rope_table = st.st_rope_table(w.S, w.D, 10000.0, device=dev)
     if args.schedule == "overlap":
         stp.setup_overlap(args.slices, args.att_sms)
         step_fn = stp.run_overlap
@@ -566,7 +580,8 @@ def run_ours(args, w, rank, world, dev):
                    f"overlap: {args.slices} shard ranges, attention on {args.att_sms} SMs",
                    "chunk_merge": "fused into the attention kernel" if stp.fused_merge else "attn_chunk_merge",
                    "vmajor": "sender side (mask on x, active K/V rows into the caches)" if stp.sender_vmajor else
-                   "receiver side (full relayouts, mask on y, scatter)"},
+                   "receiver side (full relayouts, mask on y, scatter)",
+                   "qk_rope": bool(args.rope)},
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(statistics.mean(e2e_ms), 5)},
         "roofline": {"bound": "tensor", "kernel": "st_attn_spatial", "achieved": round(achieved, 2),
@@ -652,6 +667,8 @@ def main():
     ap.add_argument("--vmajor", choices=["sender", "receiver"], default="sender",
                     help="sender: mask on x, only active K/V rows move into the caches; receiver: full relayouts, "
                          "mask on y, scatter")
+    ap.add_argument("--rope", action="store_true",
+                    help="rotary position embedding of Q and K after their RMSNorm (token index in the frame)")
     ap.add_argument("--schedule", choices=["serial", "overlap"], default="serial",
                     help="overlap: shard ranges of the step on two streams (attention / memory-bound steps)")
     ap.add_argument("--slices", type=int, default=4, help="shard ranges of the overlap schedule")

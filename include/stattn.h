@@ -214,6 +214,32 @@ st_status ulysses_relayout_range(st_relayout_mode mode, const void *in, void *ou
                                  int j1, int q0, int q1, const float *rms_gamma,
                                  int rms_head_dim, float rms_eps, st_stream_t stream);
 
+/* Rotary position embedding [CC "V-First": Q and K receive RMSNorm and
+ * RoPE, V neither].  Reading (the pages give no formula): the D channels of a
+ * head form D/2 interleaved pairs (x[2i], x[2i+1]); pair i of the token at
+ * position m turns by a = m * theta^(-2i/D):
+ *     (x0, x1) -> (x0 cos a - x1 sin a, x0 sin a + x1 cos a),
+ * applied after the RMSNorm.  A token's position is its index in the
+ * sequence the attention runs over: s inside its frame (S2T, the spatial
+ * layer) or n (SEQ2HEAD, image attention).
+ *
+ * st_rope_table fills table (fp32 device, [n_pos][head_dim / 2][2], 8-byte
+ * aligned) with (cos a, sin a) for every position m < n_pos and pair i,
+ * computed in double precision.  head_dim even, theta > 0. */
+st_status st_rope_table(int n_pos, int head_dim, float theta, float *table,
+                        st_stream_t stream);
+
+/* ulysses_relayout (S2T or SEQ2HEAD, every block and shard) with the fused
+ * per-head RMSNorm (rms_gamma required) followed by the rotary embedding of
+ * every moved head from rope_table (st_rope_table), which must hold at least
+ * S (S2T) or N (SEQ2HEAD) positions: rope_positions.  ST_ERR_UNSUPPORTED for
+ * the inverse modes, ST_ERR_SHAPE for an odd head dim or a short table. */
+st_status ulysses_relayout_rope(st_relayout_mode mode, const void *in, void *out,
+                                int elem_bytes, int P, int B, int T_or_N, int S_or_H,
+                                int C_or_D, int n_t, int n_s, const float *rms_gamma,
+                                int rms_head_dim, float rms_eps, const float *rope_table,
+                                int rope_positions, st_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * V-Major selective communication [CC "V-Major"].
  * ---------------------------------------------------------------------- */
@@ -298,12 +324,16 @@ st_status vmajor_relayout_mask(const void *v_cur_x, const void *v_prev_x, void *
  * cache [CC "V-Major"].  rms_gamma (optional, fp32 device [rms_head_dim])
  * applies the per-head RMSNorm of ulysses_relayout on the way, with the same
  * arithmetic, so a written row holds the same bytes as in the full relayout;
- * with it a row may hold at most 32 heads (else ST_ERR_UNSUPPORTED).  Rows
+ * with it a row may hold at most 32 heads (else ST_ERR_UNSUPPORTED).
+ * rope_table (optional, needs rms_gamma; see st_rope_table) then turns each
+ * moved head by the rotary angles of its token's index s in the frame, as
+ * ulysses_relayout_rope does; it must hold rope_positions >= S rows.  Rows
  * not listed are neither read nor written.  in_x and out_y must not overlap. */
 st_status vmajor_relayout_rows(const void *in_x, void *out_y, const int *idx, const int *count,
                                int P, int B, int T, int S, int C, int n_t, int n_s,
                                st_dtype dtype, const float *rms_gamma, int rms_head_dim,
-                               float rms_eps, st_stream_t stream);
+                               float rms_eps, const float *rope_table, int rope_positions,
+                               st_stream_t stream);
 
 /* vmajor_mask_compact and vmajor_scatter_rows (without `packed`) in one call
  * [CC "V-Major" section]: the pass that decides a token is active also copies

@@ -9,6 +9,7 @@ Entry points (same names as the C ABI in include/stattn.h):
     st_attn_spatial, st_attn_spatial_merge, st_attn_temporal, attn_chunk_merge, ulysses_relayout,
     ulysses_relayout_range, vmajor_mask_compact, vmajor_mask_compact_noalloc, vmajor_mask_compact_scatter,
     vmajor_scatter_rows, vmajor_workspace_bytes, vmajor_relayout_mask, vmajor_relayout_rows,
+    st_rope_table, ulysses_relayout_rope,
     st_check_device_status, st_status_string, st_set_sm_budget, st_get_sm_budget
 """
 from __future__ import annotations
@@ -84,7 +85,10 @@ _c = {
     "vmajor_relayout_mask": _proto("vmajor_relayout_mask", c_int, _VP, _VP, _VP, c_int, c_int, c_int, c_int, c_int,
                                    c_int, c_int, c_int, c_float, c_int, _VP, _VP, _VP, _VP, _VP, c_size_t, _VP),
     "vmajor_relayout_rows": _proto("vmajor_relayout_rows", c_int, _VP, _VP, _VP, _VP, c_int, c_int, c_int, c_int,
-                                   c_int, c_int, c_int, c_int, _VP, c_int, c_float, _VP),
+                                   c_int, c_int, c_int, c_int, _VP, c_int, c_float, _VP, c_int, _VP),
+    "st_rope_table": _proto("st_rope_table", c_int, c_int, c_int, c_float, _VP, _VP),
+    "ulysses_relayout_rope": _proto("ulysses_relayout_rope", c_int, c_int, _VP, _VP, c_int, c_int, c_int, c_int,
+                                    c_int, c_int, c_int, c_int, _VP, c_int, c_float, _VP, c_int, _VP),
     "st_get_sm_budget": _proto("st_get_sm_budget", c_int),
 }
 
@@ -93,7 +97,8 @@ EXPORTED = ["st_status_string", "st_abi_version", "st_attn_spatial", "st_attn_sp
             "ulysses_relayout", "vmajor_workspace_bytes", "vmajor_mask_compact", "vmajor_mask_compact_noalloc",
             "vmajor_scatter_rows", "vmajor_mask_compact_scatter",
             "st_check_device_status", "st_selftest_wait_timeout", "ulysses_relayout_range", "st_set_sm_budget",
-            "st_get_sm_budget", "vmajor_relayout_mask", "vmajor_relayout_rows"]
+            "st_get_sm_budget", "vmajor_relayout_mask", "vmajor_relayout_rows", "st_rope_table",
+            "ulysses_relayout_rope"]
 
 
 class StattnError(RuntimeError):
@@ -274,12 +279,33 @@ def vmajor_relayout_mask(v_cur_x, v_prev_x, v_cache_y, P, B, T, S, C, n_t, n_s, 
 
 
 def vmajor_relayout_rows(in_x, out_y, idx, count, P, B, T, S, C, n_t, n_s, rms_gamma=None, rms_head_dim=0,
-                         rms_eps=1e-6, *, stream=None, raw=False):
-    """S->T move of the destination rows idx[:count] (device), with the optional per-head RMSNorm."""
+                         rms_eps=1e-6, rope_table=None, *, stream=None, raw=False):
+    """S->T move of the destination rows idx[:count] (device), with the optional per-head RMSNorm
+    and rotary embedding (rope_table from st_rope_table)."""
+    n_pos = rope_table.shape[0] if rope_table is not None else 0
     r = _c["vmajor_relayout_rows"](_ptr(in_x), _ptr(out_y), _ptr(idx), _ptr(count), P, B, T, S, C, n_t, n_s,
                                    _dtype_code(in_x), _ptr(rms_gamma), int(rms_head_dim), float(rms_eps),
-                                   _stream(stream))
+                                   _ptr(rope_table), n_pos, _stream(stream))
     return r if raw else _check(r, "vmajor_relayout_rows")
+
+
+def st_rope_table(n_pos, head_dim, theta=10000.0, *, device="cuda", stream=None):
+    """Rotary (cos, sin) table, fp32 [n_pos, head_dim // 2, 2], computed on the device."""
+    import torch
+    t = torch.empty((n_pos, head_dim // 2, 2), dtype=torch.float32, device=device)
+    _check(_c["st_rope_table"](int(n_pos), int(head_dim), float(theta), _ptr(t), _stream(stream)), "st_rope_table")
+    return t
+
+
+def ulysses_relayout_rope(mode, inp, out, P, B, T_or_N, S_or_H, C_or_D, n_t=1, n_s=1, rms_gamma=None,
+                          rms_head_dim=0, rms_eps=1e-6, rope_table=None, *, stream=None, raw=False):
+    """ulysses_relayout (S2T / SEQ2HEAD) with the per-head RMSNorm and the rotary embedding."""
+    m = MODES[mode] if isinstance(mode, str) else int(mode)
+    n_pos = rope_table.shape[0] if rope_table is not None else 0
+    r = _c["ulysses_relayout_rope"](m, _ptr(inp), _ptr(out), inp.element_size(), P, B, T_or_N, S_or_H, C_or_D, n_t,
+                                    n_s, _ptr(rms_gamma), int(rms_head_dim), float(rms_eps), _ptr(rope_table), n_pos,
+                                    _stream(stream))
+    return r if raw else _check(r, "ulysses_relayout_rope")
 
 
 def st_check_device_status(stream=None) -> int:

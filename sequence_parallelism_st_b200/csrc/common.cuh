@@ -100,4 +100,43 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// One 16-byte vector of a head on its way through the per-head RMSNorm and,
+// with a rotation table, the rotary position embedding: every element x
+// becomes y = x * inv * g, then pair k of the vector (elements 2k, 2k+1, pair
+// index u * EPV / 2 + k of the head) turns by the angle whose (cos, sin) is
+// rot[k]:  (y0, y1) -> (y0 c - y1 s, y0 s + y1 c).  T: uint16_t (bf16) or
+// float.  rot == nullptr: the RMSNorm alone.
+template <typename T>
+__device__ __forceinline__ uint4 rms_rope_vec(uint4 v, float inv, const float *gg, const float2 *rot) {
+  if constexpr (sizeof(T) == 2) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float a = __uint_as_float(w[k] << 16) * inv * gg[2 * k];
+      float b = __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1];
+      if (rot) {
+        const float2 cs = rot[k];
+        const float a2 = a * cs.x - b * cs.y;
+        b = a * cs.y + b * cs.x;
+        a = a2;
+      }
+      w[k] = pack_bf16x2(a, b);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    float y[4] = {__uint_as_float(v.x) * inv * gg[0], __uint_as_float(v.y) * inv * gg[1],
+                  __uint_as_float(v.z) * inv * gg[2], __uint_as_float(v.w) * inv * gg[3]};
+    if (rot) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float2 cs = rot[k];
+        const float a = y[2 * k], b = y[2 * k + 1];
+        y[2 * k] = a * cs.x - b * cs.y;
+        y[2 * k + 1] = a * cs.y + b * cs.x;
+      }
+    }
+    return make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]), __float_as_uint(y[3]));
+  }
+}
+
 }  // namespace st

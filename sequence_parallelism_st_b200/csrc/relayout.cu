@@ -198,7 +198,8 @@ constexpr unsigned long long RMS_WAIT_NS = 2000000000ull;
 template <typename T, int D>
 __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char *__restrict__ in,
                                                                char *__restrict__ out,
-                                                               const float *__restrict__ gamma, float eps) {
+                                                               const float *__restrict__ gamma, float eps,
+                                                               const float2 *__restrict__ rope) {
   constexpr int EPV = 16 / int(sizeof(T));               // elements per 16-byte vector
   constexpr int VPH = D / EPV;                           // vectors per head
   constexpr int HB = D * int(sizeof(T));                 // bytes per head
@@ -212,6 +213,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
   st::pdl_wait();
   in = st::after_wait(in);
   gamma = st::after_wait(gamma);
+  if (rope) rope = st::after_wait(rope);
   for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
   if (lane == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");
@@ -303,25 +305,25 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
         }
       }
       const float inv = rsqrtf(ss * (1.0f / float(D)) + eps);
+      // the rotary angles of this head's token: its index s in the frame (S2T)
+      // or in the sequence (SEQ2HEAD), a row of the (cos, sin) table
+      const float2 *rot = nullptr;
+      if (rope) {
+        long long pos;
+        if (m.mode == ST_S2T) {
+          const long long r = (dst_cur + (long long)lane * HB) / m.row_bytes;   // destination (y) row
+          pos = ((r / ((long long)m.Tq * m.Ss)) % m.n_s) * m.Ss + r % m.Ss;
+        } else {
+          pos = (dst_cur / HB + lane) % m.N;                                  // destination (q, b, h1, n) row
+        }
+        rot = rope + pos * (D / 2);
+      }
 #pragma unroll
       for (int u0 = 0; u0 < VPH; ++u0) {
         const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
-        uint4 v = *reinterpret_cast<const uint4 *>(h + u * 16);
-        const float *gg = g_s + u * EPV;
-        if constexpr (sizeof(T) == 2) {
-          uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            w[k] = st::pack_bf16x2(__uint_as_float(w[k] << 16) * inv * gg[2 * k],
-                                   __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1]);
-          v = make_uint4(w[0], w[1], w[2], w[3]);
-        } else {
-          v = make_uint4(__float_as_uint(__uint_as_float(v.x) * inv * gg[0]),
-                         __float_as_uint(__uint_as_float(v.y) * inv * gg[1]),
-                         __float_as_uint(__uint_as_float(v.z) * inv * gg[2]),
-                         __float_as_uint(__uint_as_float(v.w) * inv * gg[3]));
-        }
-        *reinterpret_cast<uint4 *>(h + u * 16) = v;
+        const uint4 v = *reinterpret_cast<const uint4 *>(h + u * 16);
+        *reinterpret_cast<uint4 *>(h + u * 16) =
+            st::rms_rope_vec<T>(v, inv, g_s + u * EPV, rot ? rot + u * (EPV / 2) : nullptr);
       }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
 
 template <typename T, int D>
 st_status launch_rms_d(const Map &m, const char *in, char *out, const float *gamma, float eps, int sms,
-                       cudaStream_t s) {
+                       cudaStream_t s, const float2 *rope) {
   constexpr int BUF = 32 * D * int(sizeof(T));
   constexpr int SMEM = RMS_WARPS * 2 * BUF;
   auto kern = relayout_rms<T, D>;
@@ -359,19 +361,19 @@ st_status launch_rms_d(const Map &m, const char *in, char *out, const float *gam
   const long long want = (n_tasks + RMS_WARPS - 1) / RMS_WARPS;
   const long long cap = (long long)sms * per_sm;
   const int grid = int(want < cap ? want : cap);
-  return st::launch_pdl(kern, grid, RMS_WARPS * 32, SMEM, s, m, in, out, gamma, eps);
+  return st::launch_pdl(kern, grid, RMS_WARPS * 32, SMEM, s, m, in, out, gamma, eps, rope);
 }
 
 template <typename T>
 st_status launch_rms(const Map &m, const char *in, char *out, const float *gamma, int D, float eps, int sms,
-                     cudaStream_t s) {
+                     cudaStream_t s, const float2 *rope = nullptr) {
   switch (D) {
-    case 32: return launch_rms_d<T, 32>(m, in, out, gamma, eps, sms, s);
-    case 64: return launch_rms_d<T, 64>(m, in, out, gamma, eps, sms, s);
-    case 72: return launch_rms_d<T, 72>(m, in, out, gamma, eps, sms, s);
-    case 80: return launch_rms_d<T, 80>(m, in, out, gamma, eps, sms, s);
-    case 96: return launch_rms_d<T, 96>(m, in, out, gamma, eps, sms, s);
-    case 128: return launch_rms_d<T, 128>(m, in, out, gamma, eps, sms, s);
+    case 32: return launch_rms_d<T, 32>(m, in, out, gamma, eps, sms, s, rope);
+    case 64: return launch_rms_d<T, 64>(m, in, out, gamma, eps, sms, s, rope);
+    case 72: return launch_rms_d<T, 72>(m, in, out, gamma, eps, sms, s, rope);
+    case 80: return launch_rms_d<T, 80>(m, in, out, gamma, eps, sms, s, rope);
+    case 96: return launch_rms_d<T, 96>(m, in, out, gamma, eps, sms, s, rope);
+    case 128: return launch_rms_d<T, 128>(m, in, out, gamma, eps, sms, s, rope);
     default: return ST_ERR_UNSUPPORTED;
   }
 }
@@ -400,11 +402,11 @@ unsigned int read_and_clear_relayout_error(cudaStream_t stream, cudaError_t *err
 }
 }  // namespace st
 
-ST_API st_status ulysses_relayout_range(st_relayout_mode mode, const void *in, void *out, int elem_bytes,
-                                        int P, int B, int T_or_N, int S_or_H, int C_or_D, int n_t, int n_s,
-                                        int i0, int i1, int j0, int j1, int q0, int q1,
-                                        const float *rms_gamma, int rms_head_dim, float rms_eps,
-                                        st_stream_t stream) {
+namespace {
+st_status relayout_impl(st_relayout_mode mode, const void *in, void *out, int elem_bytes, int P, int B, int T_or_N,
+                        int S_or_H, int C_or_D, int n_t, int n_s, int i0, int i1, int j0, int j1, int q0, int q1,
+                        const float *rms_gamma, int rms_head_dim, float rms_eps, const float *rope_table,
+                        int rope_positions, st_stream_t stream) {
   if (!in || !out) return ST_ERR_NULL;
   if (!(elem_bytes == 1 || elem_bytes == 2 || elem_bytes == 4 || elem_bytes == 8)) return ST_ERR_DTYPE;
   if (P <= 0 || B <= 0 || T_or_N <= 0 || S_or_H <= 0 || C_or_D <= 0 || n_t <= 0 || n_s <= 0)
@@ -451,9 +453,18 @@ ST_API st_status ulysses_relayout_range(st_relayout_mode mode, const void *in, v
     if ((rms_head_dim * elem_bytes) % 16 || !st::is_aligned(in, 16) || !st::is_aligned(out, 16) ||
         m.row_bytes % 16)
       return ST_ERR_ALIGN;
-    return elem_bytes == 2 ? launch_rms<uint16_t>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s)
-                           : launch_rms<float>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s);
+    const float2 *rope = nullptr;
+    if (rope_table) {
+      // rotary angles of the attended sequence: tokens of a frame (S2T) or of the sequence (SEQ2HEAD)
+      if (mode != ST_S2T && mode != ST_SEQ2HEAD) return ST_ERR_UNSUPPORTED;
+      if (rms_head_dim % 2 || rope_positions < (mode == ST_S2T ? S_or_H : T_or_N)) return ST_ERR_SHAPE;
+      if (!st::is_aligned(rope_table, 8)) return ST_ERR_ALIGN;
+      rope = reinterpret_cast<const float2 *>(rope_table);
+    }
+    return elem_bytes == 2 ? launch_rms<uint16_t>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s, rope)
+                           : launch_rms<float>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s, rope);
   }
+  if (rope_table) return ST_ERR_NULL;               // the rotation rides on the RMSNorm pass
   // widest vector that divides the row pitch and both base addresses
   int vec = 16;
   while (vec > elem_bytes && (m.row_bytes % vec || !st::is_aligned(in, vec) || !st::is_aligned(out, vec)))
@@ -469,10 +480,51 @@ ST_API st_status ulysses_relayout_range(st_relayout_mode mode, const void *in, v
   }
 }
 
+// rotation table: (cos, sin) of pos * theta^(-2i/D), computed in double precision
+__global__ void rope_table_kernel(long long n, int half, double theta, float2 *out) {
+  const long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= n) return;
+  const long long pos = k / half;
+  const int i = int(k - pos * half);
+  const double a = double(pos) * pow(theta, -2.0 * double(i) / double(2 * half));
+  out[k] = make_float2(float(cos(a)), float(sin(a)));
+}
+}  // namespace
+
+ST_API st_status ulysses_relayout_range(st_relayout_mode mode, const void *in, void *out, int elem_bytes,
+                                        int P, int B, int T_or_N, int S_or_H, int C_or_D, int n_t, int n_s,
+                                        int i0, int i1, int j0, int j1, int q0, int q1,
+                                        const float *rms_gamma, int rms_head_dim, float rms_eps,
+                                        st_stream_t stream) {
+  return relayout_impl(mode, in, out, elem_bytes, P, B, T_or_N, S_or_H, C_or_D, n_t, n_s, i0, i1, j0, j1, q0, q1,
+                       rms_gamma, rms_head_dim, rms_eps, nullptr, 0, stream);
+}
+
 ST_API st_status ulysses_relayout(st_relayout_mode mode, const void *in, void *out, int elem_bytes,
                                   int P, int B, int T_or_N, int S_or_H, int C_or_D, int n_t,
                                   int n_s, int i0, int i1, int j0, int j1, const float *rms_gamma,
                                   int rms_head_dim, float rms_eps, st_stream_t stream) {
-  return ulysses_relayout_range(mode, in, out, elem_bytes, P, B, T_or_N, S_or_H, C_or_D, n_t, n_s, i0, i1, j0,
-                                j1, 0, P, rms_gamma, rms_head_dim, rms_eps, stream);
+  return relayout_impl(mode, in, out, elem_bytes, P, B, T_or_N, S_or_H, C_or_D, n_t, n_s, i0, i1, j0, j1, 0, P,
+                       rms_gamma, rms_head_dim, rms_eps, nullptr, 0, stream);
+}
+
+ST_API st_status ulysses_relayout_rope(st_relayout_mode mode, const void *in, void *out, int elem_bytes, int P, int B,
+                                       int T_or_N, int S_or_H, int C_or_D, int n_t, int n_s, const float *rms_gamma,
+                                       int rms_head_dim, float rms_eps, const float *rope_table, int rope_positions,
+                                       st_stream_t stream) {
+  if (!rms_gamma || !rope_table) return ST_ERR_NULL;
+  const int i1 = (mode == ST_S2T || mode == ST_T2S) ? n_t : 1, j1 = (mode == ST_S2T || mode == ST_T2S) ? n_s : 1;
+  return relayout_impl(mode, in, out, elem_bytes, P, B, T_or_N, S_or_H, C_or_D, n_t, n_s, 0, i1, 0, j1, 0, P,
+                       rms_gamma, rms_head_dim, rms_eps, rope_table, rope_positions, stream);
+}
+
+ST_API st_status st_rope_table(int n_pos, int head_dim, float theta, float *table, st_stream_t stream) {
+  if (!table) return ST_ERR_NULL;
+  if (n_pos <= 0 || head_dim <= 0 || head_dim % 2 || !(theta > 0.f)) return ST_ERR_SHAPE;
+  if (!st::is_aligned(table, 8)) return ST_ERR_ALIGN;
+  const long long n = (long long)n_pos * (head_dim / 2);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  rope_table_kernel<<<int((n + 255) / 256), 256, 0, s>>>(n, head_dim / 2, double(theta),
+                                                         reinterpret_cast<float2 *>(table));
+  return st::launch_status();
 }

@@ -414,7 +414,8 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
                                                                      const int *__restrict__ idx,
                                                                      const int *__restrict__ count, long long n,
                                                                      int row_vecs, const float *__restrict__ gamma,
-                                                                     float eps, RowMap rm) {
+                                                                     float eps, RowMap rm,
+                                                                     const float2 *__restrict__ rope) {
   constexpr int EPV = 16 / int(sizeof(T));
   constexpr int VPH = D / EPV;                 // vectors per head
   constexpr int HB = D * int(sizeof(T));       // bytes per head
@@ -430,6 +431,7 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
   idx = st::after_wait(idx);
   count = st::after_wait(count);
   gamma = st::after_wait(gamma);
+  if (rope) rope = st::after_wait(rope);
   for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
   if (lane == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");
@@ -527,25 +529,18 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
         }
       }
       const float inv = rsqrtf(ss * (1.0f / float(D)) + eps);
+      // rotary angles of the row's token: its index s in the frame
+      const float2 *rot = nullptr;
+      if (rope) {
+        const long long r = idx[t * rpt + j];
+        rot = rope + (((r / ((long long)rm.Tq * rm.Ss)) % rm.n_s) * rm.Ss + r % rm.Ss) * (D / 2);
+      }
 #pragma unroll
       for (int u0 = 0; u0 < VPH; ++u0) {
         const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
-        uint4 v = *reinterpret_cast<const uint4 *>(hp + u * 16);
-        const float *gg = g_s + u * EPV;
-        if constexpr (sizeof(T) == 2) {
-          uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            w[k] = st::pack_bf16x2(__uint_as_float(w[k] << 16) * inv * gg[2 * k],
-                                   __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1]);
-          v = make_uint4(w[0], w[1], w[2], w[3]);
-        } else {
-          v = make_uint4(__float_as_uint(__uint_as_float(v.x) * inv * gg[0]),
-                         __float_as_uint(__uint_as_float(v.y) * inv * gg[1]),
-                         __float_as_uint(__uint_as_float(v.z) * inv * gg[2]),
-                         __float_as_uint(__uint_as_float(v.w) * inv * gg[3]));
-        }
-        *reinterpret_cast<uint4 *>(hp + u * 16) = v;
+        const uint4 v = *reinterpret_cast<const uint4 *>(hp + u * 16);
+        *reinterpret_cast<uint4 *>(hp + u * 16) =
+            st::rms_rope_vec<T>(v, inv, g_s + u * EPV, rot ? rot + u * (EPV / 2) : nullptr);
       }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -579,7 +574,8 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
 
 template <typename T>
 st_status launch_gather_rms(int D, const char *in, char *out, const int *idx, const int *count, long long n,
-                            int row_vecs, const float *gamma, float eps, RowMap rm, cudaStream_t s) {
+                            int row_vecs, const float *gamma, float eps, RowMap rm, cudaStream_t s,
+                            const float2 *rope) {
 #define ST_GATHER(DD)                                                                                       \
   {                                                                                                         \
     auto kern = rows_gather_rms<T, DD>;                                                                     \
@@ -595,7 +591,8 @@ st_status launch_gather_rms(int D, const char *in, char *out, const int *idx, co
     const long long want = (tasks + GATHER_WARPS - 1) / GATHER_WARPS;                                       \
     const long long cap = (long long)st::num_sms() * per_sm;                                                \
     const int grid = int(want < cap ? want : cap);                                                          \
-    return st::launch_pdl(kern, grid, GATHER_WARPS * 32, smem, s, in, out, idx, count, n, row_vecs, gamma, eps, rm); \
+    return st::launch_pdl(kern, grid, GATHER_WARPS * 32, smem, s, in, out, idx, count, n, row_vecs, gamma, eps, rm, \
+                          rope);                                                                            \
   }
   switch (D) {
     case 32: ST_GATHER(32)
@@ -835,7 +832,8 @@ ST_API st_status vmajor_relayout_mask(const void *v_cur_x, const void *v_prev_x,
 
 ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const int *idx, const int *count, int P, int B,
                                       int T, int S, int C, int n_t, int n_s, st_dtype dtype, const float *rms_gamma,
-                                      int rms_head_dim, float rms_eps, st_stream_t stream) {
+                                      int rms_head_dim, float rms_eps, const float *rope_table, int rope_positions,
+                                      st_stream_t stream) {
   if (!in_x || !out_y || !idx || !count) return ST_ERR_NULL;
   if (dtype != ST_F32 && dtype != ST_BF16) return ST_ERR_DTYPE;
   const int esize = dtype == ST_F32 ? 4 : 2;
@@ -849,6 +847,11 @@ ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const int *
     if (rms_head_dim <= 0 || C % rms_head_dim || (rms_head_dim * esize) % 16) return ST_ERR_SHAPE;
     if (C / rms_head_dim > 32) return ST_ERR_UNSUPPORTED;     // a row's heads fill at most one task buffer
   }
+  if (rope_table) {                                           // rides on the RMSNorm pass
+    if (!rms_gamma) return ST_ERR_NULL;
+    if (rms_head_dim % 2 || rope_positions < S) return ST_ERR_SHAPE;
+    if (!st::is_aligned(rope_table, 8)) return ST_ERR_ALIGN;
+  }
   const long long bytes = n * C * esize;
   const char *i0 = static_cast<const char *>(in_x);
   char *o0 = static_cast<char *>(out_y);
@@ -856,9 +859,9 @@ ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const int *
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (rms_gamma)
     return dtype == ST_BF16 ? launch_gather_rms<uint16_t>(rms_head_dim, i0, o0, idx, count, n, row_vecs, rms_gamma,
-                                                          rms_eps, rm, s)
+                                                          rms_eps, rm, s, reinterpret_cast<const float2 *>(rope_table))
                             : launch_gather_rms<float>(rms_head_dim, i0, o0, idx, count, n, row_vecs, rms_gamma,
-                                                       rms_eps, rm, s);
+                                                       rms_eps, rm, s, reinterpret_cast<const float2 *>(rope_table));
   const long long want = (n + 7) / 8;
   const long long cap = (long long)st::num_sms() * 16;
   const int grid = int(want < cap ? want : cap);

@@ -171,9 +171,28 @@ def test_sender_vmajor_rejects(st):
     assert mask_call(cache=VP(0x100000 + 64)) == st.ST_ERR_SHAPE        # overlaps the input
     r = st._c["vmajor_relayout_rows"]
 
-    def rows_call(gamma=None, hd=0, C=64, out=FAKE_OUT, idx=VP(0x400000)):
-        return r(FAKE_IN, out, idx, VP(0x500000), 2, 1, 8, 16, C, 1, 1, st.ST_BF16, gamma, hd, 1e-6, None)
+    def rows_call(gamma=None, hd=0, C=64, out=FAKE_OUT, idx=VP(0x400000), rope=None, n_pos=0):
+        return r(FAKE_IN, out, idx, VP(0x500000), 2, 1, 8, 16, C, 1, 1, st.ST_BF16, gamma, hd, 1e-6, rope, n_pos, None)
     assert rows_call(idx=None) == st.ST_ERR_NULL
     assert rows_call(gamma=FAKE_IN, hd=48) == st.ST_ERR_SHAPE
     assert rows_call(gamma=FAKE_IN, hd=4) == st.ST_ERR_SHAPE            # 8-byte heads: not 16-byte rows
     assert rows_call(out=VP(0x100000 + 32)) == st.ST_ERR_SHAPE
+    assert rows_call(rope=VP(0x700000), n_pos=16) == st.ST_ERR_NULL             # RoPE rides on the RMSNorm
+    assert rows_call(gamma=FAKE_IN, hd=32, rope=VP(0x700000), n_pos=15) == st.ST_ERR_SHAPE   # table too short
+
+
+def test_rope_rejects(st):
+    VP = ctypes.c_void_p
+    t = st._c["st_rope_table"]
+    assert t(16, 64, 10000.0, None, None) == st.ST_ERR_NULL
+    assert t(16, 63, 10000.0, VP(0x700000), None) == st.ST_ERR_SHAPE
+    assert t(0, 64, 10000.0, VP(0x700000), None) == st.ST_ERR_SHAPE
+    assert t(16, 64, 0.0, VP(0x700000), None) == st.ST_ERR_SHAPE
+    rr = st._c["ulysses_relayout_rope"]
+
+    def call(mode=st.ST_S2T, gamma=FAKE_IN, rope=VP(0x700000), n_pos=16, hd=32):
+        return rr(mode, FAKE_IN, FAKE_OUT, 2, 2, 1, 8, 16, 64, 1, 1, gamma, hd, 1e-6, rope, n_pos, None)
+    assert call(gamma=None) == st.ST_ERR_NULL
+    assert call(rope=None) == st.ST_ERR_NULL
+    assert call(mode=st.ST_T2S) == st.ST_ERR_UNSUPPORTED
+    assert call(n_pos=15) == st.ST_ERR_SHAPE

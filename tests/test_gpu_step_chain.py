@@ -143,3 +143,25 @@ def test_sender_vmajor_step_matches_receiver(st):
     for i, (a, b) in enumerate(zip(res[True], res[False])):
         assert torch.equal(a, b), f"output {i} differs between sender and receiver V-Major"
     assert st.st_check_device_status() == st.ST_OK
+
+
+def test_rope_step_sender_matches_receiver(st):
+    """With the rotary embedding on Q and K, the sender-side and receiver-side
+    V-Major steps still give the same bits for every output."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    w = synth.BY_NAME["opensora_low"]
+    stp = bench.Step(st, w, "cuda")
+    stp.rope_table = st.st_rope_table(w.S, w.D, 10000.0)
+    res = {}
+    for sender in (False, True):
+        stp.sender_vmajor = sender
+        stp.reset_caches()
+        stp.idx.fill_(-1)
+        stp.run()
+        torch.cuda.synchronize()
+        res[sender] = outputs(stp) + [stp.qy.clone()]
+    for i, (a, b) in enumerate(zip(res[True], res[False])):
+        assert torch.equal(a, b), f"output {i} differs between sender and receiver V-Major with RoPE"
+    assert st.st_check_device_status() == st.ST_OK
