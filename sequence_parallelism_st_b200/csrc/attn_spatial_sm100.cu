@@ -33,13 +33,12 @@
 //     softmax, round once to bf16 (or keep fp32 partials), stage 32 x 16
 //     blocks in shared memory and write them with bulk tensor stores, plus the
 //     natural-log LSE.  The softmax warps go straight on to the next item.
-//   * Merge mode (st_attn_spatial_merge): for head dims up to 80 the epilogue
-//     seeds O in TMEM with the accumulated fp32 partial of the tile's next
-//     item right after reading this item's O, PV accumulates onto it, and the
-//     softmax starts from the partial's LSE (as running max) with row sum 1,
-//     so the online softmax simply continues; the first item of each tile is
-//     seeded before anything else.  Larger head dims merge in the epilogue,
-//     loading 32 x 16 accumulator blocks with TMA into the staging buffers.
+//   * Merge mode (st_attn_spatial_merge): the epilogue merges the chunk's
+//     normalised O with the accumulated fp32 partial of earlier chunks,
+//     o = w_a o_a + w_c O / l with w = exp(lse - M) / sum, and writes the
+//     merged LSE.  For head dims up to 80 the copy engine stages the
+//     accumulated rows of one tile in shared memory while the item runs;
+//     larger head dims load them from global memory one chunk ahead.
 //   * Head dims 32..128: Q and K split D into a 64-wide 128B-swizzled chunk and
 //     a remainder chunk padded to 16/32/64 (zero-filled by TMA beyond D); V is
 //     stored as column atoms so that PV is one instruction of N = padded D.
@@ -121,12 +120,14 @@ template <int D, bool MERGE = false> struct Cfg {
   static constexpr int VSW = VW * 2;                   // atom row bytes = swizzle span
   static constexpr int VAT = BLOCK_N * VSW;            // bytes of one atom region
   static constexpr int VTILE = VA * VAT;               // bytes of one V tile
-  static constexpr int EPI = 4 * 2 * EPI_BUF + 2 * 2 * BLOCK_M * 4;
+  // two staging buffers per epilogue warp (only without the slots: the
+  // space goes to the K/V ring), then the row statistics (m, l) of both tiles
+  static constexpr int EPI_STG = SLOTS ? 0 : 4 * 2 * EPI_BUF;
+  static constexpr int EPI = EPI_STG + 2 * 2 * BLOCK_M * 4;
   static constexpr int BUDGET = SLOTS ? 232448 - 4096 - EPI - ACCS : 204800;   // bytes for Q and the K/V ring
   static constexpr int QB = (4 * QTILE + 4 * (KTILE + VTILE) <= BUDGET) ? 2 : 1;   // Q double buffer if 4 stages fit
   static constexpr int NS_RAW = (BUDGET - 2 * QB * QTILE) / (KTILE + VTILE);
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;   // K/V ring depth
-  // epilogue: two staging buffers per epilogue warp, then the row statistics (m, l) of both tiles (EPI above)
   static constexpr int SMEM = 1024 + 2 * QB * QTILE + NS * (KTILE + VTILE) + ACCS + EPI + 1024;   // + barriers
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(DP <= 128 && DPV <= 128, "head dim too large");
@@ -403,8 +404,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *sK = sQ + QB * 2 * K::QTILE;        // NS K tiles
   uint8_t *sV = sK + NS * K::KTILE;            // NS V tiles
   uint8_t *sAcc = sV + NS * K::VTILE;          // merge mode: [epilogue warp][chunk] 32 x 16 fp32 blocks
-  uint8_t *sEpi = sAcc + K::ACCS;              // 4 warps x 2 staging buffers
-  float *sStat = reinterpret_cast<float *>(sEpi + 4 * 2 * EPI_BUF);   // [tile][m | l][row]
+  uint8_t *sEpi = sAcc + K::ACCS;              // 4 warps x 2 staging buffers (without the slots)
+  float *sStat = reinterpret_cast<float *>(sEpi + K::EPI_STG);   // [tile][m | l][row]
   uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + K::EPI);
   uint64_t *q_full = bars;                     // QB
   uint64_t *q_empty = q_full + QB;             // QB, 2 arrivals (the two S issuers)
