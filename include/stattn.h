@@ -223,7 +223,7 @@ st_status ulysses_relayout_range(st_relayout_mode mode, const void *in, void *ou
  * sequence the attention runs over: s inside its frame (S2T, the spatial
  * layer) or n (SEQ2HEAD, image attention).
  *
- * st_rope_table fills table (fp32 device, [n_pos][head_dim / 2][2], 8-byte
+ * st_rope_table fills table (fp32 device, [n_pos][head_dim / 2][2], 16-byte
  * aligned) with (cos a, sin a) for every position m < n_pos and pair i,
  * computed in double precision.  head_dim even, theta > 0. */
 st_status st_rope_table(int n_pos, int head_dim, float theta, float *table,
@@ -233,7 +233,8 @@ st_status st_rope_table(int n_pos, int head_dim, float theta, float *table,
  * per-head RMSNorm (rms_gamma required) followed by the rotary embedding of
  * every moved head from rope_table (st_rope_table), which must hold at least
  * S (S2T) or N (SEQ2HEAD) positions: rope_positions.  ST_ERR_UNSUPPORTED for
- * the inverse modes, ST_ERR_SHAPE for an odd head dim or a short table. */
+ * the inverse modes, ST_ERR_SHAPE for an odd head dim or a short table,
+ * ST_ERR_ALIGN unless rope_table is 16-byte aligned. */
 st_status ulysses_relayout_rope(st_relayout_mode mode, const void *in, void *out,
                                 int elem_bytes, int P, int B, int T_or_N, int S_or_H,
                                 int C_or_D, int n_t, int n_s, const float *rms_gamma,
@@ -327,7 +328,8 @@ st_status vmajor_relayout_mask(const void *v_cur_x, const void *v_prev_x, void *
  * with it a row may hold at most 32 heads (else ST_ERR_UNSUPPORTED).
  * rope_table (optional, needs rms_gamma; see st_rope_table) then turns each
  * moved head by the rotary angles of its token's index s in the frame, as
- * ulysses_relayout_rope does; it must hold rope_positions >= S rows.  Rows
+ * ulysses_relayout_rope does; it must hold rope_positions >= S rows and be
+ * 16-byte aligned (else ST_ERR_SHAPE / ST_ERR_ALIGN).  Rows
  * not listed are neither read nor written.  in_x and out_y must not overlap. */
 st_status vmajor_relayout_rows(const void *in_x, void *out_y, const int *idx, const int *count,
                                int P, int B, int T, int S, int C, int n_t, int n_s,

@@ -104,18 +104,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // with a rotation table, the rotary position embedding: every element x
 // becomes y = x * inv * g, then pair k of the vector (elements 2k, 2k+1, pair
 // index u * EPV / 2 + k of the head) turns by the angle whose (cos, sin) is
-// rot[k]:  (y0, y1) -> (y0 c - y1 s, y0 s + y1 c).  T: uint16_t (bf16) or
-// float.  rot == nullptr: the RMSNorm alone.
-template <typename T>
+// rot[k]:  (y0, y1) -> (y0 c - y1 s, y0 s + y1 c); rot is 16-byte aligned.
+// T: uint16_t (bf16) or float.  ROPE = false: the RMSNorm alone, rot unused
+// (the rotation is a compile-time choice, so a kernel without it holds no
+// table load at all).
+template <typename T, bool ROPE>
 __device__ __forceinline__ uint4 rms_rope_vec(uint4 v, float inv, const float *gg, const float2 *rot) {
   if constexpr (sizeof(T) == 2) {
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float4 cs4[2] = {};                        // (cos, sin) of the 4 pairs: two 16-byte reads
+    if constexpr (ROPE) {
+      cs4[0] = reinterpret_cast<const float4 *>(rot)[0];
+      cs4[1] = reinterpret_cast<const float4 *>(rot)[1];
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       float a = __uint_as_float(w[k] << 16) * inv * gg[2 * k];
       float b = __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1];
-      if (rot) {
-        const float2 cs = rot[k];
+      if constexpr (ROPE) {
+        const float2 cs = (k & 1) ? make_float2(cs4[k >> 1].z, cs4[k >> 1].w)
+                                  : make_float2(cs4[k >> 1].x, cs4[k >> 1].y);
         const float a2 = a * cs.x - b * cs.y;
         b = a * cs.y + b * cs.x;
         a = a2;
@@ -126,10 +134,11 @@ __device__ __forceinline__ uint4 rms_rope_vec(uint4 v, float inv, const float *g
   } else {
     float y[4] = {__uint_as_float(v.x) * inv * gg[0], __uint_as_float(v.y) * inv * gg[1],
                   __uint_as_float(v.z) * inv * gg[2], __uint_as_float(v.w) * inv * gg[3]};
-    if (rot) {
+    if constexpr (ROPE) {
+      const float4 c4 = reinterpret_cast<const float4 *>(rot)[0];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        const float2 cs = rot[k];
+        const float2 cs = k ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
         const float a = y[2 * k], b = y[2 * k + 1];
         y[2 * k] = a * cs.x - b * cs.y;
         y[2 * k + 1] = a * cs.y + b * cs.x;

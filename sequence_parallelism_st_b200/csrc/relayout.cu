@@ -34,9 +34,11 @@ struct Map {
   long long n_segs;
 };
 
-// Byte offsets of segment g in the source and the destination.
+// Byte offsets of segment g in the source and the destination; with pos0,
+// the sequence position of the segment's first destination row (S2T: its
+// token index s in the frame; SEQ2HEAD: its n).
 __device__ __forceinline__ void map_segment(const Map &m, long long g, long long &src,
-                                            long long &dst) {
+                                            long long &dst, int *pos0 = nullptr) {
   long long src_row, dst_row;
   if (m.mode == ST_S2T) {
     // segments enumerate destination rows (q, b, i, j, t2, p); p fastest
@@ -50,6 +52,7 @@ __device__ __forceinline__ void map_segment(const Map &m, long long g, long long
     long long blk_x = (((long long)p * m.B + b) * m.n_t + i) * m.n_s + j;
     dst_row = (blk_y * m.Tq + t2) * m.Ss + (long long)p * m.Sp;
     src_row = (blk_x * m.Tn + (long long)q * m.Tq + t2) * m.Sp;
+    if (pos0) *pos0 = j * m.Ss + p * m.Sp;
   } else if (m.mode == ST_T2S) {
     // segments enumerate destination rows (p, b, i, j, t1) whose frame comes
     // from the selected y shards: t1 in [q0 * Tq, (q0 + n_q) * Tq)
@@ -68,6 +71,7 @@ __device__ __forceinline__ void map_segment(const Map &m, long long g, long long
     // destination rows (q, b, h1, n); n fastest
     dst_row = g;
     int n = int(g % m.N); g /= m.N;
+    if (pos0) *pos0 = n;
     int h1 = int(g % m.Hp); g /= m.Hp;
     int b = int(g % m.B);
     int q = int(g / m.B);
@@ -195,7 +199,7 @@ __device__ __forceinline__ unsigned long long gtimer() {
 constexpr int RMS_WARPS = 4;
 constexpr unsigned long long RMS_WAIT_NS = 2000000000ull;
 
-template <typename T, int D>
+template <typename T, int D, bool ROPE>
 __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char *__restrict__ in,
                                                                char *__restrict__ out,
                                                                const float *__restrict__ gamma, float eps,
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
   st::pdl_wait();
   in = st::after_wait(in);
   gamma = st::after_wait(gamma);
-  if (rope) rope = st::after_wait(rope);
+  if constexpr (ROPE) rope = st::after_wait(rope);
   for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
   if (lane == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");
@@ -225,20 +229,25 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
   const bool one_src = (m.mode == ST_S2T || m.mode == ST_T2S);   // heads of a task contiguous in the source
   const long long hps = m.seg_bytes / HB;                         // heads per segment
   const long long tps = one_src ? (hps + 31) / 32 : 1;            // tasks per segment (unused otherwise)
+  const int hpr = int(m.row_bytes / HB);                          // heads per row
   const long long n_tasks = one_src ? m.n_segs * tps : (m.n_segs + 31) / 32;
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
 
-  // task -> (destination byte offset, number of heads); issues its load into buffer b
-  auto issue = [&](long long task, int b, long long &dst, int &nh) {
+  // task -> (destination byte offset, number of heads, sequence position of
+  // this lane's head when rotating); issues its load into buffer b
+  auto issue = [&](long long task, int b, long long &dst, int &nh, int &pos) {
     uint8_t *bufp = buf0 + b * BUF;
     if (one_src) {
       const long long seg = task / tps;
       const long long c = task - seg * tps;
       nh = int(min(32LL, hps - c * 32));
       long long so, dof;
-      map_segment(m, seg, so, dof);
+      int p0 = 0;
+      map_segment(m, seg, so, dof, ROPE ? &p0 : nullptr);
       dst = dof + c * 32 * HB;
+      // S2T: the segment holds Sp whole destination rows of hpr heads each
+      if constexpr (ROPE) pos = p0 + int(c * 32 + lane) / hpr;
       if (lane == 0) {
         expect_tx(&full[warp][b], nh * HB);
         bulk_g2s(bufp, in + so + c * 32 * HB, nh * HB, &full[warp][b]);
@@ -247,7 +256,9 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
       const long long g0 = task * 32;
       nh = int(min(32LL, m.n_segs - g0));
       long long so, dof;
-      map_segment(m, g0 + (lane < nh ? lane : 0), so, dof);
+      int p0 = 0;
+      map_segment(m, g0 + (lane < nh ? lane : 0), so, dof, ROPE ? &p0 : nullptr);
+      pos = p0;                                                   // SEQ2HEAD: this lane's row
       dst = __shfl_sync(0xffffffffu, dof, 0);                     // destination rows are consecutive
       if (lane == 0) expect_tx(&full[warp][b], nh * HB);
       __syncwarp();
@@ -257,8 +268,8 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
 
   bool ok = true;
   long long dst_cur = 0, dst_next = 0;
-  int nh_cur = 0, nh_next = 0;
-  if (gw < n_tasks) issue(gw, 0, dst_cur, nh_cur);
+  int nh_cur = 0, nh_next = 0, pos_cur = 0, pos_next = 0;
+  if (gw < n_tasks) issue(gw, 0, dst_cur, nh_cur, pos_cur);
   int i = 0;
   for (long long task = gw; task < n_tasks && ok; task += nw, ++i) {
     const int b = i & 1;
@@ -267,7 +278,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
       // the store of the previous task used the other buffer: it must have read it
       if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       __syncwarp();
-      issue(next, b ^ 1, dst_next, nh_next);
+      issue(next, b ^ 1, dst_next, nh_next, pos_next);
     }
     {
       const unsigned long long t0 = gtimer();
@@ -307,23 +318,13 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
       const float inv = rsqrtf(ss * (1.0f / float(D)) + eps);
       // the rotary angles of this head's token: its index s in the frame (S2T)
       // or in the sequence (SEQ2HEAD), a row of the (cos, sin) table
-      const float2 *rot = nullptr;
-      if (rope) {
-        long long pos;
-        if (m.mode == ST_S2T) {
-          const long long r = (dst_cur + (long long)lane * HB) / m.row_bytes;   // destination (y) row
-          pos = ((r / ((long long)m.Tq * m.Ss)) % m.n_s) * m.Ss + r % m.Ss;
-        } else {
-          pos = (dst_cur / HB + lane) % m.N;                                  // destination (q, b, h1, n) row
-        }
-        rot = rope + pos * (D / 2);
-      }
+      const float2 *rot = ROPE ? rope + (long long)pos_cur * (D / 2) : nullptr;
 #pragma unroll
       for (int u0 = 0; u0 < VPH; ++u0) {
         const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
         const uint4 v = *reinterpret_cast<const uint4 *>(h + u * 16);
         *reinterpret_cast<uint4 *>(h + u * 16) =
-            st::rms_rope_vec<T>(v, inv, g_s + u * EPV, rot ? rot + u * (EPV / 2) : nullptr);
+            st::rms_rope_vec<T, ROPE>(v, inv, g_s + u * EPV, ROPE ? rot + u * (EPV / 2) : nullptr);
       }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -331,6 +332,7 @@ __global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char
     if (lane == 0) bulk_s2g(out + dst_cur, bufp, nh_cur * HB);
     dst_cur = dst_next;
     nh_cur = nh_next;
+    pos_cur = pos_next;
   }
   if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   if (!ok && lane == 0) {
@@ -348,7 +350,7 @@ st_status launch_rms_d(const Map &m, const char *in, char *out, const float *gam
                        cudaStream_t s, const float2 *rope) {
   constexpr int BUF = 32 * D * int(sizeof(T));
   constexpr int SMEM = RMS_WARPS * 2 * BUF;
-  auto kern = relayout_rms<T, D>;
+  auto kern = rope ? relayout_rms<T, D, true> : relayout_rms<T, D, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
     return ST_ERR_CUDA;
   int per_sm = 0;
@@ -458,7 +460,7 @@ st_status relayout_impl(st_relayout_mode mode, const void *in, void *out, int el
       // rotary angles of the attended sequence: tokens of a frame (S2T) or of the sequence (SEQ2HEAD)
       if (mode != ST_S2T && mode != ST_SEQ2HEAD) return ST_ERR_UNSUPPORTED;
       if (rms_head_dim % 2 || rope_positions < (mode == ST_S2T ? S_or_H : T_or_N)) return ST_ERR_SHAPE;
-      if (!st::is_aligned(rope_table, 8)) return ST_ERR_ALIGN;
+      if (!st::is_aligned(rope_table, 16)) return ST_ERR_ALIGN;
       rope = reinterpret_cast<const float2 *>(rope_table);
     }
     return elem_bytes == 2 ? launch_rms<uint16_t>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s, rope)

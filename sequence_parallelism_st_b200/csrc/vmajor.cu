@@ -254,7 +254,10 @@ struct RowMap {
   int Ss, Tq, n_s, n_t, B, Sp, Tn;
 };
 
-__device__ __forceinline__ long long y_to_x(const RowMap &m, long long r) {
+// y row -> x row; optionally s1 (the row's index in its x segment of Sp
+// rows) and pos (the token's index s in its frame, j * Ss + s2).
+__device__ __forceinline__ long long y_to_x(const RowMap &m, long long r, int *s1_out = nullptr,
+                                            int *pos_out = nullptr) {
   uint32_t g = uint32_t(r);                    // rows < 2^31 (checked on the host)
   const uint32_t rest = st::fdiv(g, m.fSs), s2 = g - rest * m.Ss;
   const uint32_t blk = st::fdiv(rest, m.fTq), t2 = rest - blk * m.Tq;
@@ -262,6 +265,8 @@ __device__ __forceinline__ long long y_to_x(const RowMap &m, long long r) {
   const uint32_t qb = st::fdiv(b2, m.fnt), i = b2 - qb * m.n_t;
   const uint32_t q = st::fdiv(qb, m.fB), b = qb - q * m.B;
   const uint32_t p = st::fdiv(s2, m.fSp), s1 = s2 - p * m.Sp;
+  if (s1_out) *s1_out = int(s1);
+  if (pos_out) *pos_out = int(j * m.Ss + s2);
   const long long blk_x = (((long long)p * m.B + b) * m.n_t + i) * m.n_s + j;
   return (blk_x * m.Tn + (long long)q * m.Tq + t2) * m.Sp + s1;
 }
@@ -409,7 +414,7 @@ __device__ __forceinline__ unsigned long long gtimer() {
 // fill a 32-head buffer; the bulk copy engine brings each row in (one copy per
 // row) while the previous task is normalised, one lane normalises one head in
 // shared memory, and one bulk copy per row writes it back.
-template <typename T, int D>
+template <typename T, int D, bool ROPE>
 __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char *__restrict__ in, char *__restrict__ out,
                                                                      const int *__restrict__ idx,
                                                                      const int *__restrict__ count, long long n,
@@ -431,7 +436,7 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
   idx = st::after_wait(idx);
   count = st::after_wait(count);
   gamma = st::after_wait(gamma);
-  if (rope) rope = st::after_wait(rope);
+  if constexpr (ROPE) rope = st::after_wait(rope);
   for (int d = threadIdx.x; d < D; d += blockDim.x) g_s[d] = gamma[d];
   if (lane == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh_u32(&full[warp][0])) : "memory");
@@ -504,8 +509,9 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
     if (lane < rpt * hpr && ((vm_cur >> (lane / hpr)) & 1u)) {
       const int j = lane / hpr, h = lane - j * hpr;
       // the full relayout normalises head (s1 * hpr + h) of a segment on lane (s1 * hpr + h) % 32
-      const long long src = y_to_x(rm, idx[t * rpt + j]);
-      const int fl = int(((src % rm.Sp) * hpr + h) % 32);
+      int s1, pos = 0;
+      y_to_x(rm, idx[t * rpt + j], &s1, ROPE ? &pos : nullptr);
+      const int fl = (s1 * hpr + h) % 32;
       const int r0 = (fl * ROT) % VPH;
       uint8_t *hp = bufp + j * row_bytes + h * HB;
       float ss = 0.f;
@@ -530,17 +536,13 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
       }
       const float inv = rsqrtf(ss * (1.0f / float(D)) + eps);
       // rotary angles of the row's token: its index s in the frame
-      const float2 *rot = nullptr;
-      if (rope) {
-        const long long r = idx[t * rpt + j];
-        rot = rope + (((r / ((long long)rm.Tq * rm.Ss)) % rm.n_s) * rm.Ss + r % rm.Ss) * (D / 2);
-      }
+      const float2 *rot = ROPE ? rope + (long long)pos * (D / 2) : nullptr;
 #pragma unroll
       for (int u0 = 0; u0 < VPH; ++u0) {
         const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
         const uint4 v = *reinterpret_cast<const uint4 *>(hp + u * 16);
         *reinterpret_cast<uint4 *>(hp + u * 16) =
-            st::rms_rope_vec<T>(v, inv, g_s + u * EPV, rot ? rot + u * (EPV / 2) : nullptr);
+            st::rms_rope_vec<T, ROPE>(v, inv, g_s + u * EPV, ROPE ? rot + u * (EPV / 2) : nullptr);
       }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -578,7 +580,7 @@ st_status launch_gather_rms(int D, const char *in, char *out, const int *idx, co
                             const float2 *rope) {
 #define ST_GATHER(DD)                                                                                       \
   {                                                                                                         \
-    auto kern = rows_gather_rms<T, DD>;                                                                     \
+    auto kern = rope ? rows_gather_rms<T, DD, true> : rows_gather_rms<T, DD, false>;                       \
     const int smem = GATHER_WARPS * 2 * 32 * DD * int(sizeof(T));                                           \
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)       \
       return ST_ERR_CUDA;                                                                                   \
@@ -850,7 +852,7 @@ ST_API st_status vmajor_relayout_rows(const void *in_x, void *out_y, const int *
   if (rope_table) {                                           // rides on the RMSNorm pass
     if (!rms_gamma) return ST_ERR_NULL;
     if (rms_head_dim % 2 || rope_positions < S) return ST_ERR_SHAPE;
-    if (!st::is_aligned(rope_table, 8)) return ST_ERR_ALIGN;
+    if (!st::is_aligned(rope_table, 16)) return ST_ERR_ALIGN;
   }
   const long long bytes = n * C * esize;
   const char *i0 = static_cast<const char *>(in_x);
