@@ -179,6 +179,7 @@ def test_sender_vmajor_rejects(st):
     assert rows_call(out=VP(0x100000 + 32)) == st.ST_ERR_SHAPE
     assert rows_call(rope=VP(0x700000), n_pos=16) == st.ST_ERR_NULL             # RoPE rides on the RMSNorm
     assert rows_call(gamma=FAKE_IN, hd=32, rope=VP(0x700000), n_pos=15) == st.ST_ERR_SHAPE   # table too short
+    assert rows_call(gamma=FAKE_IN, hd=32, rope=VP(0x700008), n_pos=16) == st.ST_ERR_ALIGN   # table read 16 B at a time
 
 
 def test_rope_rejects(st):
@@ -196,3 +197,4 @@ def test_rope_rejects(st):
     assert call(rope=None) == st.ST_ERR_NULL
     assert call(mode=st.ST_T2S) == st.ST_ERR_UNSUPPORTED
     assert call(n_pos=15) == st.ST_ERR_SHAPE
+    assert call(rope=VP(0x700008)) == st.ST_ERR_ALIGN
