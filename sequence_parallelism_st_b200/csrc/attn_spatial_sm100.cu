@@ -323,6 +323,8 @@ struct Params {
   // LSE (read per row by the epilogue; o may alias o_acc)
   const float *o_acc;
   const float *lse_acc;
+  int n_items;               // work items of the launch
+  int reverse;               // 1: items are walked from the last (merge launches)
   uint32_t epoch;
 };
 
@@ -371,6 +373,10 @@ struct Item {
 };
 __device__ __forceinline__ Item decode(const Params &p, int x) {
   Item it;
+  // A merge launch walks the items from the last: the accumulated rows the
+  // previous launch wrote last, and the Q tiles it read last, are still in L2
+  // when this launch starts.  Every role decodes through here, so all agree.
+  if (p.reverse) x = p.n_items - 1 - x;
   it.qb = x % p.q_blocks;
   x /= p.q_blocks;
   it.h = x % p.g.H;
@@ -1137,6 +1143,8 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   const long long items = (long long)p.q_blocks * g.H * g.B * p.n_frames;
   if (items <= 0) return ST_OK;
   if (items > 0x7fffffffLL) return ST_ERR_SHAPE;
+  p.n_items = int(items);
+  p.reverse = o_acc != nullptr ? 1 : 0;
   const int ctas = int(items < st::num_sms() ? items : st::num_sms());  // persistent: one CTA per SM
   auto kern = attn_fwd_sm100<D, MERGE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM) != cudaSuccess)
