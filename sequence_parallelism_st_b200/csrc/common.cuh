@@ -100,32 +100,38 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// The (cos, sin) pairs of one 16-byte vector of a head (EPV / 2 pairs, 16-byte
+// aligned in the table): two 16-byte reads for bf16, one for fp32.
+template <typename T> struct RotVec {
+  float4 c[sizeof(T) == 2 ? 2 : 1];
+};
+template <typename T> __device__ __forceinline__ RotVec<T> load_rot(const float2 *rot) {
+  RotVec<T> r;
+#pragma unroll
+  for (int i = 0; i < (sizeof(T) == 2 ? 2 : 1); ++i) r.c[i] = reinterpret_cast<const float4 *>(rot)[i];
+  return r;
+}
+
 // One 16-byte vector of a head on its way through the per-head RMSNorm and,
-// with a rotation table, the rotary position embedding: every element x
-// becomes y = x * inv * g, then pair k of the vector (elements 2k, 2k+1, pair
-// index u * EPV / 2 + k of the head) turns by the angle whose (cos, sin) is
-// rot[k]:  (y0, y1) -> (y0 c - y1 s, y0 s + y1 c); rot is 16-byte aligned.
-// T: uint16_t (bf16) or float.  ROPE = false: the RMSNorm alone, rot unused
-// (the rotation is a compile-time choice, so a kernel without it holds no
-// table load at all).
+// with ROPE, the rotary position embedding: every element x becomes
+// y = x * inv * g, then pair k of the vector (elements 2k, 2k+1, pair index
+// u * EPV / 2 + k of the head) turns by the angle whose (cos, sin) is pair k
+// of cs:  (y0, y1) -> (y0 c - y1 s, y0 s + y1 c).  T: uint16_t (bf16) or
+// float.  The rotation is a compile-time choice, so a kernel without it holds
+// no table load at all; kernels load cs (load_rot) a few vectors ahead.
 template <typename T, bool ROPE>
-__device__ __forceinline__ uint4 rms_rope_vec(uint4 v, float inv, const float *gg, const float2 *rot) {
+__device__ __forceinline__ uint4 rms_rope_vec(uint4 v, float inv, const float *gg, const RotVec<T> &cs) {
   if constexpr (sizeof(T) == 2) {
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float4 cs4[2] = {};                        // (cos, sin) of the 4 pairs: two 16-byte reads
-    if constexpr (ROPE) {
-      cs4[0] = reinterpret_cast<const float4 *>(rot)[0];
-      cs4[1] = reinterpret_cast<const float4 *>(rot)[1];
-    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       float a = __uint_as_float(w[k] << 16) * inv * gg[2 * k];
       float b = __uint_as_float(w[k] & 0xffff0000u) * inv * gg[2 * k + 1];
       if constexpr (ROPE) {
-        const float2 cs = (k & 1) ? make_float2(cs4[k >> 1].z, cs4[k >> 1].w)
-                                  : make_float2(cs4[k >> 1].x, cs4[k >> 1].y);
-        const float a2 = a * cs.x - b * cs.y;
-        b = a * cs.y + b * cs.x;
+        const float4 c = cs.c[k >> 1];
+        const float2 r = (k & 1) ? make_float2(c.z, c.w) : make_float2(c.x, c.y);
+        const float a2 = a * r.x - b * r.y;
+        b = a * r.y + b * r.x;
         a = a2;
       }
       w[k] = pack_bf16x2(a, b);
@@ -135,17 +141,23 @@ __device__ __forceinline__ uint4 rms_rope_vec(uint4 v, float inv, const float *g
     float y[4] = {__uint_as_float(v.x) * inv * gg[0], __uint_as_float(v.y) * inv * gg[1],
                   __uint_as_float(v.z) * inv * gg[2], __uint_as_float(v.w) * inv * gg[3]};
     if constexpr (ROPE) {
-      const float4 c4 = reinterpret_cast<const float4 *>(rot)[0];
+      const float4 c = cs.c[0];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        const float2 cs = k ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+        const float2 r = k ? make_float2(c.z, c.w) : make_float2(c.x, c.y);
         const float a = y[2 * k], b = y[2 * k + 1];
-        y[2 * k] = a * cs.x - b * cs.y;
-        y[2 * k + 1] = a * cs.y + b * cs.x;
+        y[2 * k] = a * r.x - b * r.y;
+        y[2 * k + 1] = a * r.y + b * r.x;
       }
     }
     return make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]), __float_as_uint(y[3]));
   }
 }
+
+// Rotation table reads of a head, RG vectors at a time: the normalise loop of
+// the RMSNorm kernels loads the pairs of RG vectors together (one round trip
+// per group instead of one per vector), the first group before the head's sum
+// of squares.
+constexpr int RG = 4;
 
 }  // namespace st

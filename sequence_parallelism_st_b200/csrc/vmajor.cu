@@ -513,7 +513,16 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
       y_to_x(rm, idx[t * rpt + j], &s1, ROPE ? &pos : nullptr);
       const int fl = (s1 * hpr + h) % 32;
       const int r0 = (fl * ROT) % VPH;
+      auto uix = [&](int u0) { return u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH; };
       uint8_t *hp = bufp + j * row_bytes + h * HB;
+      // rotary angles of the row's token (its index s in the frame); the first
+      // group of pairs is on its way during the sum of squares
+      const float2 *rot = ROPE ? rope + (long long)pos * (D / 2) : nullptr;
+      st::RotVec<T> cs[st::RG];
+      if constexpr (ROPE) {
+#pragma unroll
+        for (int g = 0; g < st::RG && g < VPH; ++g) cs[g] = st::load_rot<T>(rot + uix(g) * (EPV / 2));
+      }
       float ss = 0.f;
 #pragma unroll
       for (int u0 = 0; u0 < VPH; ++u0) {
@@ -535,14 +544,18 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
         }
       }
       const float inv = rsqrtf(ss * (1.0f / float(D)) + eps);
-      // rotary angles of the row's token: its index s in the frame
-      const float2 *rot = ROPE ? rope + (long long)pos * (D / 2) : nullptr;
 #pragma unroll
       for (int u0 = 0; u0 < VPH; ++u0) {
-        const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
+        if constexpr (ROPE) {
+          if (u0 > 0 && u0 % st::RG == 0) {
+#pragma unroll
+            for (int g = 0; g < st::RG; ++g)
+              if (u0 + g < VPH) cs[g] = st::load_rot<T>(rot + uix(u0 + g) * (EPV / 2));
+          }
+        }
+        const int u = uix(u0);
         const uint4 v = *reinterpret_cast<const uint4 *>(hp + u * 16);
-        *reinterpret_cast<uint4 *>(hp + u * 16) =
-            st::rms_rope_vec<T, ROPE>(v, inv, g_s + u * EPV, ROPE ? rot + u * (EPV / 2) : nullptr);
+        *reinterpret_cast<uint4 *>(hp + u * 16) = st::rms_rope_vec<T, ROPE>(v, inv, g_s + u * EPV, cs[u0 % st::RG]);
       }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
