@@ -68,16 +68,17 @@ def peaks():
     return FALLBACK, "fallback"
 
 
-def kernel_traffic():
+def kernel_traffic(workload):
     """DRAM bytes per launch of the spatial kernel from the committed ncu summary,
-    or None when the kernel source changed since the capture."""
+    or None when the kernel source changed since the capture or the bench runs
+    another workload than the captured one."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     h = hashlib.sha256(open(SPATIAL_SRC, "rb").read()).hexdigest()[:16]
     e = d.get("st_attn_spatial", {})
-    if e.get("source_sha") != h or e.get("workload") != "opensora_low":
+    if e.get("source_sha") != h or e.get("workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -586,7 +587,7 @@ def run_ours(args, w, rank, world, dev):
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(statistics.mean(e2e_ms), 5)},
         "roofline": {"bound": "tensor", "kernel": "st_attn_spatial", "achieved": round(achieved, 2),
                      "peak": tc_peak, "peak_source": tc_src, "unit": "TFLOP/s",
-                     "frac": round(achieved / tc_peak, 4), "traffic": kernel_traffic(),
+                     "frac": round(achieved / tc_peak, 4), "traffic": kernel_traffic(w.name),
                      "algorithmic_flop_per_launch": w.spatial_flops() / w.R},
         "kernels": kernels,
         "gpu_launches": launches * n_steps,
