@@ -526,7 +526,7 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char 
       float ss = 0.f;
 #pragma unroll
       for (int u0 = 0; u0 < VPH; ++u0) {
-        const int u = u0 + r0 < VPH ? u0 + r0 : u0 + r0 - VPH;
+        const int u = uix(u0);
         const uint4 v = *reinterpret_cast<const uint4 *>(hp + u * 16);
         if constexpr (sizeof(T) == 2) {
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
