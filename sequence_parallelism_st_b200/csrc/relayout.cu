@@ -199,8 +199,10 @@ __device__ __forceinline__ unsigned long long gtimer() {
 constexpr int RMS_WARPS = 4;
 constexpr unsigned long long RMS_WAIT_NS = 2000000000ull;
 
+// Five CTAs per SM (20 warps) without the rotation: registers capped for it,
+// and the launch asks for the largest shared-memory carveout.
 template <typename T, int D, bool ROPE>
-__global__ void __launch_bounds__(RMS_WARPS * 32) relayout_rms(Map m, const char *__restrict__ in,
+__global__ void __launch_bounds__(RMS_WARPS * 32, ROPE ? 1 : 5) relayout_rms(Map m, const char *__restrict__ in,
                                                                char *__restrict__ out,
                                                                const float *__restrict__ gamma, float eps,
                                                                const float2 *__restrict__ rope) {
@@ -364,7 +366,8 @@ st_status launch_rms_d(const Map &m, const char *in, char *out, const float *gam
   constexpr int BUF = 32 * D * int(sizeof(T));
   constexpr int SMEM = RMS_WARPS * 2 * BUF;
   auto kern = rope ? relayout_rms<T, D, true> : relayout_rms<T, D, false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return ST_ERR_CUDA;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, RMS_WARPS * 32, SMEM) != cudaSuccess ||

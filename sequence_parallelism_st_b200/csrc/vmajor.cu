@@ -414,8 +414,10 @@ __device__ __forceinline__ unsigned long long gtimer() {
 // fill a 32-head buffer; the bulk copy engine brings each row in (one copy per
 // row) while the previous task is normalised, one lane normalises one head in
 // shared memory, and one bulk copy per row writes it back.
+// Five CTAs per SM (20 warps) without the rotation: registers capped for it,
+// and the launch asks for the largest shared-memory carveout.
 template <typename T, int D, bool ROPE>
-__global__ void __launch_bounds__(GATHER_WARPS * 32) rows_gather_rms(const char *__restrict__ in, char *__restrict__ out,
+__global__ void __launch_bounds__(GATHER_WARPS * 32, ROPE ? 1 : 5) rows_gather_rms(const char *__restrict__ in, char *__restrict__ out,
                                                                      const int *__restrict__ idx,
                                                                      const int *__restrict__ count, long long n,
                                                                      int row_vecs, const float *__restrict__ gamma,
@@ -595,7 +597,8 @@ st_status launch_gather_rms(int D, const char *in, char *out, const int *idx, co
   {                                                                                                         \
     auto kern = rope ? rows_gather_rms<T, DD, true> : rows_gather_rms<T, DD, false>;                       \
     const int smem = GATHER_WARPS * 2 * 32 * DD * int(sizeof(T));                                           \
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)       \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||     \
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)     \
       return ST_ERR_CUDA;                                                                                   \
     int per_sm = 0;                                                                                         \
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, GATHER_WARPS * 32, smem) != cudaSuccess || \
