@@ -55,8 +55,10 @@ import synth  # noqa: E402
 
 METRIC = "attention TFLOP/s & relayout GB/s on 1 B200, as fraction of bf16/HBM peak"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP_BASE = 9            # relayouts 3+1, vmajor 3 (mask, compaction, scatter), merge 1, temporal 1
-                                      # (+ R spatial launches; the fused merge has no merge launch)
+LAUNCHES_PER_STEP_BASE = 9            # receiver side: relayouts 3+1, vmajor 3 (mask, compaction, scatter),
+                                      # merge 1, temporal 1; + R spatial launches; the fused merge has no
+                                      # merge launch; sender side: mask + V rows, compaction and K rows
+                                      # replace the K and V relayouts and the three vmajor launches (2 fewer)
 SPATIAL_SRC = os.path.join(ROOT, "sequence_parallelism_st_b200", "csrc", "attn_spatial_sm100.cu")
 
 
@@ -431,6 +433,22 @@ def kernel_bytes(w, frac_active, sender=False):
     }
 
 
+def max_over_ranks(total_ms, world, dev):
+    """The job's time: the largest of the ranks' device times (every rank
+    takes part in the same collective; a single rank returns its own)."""
+    if world <= 1:
+        return float(total_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world, flop_per_replica_step, ms_per_step):
+    """Whole-job throughput in TFLOP/s: every rank runs one replica of the step
+    (weak scaling), so the job does world x the flop of a step per step time."""
+    return world * flop_per_replica_step / (ms_per_step * 1e-3) / 1e12
+
+
 def run_ours(args, w, rank, world, dev):
     import sequence_parallelism_st_b200 as st
     stp = Step(st, w, dev)
@@ -471,11 +489,7 @@ def run_ours(args, w, rank, world, dev):
     if world > 1:
         torch.distributed.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     status = st.st_check_device_status()
     # per-kernel breakdown from a separate pass: events between the kernel
     # groups would otherwise sit inside the timed steps
@@ -543,8 +557,8 @@ def run_ours(args, w, rank, world, dev):
     f = flops(w)
     n_steps = args.steps
     ms = total_ms / n_steps
-    value = world * f / (ms * 1e-3) / 1e12
-    e2e_val = world * f / (statistics.mean(e2e_ms) * 1e-3) / 1e12
+    value = whole_job_value(world, f, ms)
+    e2e_val = whole_job_value(world, f, statistics.mean(e2e_ms))
     frac_active = active / stp.n
     kb = kernel_bytes(w, frac_active, stp.sender_vmajor)
     kernels = {}

@@ -1,0 +1,67 @@
+"""The multi-rank host logic of bench.py on CPU: two gloo ranks (one process
+each, 127.0.0.1) agree on the job time as the max over ranks, the whole-job
+value counts every replica, and a single rank needs no process group."""
+import datetime
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, times, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
+                                         timeout=datetime.timedelta(seconds=30))
+    try:
+        torch.distributed.barrier()
+        q.put((rank, bench.max_over_ranks(times[rank], world, torch.device("cpu"))))
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+@pytest.mark.parametrize("times", [(12.5, 17.25), (9.0, 3.0)])
+def test_max_over_ranks_two_gloo_ranks(times):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, times, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = {}
+    try:
+        for _ in procs:
+            r, v = q.get(timeout=60)
+            got[r] = v
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    assert got == {0: max(times), 1: max(times)}
+
+
+def test_single_rank_needs_no_group():
+    assert not torch.distributed.is_initialized()
+    assert bench.max_over_ranks(4.5, 1, torch.device("cpu")) == 4.5
+
+
+def test_whole_job_value_counts_every_replica():
+    f = 106.17e9                                      # flop of one replica's step
+    one = bench.whole_job_value(1, f, 0.36)
+    assert one == pytest.approx(f / 0.36e-3 / 1e12)
+    # weak scaling: N replicas in the same time are N times the work
+    assert bench.whole_job_value(8, f, 0.36) == pytest.approx(8 * one)
+    # the max-over-ranks time decides: a slower rank lowers the job's value
+    assert bench.whole_job_value(2, f, 0.40) < bench.whole_job_value(2, f, 0.36)
