@@ -1,9 +1,17 @@
 """Benchmark of the spatial-temporal attention hot path on B200.
 
-One step = one pass of every hot-path step over one ST-DiT attention block of
-the OpenSora-like low-resolution workload (B=1, T=16 frames, S=1200 tokens,
-16 heads x 72, bf16, virtual P=4, N_T=N_S=4, KV chunks R=2):
+One step = one pass of every hot-path step of one attention block over one
+batch of seeded synthetic inputs.  ``--workload`` picks the block:
 
+* ``image_4096px`` (default): image-DiT full attention, B=1, N=65536 tokens
+  (256x256 patches), 24 heads x 128, bf16, per-head RMSNorm on Q/K, KV in
+  R=8 ring chunks merged by log-sum-exp, virtual Ulysses P=8 (ImageStep):
+  SEQ2HEAD of V, K, Q (RMSNorm fused), attention, HEAD2SEQ of the output.
+* ``vmajor_2304px``: V-Major selective attention, N=20736 (144x144), 24 x
+  128 (VMajorStep): L1 change mask of V, compaction, cache update of the
+  active tokens' K/V rows, attention of the fresh Q on the caches.
+* ``opensora_low`` / ``video_1080p`` / ``tiny``: ST-DiT block (Step),
+  B=1, T frames of S tokens, virtual P, N_T/N_S slices, R KV chunks:
   1. V-Major on the sending side: the L1 change of V against the previous
      step's V is measured on the spatially sharded layout, and only the
      active tokens take part in the all-to-all S->T -- their V rows and
@@ -24,12 +32,12 @@ the OpenSora-like low-resolution workload (B=1, T=16 frames, S=1200 tokens,
   5. temporal attention over the T frames of every token, read in place from
      the spatially sharded slice layout (st_attn_temporal).
 
-value = attention FLOP of the step (4*rows*keys*D per head, spatial and
-temporal) / device time of the step; the per-kernel breakdown (TFLOP/s or
-GB/s) is in "kernels".  Inputs are resident in HBM; L2 is flushed (a
-256 MiB write) between timed steps, outside the timed events.  Under torchrun
-every rank runs its own replica (weak scaling, no collective on the data
-path); the time is the max over ranks.
+value = attention FLOP of the step (4*rows*keys*D per head) / device time of
+the step; the per-kernel breakdown (TFLOP/s or GB/s) is in "kernels".  Inputs
+are resident in HBM; L2 is flushed (a 256 MiB write) between timed steps,
+outside the timed events.  Under torchrun every rank runs its own replica
+(weak scaling, no collective on the data path); the time is the max over
+ranks.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
 same workload instead (rank 0 only).
@@ -410,6 +418,274 @@ class Step:
             out[name] = sum(ts) / len(ts)
         return out
 
+    # ------------------------------------------------------------ bench interface
+    def outputs(self):
+        """Device results a caller reads back after the step."""
+        return [self.ox, self.ot]
+
+    def set_io(self, d, outs):
+        self.d = d
+        self.ox, self.ot = outs
+
+    def flops(self):
+        return self.w.spatial_flops() + self.w.temporal_flops()
+
+    def active_tokens(self):
+        return int(self.count.item()) if not hasattr(self, "n_sl") else int(self.counts.sum().item())
+
+    def launches(self):
+        w = self.w
+        if hasattr(self, "n_sl"):
+            return (3 + 3 + w.R + (1 if self.fused_merge else 2)) * self.n_sl + 1
+        # sender-side V-Major: V mask-relayout, compaction and K rows (3) replace 2 relayouts + 3 V-Major launches
+        return LAUNCHES_PER_STEP_BASE + w.R - (1 if self.fused_merge else 0) - (2 if self.sender_vmajor else 0)
+
+    def group_flops(self):
+        """Attention FLOP of each timed kernel group (the tensor-bound ones)."""
+        w, R = self.w, self.w.R
+        sp = w.spatial_flops()
+        if self.fused_merge:
+            return {"spatial": sp / R, "spatial_merge": sp * (R - 1) / R, "temporal": w.temporal_flops()}
+        return {"spatial": sp, "temporal": w.temporal_flops()}
+
+    def group_bytes(self, frac_active):
+        return kernel_bytes(self.w, frac_active, self.sender_vmajor)
+
+    def roofline_launch(self, ktimes):
+        """(flop of one launch of the dominant kernel, its mean duration in ms):
+        the chunk-0 spatial launch."""
+        w = self.w
+        return w.spatial_flops() / w.R, ktimes["spatial"] / (1 if self.fused_merge else w.R)
+
+    def describe(self, args):
+        w = self.w
+        return {"B": w.B, "T": w.T, "S": w.S, "H": w.H, "D": w.D, "P": w.P, "N_T": w.n_t, "N_S": w.n_s,
+                "kv_chunks": w.R,
+                "schedule": "serial" if not hasattr(self, "n_sl") else
+                f"overlap: {self.n_sl} shard ranges, attention on {self.att_sms} SMs",
+                "chunk_merge": "fused into the attention kernel" if self.fused_merge else "attn_chunk_merge",
+                "vmajor": "sender side (mask on x, active K/V rows into the caches)" if self.sender_vmajor else
+                "receiver side (full relayouts, mask on y, scatter)",
+                "qk_rope": self.rope_table is not None}
+
+
+class ImageStep:
+    """Buffers and launches of one image-DiT full-attention block step: B = 1,
+    N tokens of H heads x D, virtual Ulysses partition P, R KV ring chunks.
+
+      1. SEQ2HEAD of V (V first: it needs no normalisation), then of K and Q
+         with the per-head RMSNorm fused into the move (ulysses_relayout);
+         the head-sharded layout [P, B, H/P, N, D] holds each head's sequence
+         contiguously, so its B*H head sequences are the attention's frames;
+      2. full attention over the N keys in R ring chunks merged by log-sum-exp:
+         ``ring`` runs one launch that walks each query block's chunks from its
+         own (stationary) chunk onwards and carries the running max, row sum and
+         O across the chunk boundaries (st_attn_ring); ``chunks`` runs chunk 0
+         (st_attn_spatial, fp32 partial + LSE) and merges every later chunk
+         into it inside the attention kernel (st_attn_spatial_merge);
+      3. HEAD2SEQ of the output back to the sequence-sharded layout.
+    """
+
+    def __init__(self, st, w, dev, attn="ring"):
+        self.st, self.w, self.dev, self.attn = st, w, dev, attn
+        N, H, D, C, P, B = w.S, w.H, w.D, w.C, w.P, w.B
+        assert w.T == 1 and N % P == 0 and H % P == 0
+        q, k, v = synth.qkv(w)                                # [B, 1, N, H, D] = the stacked sequence shards
+        self.host = {"q": q.reshape(-1), "k": k.reshape(-1), "v": v.reshape(-1)}
+        self.d = {name: t.to(dev) for name, t in self.host.items()}
+        self.gamma = synth.rms_gamma(w).to(dev)
+        mk = lambda dt=torch.bfloat16: torch.empty(B * N * C, dtype=dt, device=dev)
+        self.qy, self.ky, self.vy, self.oy, self.ox = mk(), mk(), mk(), mk(), mk()
+        self.lse = [torch.empty(B * H * N, dtype=torch.float32, device=dev) for _ in range(2)]
+        R = w.R
+        # head-sharded y: frames (p, b, h1) of N contiguous tokens, one head each
+        self.frames = B * H
+        if attn == "ring":
+            self.rdesc = st.make_desc(1, self.frames, N, 1, D, st.ST_BF16)
+        else:
+            self.part = mk(torch.float32)
+            self.sdesc = [st.make_desc(1, self.frames, N, 1, D, st.ST_BF16, kv_begin=c * N // R,
+                                       kv_end=(c + 1) * N // R, o_fp32=0 if c == R - 1 else 1) for c in range(R)]
+        self.ev = {}
+        self.timing = False
+
+    _mark = Step._mark
+    kernel_times = Step.kernel_times
+
+    def run(self, timing=False):
+        st, w, d = self.st, self.w, self.d
+        self.timing = timing
+        P, B, N, H, D = w.P, w.B, w.S, w.H, w.D
+        self._mark("relayout_seq2head", True)
+        st.ulysses_relayout("SEQ2HEAD", d["v"], self.vy, P, B, N, H, D)
+        st.ulysses_relayout("SEQ2HEAD", d["k"], self.ky, P, B, N, H, D, rms_gamma=self.gamma, rms_head_dim=D,
+                            rms_eps=w.rms_eps)
+        st.ulysses_relayout("SEQ2HEAD", d["q"], self.qy, P, B, N, H, D, rms_gamma=self.gamma, rms_head_dim=D,
+                            rms_eps=w.rms_eps)
+        self._mark("relayout_seq2head", False)
+        self._mark("spatial", True)
+        if self.attn == "ring":
+            st.st_attn_ring(self.qy, self.ky, self.vy, self.oy, self.lse[0], w.R, desc=self.rdesc)
+            self._mark("spatial", False)
+        elif w.R == 1:
+            st.st_attn_spatial(self.qy, self.ky, self.vy, self.oy, self.lse[0], desc=self.sdesc[0])
+            self._mark("spatial", False)
+        else:
+            st.st_attn_spatial(self.qy, self.ky, self.vy, self.part, self.lse[0], desc=self.sdesc[0])
+            self._mark("spatial", False)
+            self._mark("spatial_merge", True)
+            for c in range(1, w.R - 1):
+                st.st_attn_spatial_merge(self.qy, self.ky, self.vy, self.part, self.lse[0], self.part, self.lse[0],
+                                         desc=self.sdesc[c])
+            st.st_attn_spatial_merge(self.qy, self.ky, self.vy, self.part, self.lse[0], self.oy, self.lse[1],
+                                     desc=self.sdesc[w.R - 1])
+            self._mark("spatial_merge", False)
+        self._mark("relayout_head2seq", True)
+        st.ulysses_relayout("HEAD2SEQ", self.oy, self.ox, P, B, N, H, D)
+        self._mark("relayout_head2seq", False)
+
+    def outputs(self):
+        return [self.ox]
+
+    def set_io(self, d, outs):
+        self.d = d
+        (self.ox,) = outs
+
+    def flops(self):
+        return self.w.spatial_flops()
+
+    def active_tokens(self):
+        return None
+
+    def launches(self):
+        return 3 + (1 if self.attn == "ring" else self.w.R) + 1
+
+    def group_flops(self):
+        sp, R = self.w.spatial_flops(), self.w.R
+        if self.attn == "ring" or R == 1:
+            return {"spatial": sp}
+        return {"spatial": sp / R, "spatial_merge": sp * (R - 1) / R}
+
+    def group_bytes(self, frac_active):
+        t = self.w.tensor_bytes()
+        return {"relayout_seq2head": 3 * 2 * t, "relayout_head2seq": 2 * t}
+
+    def roofline_launch(self, ktimes):
+        """The ring launch (all R chunks), or the chunk-0 launch of the chunk chain."""
+        sp = self.w.spatial_flops()
+        return (sp if self.attn == "ring" else sp / self.w.R), ktimes["spatial"]
+
+    def describe(self, args):
+        w = self.w
+        return {"B": w.B, "N": w.S, "H": w.H, "D": w.D, "P": w.P, "kv_chunks": w.R, "qk_rmsnorm": True,
+                "relayout": "SEQ2HEAD (V, then K and Q with the RMSNorm) -> attention -> HEAD2SEQ",
+                "chunk_merge": ("one launch, stationary chunk first, running (m, l, O) carried across chunks"
+                                if self.attn == "ring" else
+                                "chunk 0 partial, later chunks merged inside the attention kernel")}
+
+
+class VMajorStep:
+    """Buffers and launches of one V-Major selective attention step: N tokens of
+    H heads x D (T = 1), fresh Q, K and V of this step, the previous step's V
+    and the K/V caches.
+
+      1. per-token L1 change of V against the previous step's V, the mask
+         (L1 > tau), the ascending list of active tokens and the update of the
+         K/V caches with the active tokens' rows (vmajor_mask_compact_scatter);
+      2. attention of the fresh Q against the cached K/V (st_attn_spatial).
+    tau is the golden threshold for the active fraction f.
+    """
+
+    def __init__(self, st, w, dev, frac=0.5):
+        self.st, self.w, self.dev = st, w, dev
+        N, H, D, C = w.S, w.H, w.D, w.C
+        assert w.B == 1 and w.T == 1
+        self.n = N
+        q = synth.randn(w, "q", (1, 1, N, H, D))
+        cur_v, prev_v = synth.vmajor_pair(w, N, C)
+        cur_k, prev_k = synth.vmajor_pair(w, N, C, prev="kprev", noise="knoise")
+        self.frac_target = frac
+        self.tau = json.load(open(os.path.join(ROOT, "tests", "golden", "vmajor_tau.json")))[
+            "workloads"][w.name][str(frac)]["tau"]
+        self.host = {"q": q.reshape(-1), "k": cur_k.reshape(-1), "v": cur_v.reshape(-1)}
+        self.d = {name: t.to(dev) for name, t in self.host.items()}
+        self.vprev = prev_v.reshape(-1).to(dev)
+        self.kcache0, self.vcache0 = prev_k.reshape(-1).to(dev), prev_v.reshape(-1).to(dev)
+        self.kc, self.vc = self.kcache0.clone(), self.vcache0.clone()
+        self.o = torch.empty(N * C, dtype=torch.bfloat16, device=dev)
+        self.mask = torch.empty(N, dtype=torch.uint8, device=dev)
+        self.idx = torch.empty(N, dtype=torch.int32, device=dev)
+        self.count = torch.empty(1, dtype=torch.int32, device=dev)
+        self.ws = torch.empty(max(16, st.vmajor_workspace_bytes(N)), dtype=torch.uint8, device=dev)
+        self.desc = st.make_desc(1, 1, N, H, D, st.ST_BF16)
+        self.ev = {}
+        self.timing = False
+
+    _mark = Step._mark
+    kernel_times = Step.kernel_times
+
+    def reset_caches(self):
+        self.kc.copy_(self.kcache0)
+        self.vc.copy_(self.vcache0)
+
+    def run(self, timing=False):
+        st, d, n, C = self.st, self.d, self.n, self.w.C
+        self.timing = timing
+        self._mark("vmajor", True)
+        st.vmajor_mask_compact_scatter(d["v"].view(n, C), self.vprev.view(n, C), self.tau, self.mask, self.idx,
+                                       self.count, self.ws, [d["k"].view(n, C), d["v"].view(n, C)],
+                                       [self.kc.view(n, C), self.vc.view(n, C)])
+        self._mark("vmajor", False)
+        self._mark("spatial", True)
+        st.st_attn_spatial(d["q"], self.kc, self.vc, self.o, None, desc=self.desc)
+        self._mark("spatial", False)
+
+    def outputs(self):
+        return [self.o]
+
+    def set_io(self, d, outs):
+        self.d = d
+        (self.o,) = outs
+
+    def flops(self):
+        return self.w.spatial_flops()
+
+    def active_tokens(self):
+        return int(self.count.item())
+
+    def launches(self):
+        return 3                      # mask with the fused cache update, compaction, attention
+
+    def group_flops(self):
+        return {"spatial": self.w.spatial_flops()}
+
+    def group_bytes(self, frac_active):
+        # V and its previous value read; the active rows of K and V read and written into the caches
+        t = self.w.tensor_bytes()
+        return {"vmajor": 2 * t + 4 * frac_active * t}
+
+    def roofline_launch(self, ktimes):
+        return self.w.spatial_flops(), ktimes["spatial"]
+
+    def describe(self, args):
+        w = self.w
+        return {"B": w.B, "N": w.S, "H": w.H, "D": w.D, "vmajor_target_fraction": self.frac_target,
+                "vmajor": "mask + compaction + cache update of active K/V rows, attention on the caches"}
+
+
+STEPS = {"st": Step, "image": ImageStep, "vmajor": VMajorStep}
+
+
+def step_kind(w):
+    """The step a workload runs: image-DiT full attention (T = 1 with the Q/K
+    RMSNorm), V-Major selective attention (T = 1 with change fractions), or the
+    ST-DiT block."""
+    if w.T == 1 and w.vmajor_f and not w.rms:
+        return "vmajor"
+    if w.T == 1:
+        return "image"
+    return "st"
+
 
 def flops(w):
     return w.spatial_flops() + w.temporal_flops()
@@ -449,8 +725,12 @@ def whole_job_value(world, flop_per_replica_step, ms_per_step):
     return world * flop_per_replica_step / (ms_per_step * 1e-3) / 1e12
 
 
-def run_ours(args, w, rank, world, dev):
-    import sequence_parallelism_st_b200 as st
+def make_step(st, args, w, dev):
+    kind = step_kind(w)
+    if kind == "image":
+        return ImageStep(st, w, dev, attn=args.attn)
+    if kind == "vmajor":
+        return VMajorStep(st, w, dev, frac=args.vmajor_f)
     stp = Step(st, w, dev)
     stp.fused_merge = args.merge == "fused"
     stp.sender_vmajor = args.vmajor == "sender"
@@ -458,12 +738,14 @@ def run_ours(args, w, rank, world, dev):
         stp.rope_table = st.st_rope_table(w.S, w.D, 10000.0, device=dev)
     if args.schedule == "overlap":
         stp.setup_overlap(args.slices, args.att_sms)
-        step_fn = stp.run_overlap
-        launches = (3 + 3 + w.R + (1 if stp.fused_merge else 2)) * args.slices + 1
-    else:
-        step_fn = stp.run
-        # sender-side V-Major: V mask-relayout, compaction and K rows (3) replace 2 relayouts + 3 V-Major launches
-        launches = LAUNCHES_PER_STEP_BASE + w.R - (1 if stp.fused_merge else 0) - (2 if stp.sender_vmajor else 0)
+    return stp
+
+
+def run_ours(args, w, rank, world, dev):
+    import sequence_parallelism_st_b200 as st
+    stp = make_step(st, args, w, dev)
+    step_fn = stp.run_overlap if hasattr(stp, "n_sl") else stp.run
+    launches = stp.launches()
     pk, pk_src = peaks()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
@@ -471,7 +753,7 @@ def run_ours(args, w, rank, world, dev):
     torch.cuda.synchronize()
     if st.st_check_device_status() != st.ST_OK:
         raise RuntimeError("device status not OK after warm-up")
-    active = int(stp.count.item()) if args.schedule == "serial" else int(stp.counts.sum().item())
+    active = stp.active_tokens()
     # ---- timed: device time of exactly K steps, L2 flushed between steps outside the events
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -506,9 +788,10 @@ def run_ours(args, w, rank, world, dev):
     # step i-1 computes and step i-2's results come down on another, with
     # two device sets of inputs and outputs.  Every step still carries its
     # own host->device and device->host copies inside the timed region.
+    outs0 = stp.outputs()
     d_sets = [stp.d, {k: torch.empty_like(v) for k, v in stp.d.items()}]
-    o_sets = [(stp.ox, stp.ot), (torch.empty_like(stp.ox), torch.empty_like(stp.ot))]
-    out_host = [[torch.empty(stp.n * w.C, dtype=torch.bfloat16).pin_memory() for _ in range(2)] for _ in range(2)]
+    o_sets = [outs0, [torch.empty_like(o) for o in outs0]]
+    out_host = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs0] for _ in range(2)]
     d2h = sum(v.numel() * v.element_size() for v in out_host[0])
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
@@ -533,14 +816,13 @@ def run_ours(args, w, rank, world, dev):
             comp.wait_event(ev_in[i])
             if i >= 2:
                 comp.wait_event(ev_out[i - 2])           # set j's outputs already copied down
-            stp.d = d_sets[j]
-            stp.ox, stp.ot = o_sets[j]
+            stp.set_io(d_sets[j], o_sets[j])
             step_fn()
             ev_comp[i].record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[i])
-                out_host[j][0].copy_(o_sets[j][0], non_blocking=True)
-                out_host[j][1].copy_(o_sets[j][1], non_blocking=True)
+                for hb, db in zip(out_host[j], o_sets[j]):
+                    hb.copy_(db, non_blocking=True)
                 ev_out[i].record(s_out)
         comp.wait_event(ev_out[n - 1])
         b.record(comp)
@@ -550,82 +832,140 @@ def run_ours(args, w, rank, world, dev):
     e2e_pass(3)                                          # warm-up of the pipeline
     n_e2e = max(4, args.steps // 4)
     e2e_ms = [e2e_pass(n_e2e)]
-    stp.d = d_sets[0]
-    stp.ox, stp.ot = o_sets[0]
+    stp.set_io(d_sets[0], o_sets[0])
     if rank != 0:
         return None
-    f = flops(w)
+    f = stp.flops()
     n_steps = args.steps
     ms = total_ms / n_steps
     value = whole_job_value(world, f, ms)
     e2e_val = whole_job_value(world, f, statistics.mean(e2e_ms))
-    frac_active = active / stp.n
-    kb = kernel_bytes(w, frac_active, stp.sender_vmajor)
+    frac_active = None if active is None else active / stp.n
+    gb = stp.group_bytes(frac_active or 0.0)
+    gf = stp.group_flops()
     kernels = {}
     for name, t in ktimes.items():
         ent = {"ms": round(t, 5)}
-        if name in ("spatial", "spatial_merge"):
-            # fused merge: "spatial" is chunk 0, "spatial_merge" the other R-1 chunks with the merge
-            share = (1.0 if not stp.fused_merge else (1.0 / w.R if name == "spatial" else (w.R - 1.0) / w.R))
-            ent["tflops"] = round(w.spatial_flops() * share / (t * 1e-3) / 1e12, 2)
-            ent["frac_of_bf16_peak"] = round(ent["tflops"] / pk["bf16_tflops"], 4)
-        else:
-            ent["gbs"] = round(kb[name] / (t * 1e-3) / 1e9, 1)
+        if name in gf:
+            ent["tflops"] = round(gf[name] / (t * 1e-3) / 1e12, 2)
+            if name != "temporal":
+                ent["frac_of_bf16_peak"] = round(ent["tflops"] / pk["bf16_tflops"], 4)
+        if name in gb:
+            ent["gbs"] = round(gb[name] / (t * 1e-3) / 1e9, 1)
             ent["frac_of_hbm_peak"] = round(ent["gbs"] / pk["hbm_gbs"], 4)
-            if name == "temporal":
-                ent["tflops"] = round(w.temporal_flops() / (t * 1e-3) / 1e12, 2)
         kernels[name] = ent
-    # roofline of the dominant kernel: spatial attention, R launches per step.
+    # roofline of the dominant kernel: the spatial / full attention launch.
     # Peak: the burst GEMM figure while the clocks ran free, the sustained one
     # when the power cap throttled them during the timed region.
-    sp_launch_ms = ktimes["spatial"] / (1 if stp.fused_merge else w.R)   # one plain chunk launch
-    achieved = (w.spatial_flops() / w.R) / (sp_launch_ms * 1e-3) / 1e12
+    fl_launch, launch_ms = stp.roofline_launch(ktimes)
+    achieved = fl_launch / (launch_ms * 1e-3) / 1e12
     clocks = clk.summary()
     capped = "sw_power_cap" in clocks.get("reasons", []) and "bf16_tflops_sustained" in pk
     tc_peak = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
     tc_src = f"{pk_src} bf16 " + ("sustained (power cap active)" if capped else "burst")
+    cfg = {"workload": w.name}
+    cfg.update(stp.describe(args))
+    cfg.update({"parallelism": f"replicas{world}",
+                "l2": "flushed between timed steps (256 MiB write, outside the step events)"})
+    if frac_active is not None:
+        cfg["vmajor_active"] = round(frac_active, 4)
     return {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": n_steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "H": w.H, "D": w.D, "P": w.P,
-                   "N_T": w.n_t, "N_S": w.n_s, "kv_chunks": w.R, "vmajor_active": round(frac_active, 4),
-                   "parallelism": f"replicas{world}", "l2": "flushed between timed steps (256 MiB write, "
-                   "outside the step events)", "schedule": args.schedule if args.schedule == "serial" else
-                   f"overlap: {args.slices} shard ranges, attention on {args.att_sms} SMs",
-                   "chunk_merge": "fused into the attention kernel" if stp.fused_merge else "attn_chunk_merge",
-                   "vmajor": "sender side (mask on x, active K/V rows into the caches)" if stp.sender_vmajor else
-                   "receiver side (full relayouts, mask on y, scatter)",
-                   "qk_rope": bool(args.rope)},
+        "config": cfg,
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(statistics.mean(e2e_ms), 5)},
-        "roofline": {"bound": "tensor", "kernel": "st_attn_spatial", "achieved": round(achieved, 2),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_sm100 (st_attn_*)", "achieved": round(achieved, 2),
                      "peak": tc_peak, "peak_source": tc_src, "unit": "TFLOP/s",
-                     "frac": round(achieved / tc_peak, 4), "traffic": kernel_traffic(w.name),
-                     "algorithmic_flop_per_launch": w.spatial_flops() / w.R},
+                     "frac": round(achieved / tc_peak, 4), "frac_of_burst": round(achieved / pk["bf16_tflops"], 4),
+                     "traffic": kernel_traffic(w.name),
+                     "algorithmic_flop_per_launch": fl_launch, "launch_ms": round(launch_ms, 5)},
         "kernels": kernels,
         "gpu_launches": launches * n_steps,
         "device_status": st.st_status_string(status),
         "clocks": clocks,
-        "cpu_baseline": cpu_baseline(w, budget_s=args.cpu_budget) if world == 1 else None,
+        "cpu_baseline": cpu_baseline(w, budget_s=args.cpu_budget) if world == 1 and args.cpu_budget > 0 else None,
     }
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_sample(w, n_frames, n_tokens):
-    """The oracle on a bounded sample of the step: spatial attention of n_frames
-    frames and temporal attention of n_tokens tokens.  Returns (seconds, flop)."""
-    import numpy as np
-    import oracle
-    q, k, v = synth.qkv(w)
-    frames = list(range(n_frames))
-    toks = np.arange(n_tokens)
-    t0 = time.perf_counter()
-    oracle.spatial(q, k, v, frames=frames)
-    oracle.temporal(q, k, v, tokens=toks)
-    dt = time.perf_counter() - t0
-    fl = 4.0 * w.B * n_frames * w.S * w.S * w.C + 4.0 * w.B * n_tokens * w.T * w.T * w.C
-    return dt, fl
+class OracleSample:
+    """The fp64 oracle on a bounded sample of one step of workload ``w``.
+
+    ST-DiT step: spatial attention of whole frames and temporal attention of a
+    set of tokens.  Image step: the attention rows of a set of query tokens
+    (every head, all N keys) on Q and K normalised by the oracle's RMSNorm.
+    V-Major step: the attention rows of a set of query tokens against the K/V
+    caches the oracle's mask, compaction and cache update produce.  The
+    preparation (input generation, RMSNorm of the whole K, mask, cache update,
+    fp64 conversion) happens before any timing; ``run`` times the sampled
+    attention only.
+    """
+
+    def __init__(self, w):
+        import numpy as np
+        import oracle
+        self.w, self.kind = w, step_kind(w)
+        self.np, self.oracle = np, oracle
+        if self.kind == "st":
+            self.q, self.k, self.v = synth.qkv(w)
+            return
+        N, H, D, C = w.S, w.H, w.D, w.C
+        shape = (1, 1, N, H, D)
+        if self.kind == "image":
+            q, k, v = synth.qkv(w)
+            g = synth.rms_gamma(w)
+            self.k = oracle.rmsnorm_heads(k.reshape(N, C), g, D, w.rms_eps).reshape(shape)
+            self.q_raw, self.g = q.reshape(N, C), g
+            self.v = v.to(torch.float64).numpy().reshape(shape)
+        else:
+            q = synth.randn(w, "q", shape)
+            cur_v, prev_v = synth.vmajor_pair(w, N, C)
+            cur_k, prev_k = synth.vmajor_pair(w, N, C, prev="kprev", noise="knoise")
+            tau = json.load(open(os.path.join(ROOT, "tests", "golden", "vmajor_tau.json")))[
+                "workloads"][w.name]["0.5"]["tau"]
+            idx, cnt = oracle.compact(oracle.change_mask(oracle.l1_change(cur_v, prev_v), tau))
+            self.k = oracle.scatter_rows(idx, cnt, cur_k, prev_k).reshape(shape)
+            self.v = oracle.scatter_rows(idx, cnt, cur_v, prev_v).reshape(shape)
+            self.q_raw = q.reshape(N, C)
+
+    def unit_flop(self):
+        """FLOP of one sampled unit: a frame (ST) or a query row (image, V-Major)."""
+        w = self.w
+        if self.kind == "st":
+            return 4.0 * w.B * w.S * w.S * w.C
+        return 4.0 * w.S * w.C
+
+    def full_flop(self):
+        w = self.w
+        return w.spatial_flops() + (w.temporal_flops() if self.kind == "st" else 0.0)
+
+    def run(self, n_units, n_tokens=0):
+        """Times the oracle on n_units frames (ST, plus temporal attention of
+        n_tokens tokens) or n_units query rows.  Returns (seconds, flop)."""
+        np, oracle, w = self.np, self.oracle, self.w
+        if self.kind == "st":
+            t0 = time.perf_counter()
+            oracle.spatial(self.q, self.k, self.v, frames=list(range(n_units)))
+            if n_tokens:
+                oracle.temporal(self.q, self.k, self.v, tokens=np.arange(n_tokens))
+            dt = time.perf_counter() - t0
+            return dt, n_units * self.unit_flop() + 4.0 * w.B * n_tokens * w.T * w.T * w.C
+        N, H, D, C = w.S, w.H, w.D, w.C
+        rows = np.arange(n_units) * max(1, N // max(n_units, 1)) % N
+        t0 = time.perf_counter()
+        for r0 in range(0, len(rows), 64):                   # 64 query rows per call bounds the score matrix
+            sel = rows[r0:r0 + 64]
+            q = self.q_raw[torch.from_numpy(sel)]
+            if self.kind == "image":
+                q = oracle.rmsnorm_heads(q, self.g, D, w.rms_eps)
+            if isinstance(q, torch.Tensor):
+                q = q.to(torch.float64).numpy()
+            q = q.reshape(1, 1, len(sel), H, D)
+            oracle.spatial(q, self.k, self.v, kv=(0, N))     # every query row attends to all N keys
+        dt = time.perf_counter() - t0
+        return dt, len(rows) * self.unit_flop()
 
 
 def cpu_threads():
@@ -636,30 +976,69 @@ def cpu_threads():
         return os.cpu_count()
 
 
+def _fit_units(sample, budget_s, cap, probe, n_tokens=0):
+    """Units of the sample whose timing fills about budget_s seconds."""
+    dt, _ = sample.run(probe, n_tokens)
+    per = max(dt / probe, 1e-4)
+    return max(1, min(cap, int(budget_s / per)))
+
+
 def cpu_baseline(w, budget_s=15.0):
-    dt, fl = oracle_sample(w, 1, 256)
-    n_frames = max(1, min(w.T, int(budget_s / max(dt, 1e-3))))
-    dt, fl = oracle_sample(w, n_frames, 1200)
-    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle: spatial attention of {n_frames} of {w.T} frames (all heads, all "
-                      f"{w.S} queries and keys) + temporal attention of 1200 of {w.S} tokens; {dt:.1f} s"}
+    """The oracle timed on the host cores on a bounded sample of the step (all
+    cores, then one BLAS thread on a smaller sample), with the full-size step
+    time extrapolated linearly from the per-unit time (every unit -- a frame or
+    a query row -- costs the same)."""
+    from threadpoolctl import threadpool_limits
+    smp = OracleSample(w)
+    st_kind = smp.kind == "st"
+    cap = w.T if st_kind else w.S
+    probe = 1 if st_kind else 64
+    n_tok = 1200 if st_kind else 0
+    units = _fit_units(smp, budget_s, cap, probe, n_tok)
+    dt, fl = smp.run(units, n_tok)
+    val = fl / dt / 1e12
+    full_s = smp.full_flop() / (val * 1e12)
+    with threadpool_limits(limits=1):
+        u1 = max(1, min(units, _fit_units(smp, budget_s / 3, cap, 1 if st_kind else 16)))
+        dt1, fl1 = smp.run(u1, 0 if st_kind else 0)
+    val1 = fl1 / dt1 / 1e12
+    what = (f"spatial attention of {units} of {w.T} frames (all heads, all {w.S} queries and keys) + temporal "
+            f"attention of {n_tok} of {w.S} tokens" if st_kind else
+            f"attention rows of {units} of {w.S} query tokens (all {w.H} heads, all {w.S} keys)"
+            + (" on RMS-normalised Q/K" if smp.kind == "image" else " on the oracle-updated K/V caches"))
+    return {"value": round(val, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle: {what}; {dt:.1f} s",
+            "single_thread": {"value": round(val1, 6), "unit": "TFLOP/s", "cores": 1,
+                              "sample": f"{u1} {'frames' if st_kind else 'query rows'}, {dt1:.1f} s"},
+            "extrapolated_full_step_s": {"all_cores": round(full_s, 1),
+                                         "single_thread": round(smp.full_flop() / (val1 * 1e12), 1),
+                                         "note": "extrapolated linearly from the sampled units"}}
 
 
 def run_reference(args, w):
-    dt, fl = oracle_sample(w, 1, 256)
-    n_frames = max(1, min(w.T, int(args.cpu_budget / max(args.steps, 1) / max(dt, 1e-3))))
+    smp = OracleSample(w)
+    st_kind = smp.kind == "st"
+    cap = w.T if st_kind else w.S
+    n_tok = 300 if st_kind else 0
+    units = _fit_units(smp, args.cpu_budget / max(args.steps, 1), cap, 1 if st_kind else 16, n_tok)
+    if not st_kind:
+        units = max(8, units // 8 * 8)
     for _ in range(args.warmup):
-        oracle_sample(w, 1, 64)
+        smp.run(1 if st_kind else 8, 64 if st_kind else 0)
     times, fls = [], []
     for _ in range(args.steps):
-        dt, fl = oracle_sample(w, n_frames, 300)
+        dt, fl = smp.run(units, n_tok)
         times.append(dt)
         fls.append(fl)
     tot = sum(times)
     val = sum(fls) / tot / 1e12
     ms = 1e3 * tot / args.steps
-    sample = (f"fp64 numpy oracle per step: spatial attention of {n_frames} of {w.T} frames (all heads, all "
-              f"{w.S} queries and keys) + temporal attention of 300 of {w.S} tokens")
+    if st_kind:
+        sample = (f"fp64 numpy oracle per step: spatial attention of {units} of {w.T} frames (all heads, all "
+                  f"{w.S} queries and keys) + temporal attention of {n_tok} of {w.S} tokens")
+    else:
+        sample = (f"fp64 numpy oracle per step: attention rows of {units} of {w.S} query tokens (all {w.H} heads, "
+                  f"all {w.S} keys)")
     return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -675,8 +1054,16 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="opensora_low")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--workload", default="image_4096px", choices=sorted(synth.BY_NAME))
+    ap.add_argument("--attn", choices=["ring", "chunks"], default="chunks",
+                    help="image step: ring = one launch over every KV ring chunk (stationary chunk first); "
+                         "chunks = one launch per chunk, later chunks merged inside the attention kernel")
+    ap.add_argument("--vmajor-f", type=float, default=0.5, choices=[0.1, 0.5, 0.9],
+                    help="V-Major step: target active fraction of the golden threshold")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle time for cpu_baseline (0: no cpu_baseline)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="image workload only: run it at this many tokens instead (profiler captures)")
     ap.add_argument("--merge", choices=["fused", "separate"], default="fused",
                     help="fused: KV chunks 1..R-1 merged inside the attention kernel; separate: attn_chunk_merge")
     ap.add_argument("--vmajor", choices=["sender", "receiver"], default="sender",
@@ -692,6 +1079,12 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = synth.BY_NAME[args.workload]
+    if args.tokens:
+        # a smaller instance of the image step (same kernels), for profiler captures
+        if step_kind(w) != "image" or args.tokens % w.P:
+            ap.error("--tokens applies to the image workload and must be a multiple of its P")
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}@N{args.tokens}", S=args.tokens)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     if args.impl == "reference":

@@ -139,6 +139,29 @@ st_status st_attn_spatial_merge(const st_attn_desc *desc, const void *q, const v
                                 const void *v, const float *o_acc, const float *lse_acc,
                                 void *o, float *lse, st_stream_t stream);
 
+/* Full attention over R KV ring chunks in one launch, the chunk-and-merge
+ * scheme of ring / Torus attention [SW Methodology 2; SF "六" RingAttention]
+ * with the merge carried inside the kernel:
+ *   the S keys of each frame are cut into n_chunks chunks, chunk c holding keys
+ *   [floor(c*S/R), floor((c+1)*S/R)).  A block of 256 query rows (one frame,
+ *   one head) attends to its chunks in ring order, starting at the chunk that
+ *   holds its first row -- the stationary chunk a ring rank owns -- and then
+ *   c+1, c+2, ... modulo R, as the other chunks would arrive.  The running row
+ *   max, row sum and unnormalised O are carried from one chunk into the next,
+ *   which is the log-sum-exp merge of attn_chunk_merge applied chunk by chunk
+ *   without writing a partial; the result equals the merge of the R
+ *   per-chunk partials (and full attention over the S keys) up to rounding
+ *   order.
+ *   desc: as st_attn_spatial; kv_begin and kv_end must be 0 (the chunks
+ *     partition the whole frame).  o_fp32 may be set.
+ *   lse: optional fp32 [B, T, H, S], the merged natural-log LSE.
+ *   n_chunks: 1..64 and at most S.  ST_ERR_SHAPE otherwise.
+ *   fp32 Q/K/V run the fp32 FMA kernel over the keys in natural order.
+ *   Other errors as st_attn_spatial.  The pages give no API for this form. */
+st_status st_attn_ring(const st_attn_desc *desc, const void *q, const void *k,
+                       const void *v, void *o, float *lse, int n_chunks,
+                       st_stream_t stream);
+
 /* Temporal attention [SF "三、技术架构"]: for every (b, s, h) in the selected
  * tokens, attention over the T frames of token s.  T <= 64.
  *   lse: optional fp32 [B, S, H, T] dense.
@@ -154,7 +177,9 @@ st_status st_attn_temporal(const st_attn_desc *desc, const void *q, const void *
  *     o_parts[c] is fp32 dense [n_units, S, H, D] (n_units = B*T frames),
  *     lse_parts[c] is fp32 dense [n_units, H, S].
  *   o_out: dense [n_units, S, H, D] in out_dtype.  lse_out: optional
- *   [n_units, H, S].  Rows whose every chunk has lse = -inf get o = 0. */
+ *   [n_units, H, S].  Rows whose every chunk has lse = -inf get o = 0.
+ *   o_out and lse_out must not overlap each other or any part (ST_ERR_SHAPE):
+ *   outputs are written while other threads still read the parts. */
 st_status attn_chunk_merge(int n_chunks, const float *const *o_parts,
                            const float *const *lse_parts, long long n_units, int S,
                            int H, int D, void *o_out, st_dtype out_dtype,
@@ -275,10 +300,17 @@ st_status vmajor_mask_compact(const void *v_cur, const void *v_prev,
  * per-tile counts live in a file-scope device array of 512 KiB that every GPU
  * loading the library keeps until the process exits.
  *   n_tokens above 4,194,304 (1 << 22) returns ST_ERR_SHAPE.
- *   Allocates nothing: no cudaMalloc/cudaFree and no allocating library call.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   Makes no cudaMalloc/cudaFree and no allocating library call.  The first
+ *   call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current.  Under CUDA's lazy
+ *   module loading that lookup may be what loads the library's device code
+ *   on the device, and loading the code allocates its device globals, this
+ *   array among them: make the first call at start-up, before any stream
+ *   capture, and later calls allocate nothing.
+ *   The address is cached per device for the life of the process: do not
+ *   call this entry point again after cudaDeviceReset (or any other teardown
+ *   of the device's context) in the same process -- the cached address would
+ *   no longer belong to the new context.
  *   All calls share the one array (it keeps the last call's contents, and
  *   nothing in it needs to start at zero): calls whose work overlaps on the GPU
  *   (two streams, or two host threads) race and must be serialised by the
@@ -373,6 +405,22 @@ int st_get_sm_budget(void);
  * st_check_device_status(stream) must report ST_ERR_TIMEOUT (and clears the
  * word).  Nothing faults, traps or hangs. */
 st_status st_selftest_wait_timeout(st_stream_t stream);
+
+/* Exponential self test: for each of the n fp32 values x[i] (device), writes
+ * the two base-2 exponentials the attention kernel's softmax uses, evaluated
+ * by the same device functions:
+ *   y_poly[i]: 2^x on the FMA pipe -- range reduction x = j + f with j the
+ *     nearest integer, 2^f from a degree-3 polynomial (coefficients from a
+ *     Remez exchange on relative error over [-1/2, 1/2], maximum relative
+ *     error 7.48e-5 before fp32 rounding), 2^j added into the exponent; x is
+ *     clamped below at -125 and must be <= 8 (the softmax's arguments are
+ *     scores minus a running max that trails the true max by at most 8);
+ *   y_mufu[i]: ex2.approx.ftz.f32 on the special-function unit.
+ * Device pointers, 4-byte aligned; n >= 0.  ST_ERR_NULL / ST_ERR_ALIGN /
+ * ST_ERR_SHAPE on bad arguments.  Not part of the pages' method: it exists so
+ * that the tests can bound the error of the kernel's exponentials. */
+st_status st_selftest_ex2(const float *x, float *y_poly, float *y_mufu, int n,
+                          st_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -6,7 +6,7 @@ asynchronous on ``torch.cuda.current_stream()`` unless a stream is given.
 Importing this module fails loudly when the library has not been built.
 
 Entry points (same names as the C ABI in include/stattn.h):
-    st_attn_spatial, st_attn_spatial_merge, st_attn_temporal, attn_chunk_merge, ulysses_relayout,
+    st_attn_spatial, st_attn_ring, st_attn_spatial_merge, st_attn_temporal, attn_chunk_merge, ulysses_relayout,
     ulysses_relayout_range, vmajor_mask_compact, vmajor_mask_compact_noalloc, vmajor_mask_compact_scatter,
     vmajor_scatter_rows, vmajor_workspace_bytes, vmajor_relayout_mask, vmajor_relayout_rows,
     st_rope_table, ulysses_relayout_rope,
@@ -60,6 +60,7 @@ _c = {
     "st_abi_version": _proto("st_abi_version", c_int),
     "st_attn_spatial": _proto("st_attn_spatial", c_int, ctypes.POINTER(st_attn_desc), _VP, _VP, _VP, _VP, _VP, _VP),
     "st_attn_temporal": _proto("st_attn_temporal", c_int, ctypes.POINTER(st_attn_desc), _VP, _VP, _VP, _VP, _VP, _VP),
+    "st_attn_ring": _proto("st_attn_ring", c_int, ctypes.POINTER(st_attn_desc), _VP, _VP, _VP, _VP, _VP, c_int, _VP),
     "st_attn_spatial_merge": _proto("st_attn_spatial_merge", c_int, ctypes.POINTER(st_attn_desc), _VP, _VP, _VP,
                                     _VP, _VP, _VP, _VP, _VP),
     "attn_chunk_merge": _proto("attn_chunk_merge", c_int, c_int, ctypes.POINTER(_VP), ctypes.POINTER(_VP), c_ll,
@@ -81,6 +82,7 @@ _c = {
                                   ctypes.POINTER(_VP), ctypes.POINTER(_VP), c_int, ctypes.POINTER(_VP), _VP),
     "st_check_device_status": _proto("st_check_device_status", c_int, _VP),
     "st_selftest_wait_timeout": _proto("st_selftest_wait_timeout", c_int, _VP),
+    "st_selftest_ex2": _proto("st_selftest_ex2", c_int, _VP, _VP, _VP, c_int, _VP),
     "st_set_sm_budget": _proto("st_set_sm_budget", c_int, c_int),
     "vmajor_relayout_mask": _proto("vmajor_relayout_mask", c_int, _VP, _VP, _VP, c_int, c_int, c_int, c_int, c_int,
                                    c_int, c_int, c_int, c_float, c_int, _VP, _VP, _VP, _VP, _VP, c_size_t, _VP),
@@ -92,13 +94,14 @@ _c = {
     "st_get_sm_budget": _proto("st_get_sm_budget", c_int),
 }
 
-EXPORTED = ["st_status_string", "st_abi_version", "st_attn_spatial", "st_attn_spatial_merge", "st_attn_temporal",
+EXPORTED = ["st_status_string", "st_abi_version", "st_attn_spatial", "st_attn_ring", "st_attn_spatial_merge",
+            "st_attn_temporal",
             "attn_chunk_merge",
             "ulysses_relayout", "vmajor_workspace_bytes", "vmajor_mask_compact", "vmajor_mask_compact_noalloc",
             "vmajor_scatter_rows", "vmajor_mask_compact_scatter",
             "st_check_device_status", "st_selftest_wait_timeout", "ulysses_relayout_range", "st_set_sm_budget",
             "st_get_sm_budget", "vmajor_relayout_mask", "vmajor_relayout_rows", "st_rope_table",
-            "ulysses_relayout_rope"]
+            "ulysses_relayout_rope", "st_selftest_ex2"]
 
 
 class StattnError(RuntimeError):
@@ -158,6 +161,19 @@ def st_attn_spatial(q, k, v, o, lse=None, *, desc: st_attn_desc | None = None, s
         desc = make_desc(B, T, S, H, D, _dtype_code(q), **kw)
     r = _c["st_attn_spatial"](ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _stream(stream))
     return r if raw else _check(r, "st_attn_spatial")
+
+
+def st_attn_ring(q, k, v, o, lse=None, n_chunks=1, *, desc: st_attn_desc | None = None, stream=None, raw=False,
+                 **kw):
+    """Full attention over ``n_chunks`` KV ring chunks in one launch: each query
+    block starts at the chunk holding its first row and carries its running
+    statistics across the chunks (include/stattn.h)."""
+    if desc is None:
+        B, T, S, H, D = q.shape
+        desc = make_desc(B, T, S, H, D, _dtype_code(q), **kw)
+    r = _c["st_attn_ring"](ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(n_chunks),
+                           _stream(stream))
+    return r if raw else _check(r, "st_attn_ring")
 
 
 def st_attn_spatial_merge(q, k, v, o_acc, lse_acc, o, lse=None, *, desc: st_attn_desc | None = None, stream=None,
@@ -323,3 +339,9 @@ def st_get_sm_budget() -> int:
 
 def st_selftest_wait_timeout(stream=None) -> int:
     return int(_c["st_selftest_wait_timeout"](_stream(stream)))
+
+
+def st_selftest_ex2(x, y_poly, y_mufu, *, stream=None, raw=False):
+    """The softmax's two exp2 implementations evaluated on the fp32 device tensor x."""
+    r = _c["st_selftest_ex2"](_ptr(x), _ptr(y_poly), _ptr(y_mufu), int(x.numel()), _stream(stream))
+    return r if raw else _check(r, "st_selftest_ex2")

@@ -20,7 +20,7 @@ bool strides_aligned(const st::Geom &g, int esize) {
 namespace {
 
 st_status spatial(const st_attn_desc *desc, const void *q, const void *k, const void *v, void *o, float *lse,
-                  const float *o_acc, const float *lse_acc, st_stream_t stream) {
+                  const float *o_acc, const float *lse_acc, st_stream_t stream, int n_chunks = 1, int ring = 0) {
   if (!desc) return ST_ERR_NULL;
   if (!q || !k || !v || !o) return ST_ERR_NULL;
   st::Geom g;
@@ -30,11 +30,15 @@ st_status spatial(const st_attn_desc *desc, const void *q, const void *k, const 
   int kv0 = desc->kv_begin, kv1 = desc->kv_end;
   if (kv0 == 0 && kv1 == 0) kv1 = g.S;
   if (kv0 < 0 || kv1 > g.S || kv0 > kv1) return ST_ERR_SHAPE;
+  if (ring && (desc->kv_begin != 0 || desc->kv_end != 0)) return ST_ERR_SHAPE;
+  if (n_chunks < 1 || n_chunks > 64 || n_chunks > g.S) return ST_ERR_SHAPE;
   const float scale = desc->scale > 0.f ? desc->scale : 1.0f / sqrtf((float)g.D);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (desc->dtype == ST_F32) {
     if (!st::is_aligned(q, 4) || !st::is_aligned(k, 4) || !st::is_aligned(v, 4) || !st::is_aligned(o, 4))
       return ST_ERR_ALIGN;
+    // the fp32 kernel attends the whole range in key order (the same result
+    // as the chunk walk up to rounding order)
     return st::attn_f32(g, false, lo, hi, kv0, kv1, scale, static_cast<const float *>(q),
                         static_cast<const float *>(k), static_cast<const float *>(v), static_cast<float *>(o),
                         lse, st, o_acc, lse_acc);
@@ -51,7 +55,8 @@ st_status spatial(const st_attn_desc *desc, const void *q, const void *k, const 
     g.sblk = g.S;
     g.ssb = (long long)g.S * g.ss;
   }
-  return st::attn_spatial_sm100(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, desc->o_fp32, st, o_acc, lse_acc);
+  return st::attn_spatial_sm100(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, desc->o_fp32, st, o_acc, lse_acc,
+                                n_chunks, ring);
 }
 
 }  // namespace
@@ -59,6 +64,11 @@ st_status spatial(const st_attn_desc *desc, const void *q, const void *k, const 
 ST_API st_status st_attn_spatial(const st_attn_desc *desc, const void *q, const void *k, const void *v, void *o,
                                  float *lse, st_stream_t stream) {
   return spatial(desc, q, k, v, o, lse, nullptr, nullptr, stream);
+}
+
+ST_API st_status st_attn_ring(const st_attn_desc *desc, const void *q, const void *k, const void *v, void *o,
+                              float *lse, int n_chunks, st_stream_t stream) {
+  return spatial(desc, q, k, v, o, lse, nullptr, nullptr, stream, n_chunks, 1);
 }
 
 ST_API st_status st_attn_spatial_merge(const st_attn_desc *desc, const void *q, const void *k, const void *v,

@@ -70,9 +70,12 @@ st_status attn_f32(const Geom &g, bool temporal, int lo, int hi, int kv0, int kv
 st_status attn_temporal_bf16(const Geom &g, int lo, int hi, float scale, const void *q,
                              const void *k, const void *v, void *o, float *lse, int o_f32,
                              cudaStream_t s);
+// n_chunks / ring: the key range cut into n_chunks KV chunks walked in one
+// launch; ring = 1 starts every query block at the chunk holding its first row
+// (key range = the whole frame, no accumulator).
 st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, float scale,
                              const void *q, const void *k, const void *v, void *o, float *lse,
                              int o_f32, cudaStream_t s, const float *o_acc = nullptr,
-                             const float *lse_acc = nullptr);
+                             const float *lse_acc = nullptr, int n_chunks = 1, int ring = 0);
 
 }  // namespace st

@@ -313,6 +313,9 @@ struct Params {
   st::Geom g;
   int lo, n_frames;          // selected frames
   int kv0, kv1;              // key range
+  int n_chunks;              // KV chunks the key range is cut into (1: one range)
+  int ring;                  // 1: every query block starts at the chunk holding its first row
+  int n_kv;                  // 64-key steps per item (over all chunks)
   int q_blocks;              // ceil(S / 256)
   int tmode;                 // 1: frames addressed as (t % tblk, b*T/tblk + t/tblk)
   float scale_log2, scale;
@@ -364,6 +367,42 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
   q = ffma2(q, f, make_float2(kP0, kP0));
   return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// KV chunks: the key range [kv0, kv1) is cut into n_chunks chunks, chunk c
+// starting at key kv0 + floor(c * (kv1 - kv0) / n_chunks).  An item walks its
+// chunks in ring order from a start chunk (the stationary one), each chunk in
+// 64-key steps whose last one may be ragged; the running max, row sum and O
+// carry over from one chunk to the next, which is the log-sum-exp merge of the
+// chunks in unnormalised form.
+__device__ __forceinline__ int chunk_lo(const Params &p, int c) {
+  return p.kv0 + (int)(((long long)c * (p.kv1 - p.kv0)) / p.n_chunks);
+}
+struct KeyWalk {
+  int c, key, end;           // chunk, first key of the step, end of the chunk
+  __device__ __forceinline__ void begin(const Params &p, int c0) {
+    c = c0;
+    key = chunk_lo(p, c0);
+    end = chunk_lo(p, c0 + 1);
+  }
+  __device__ __forceinline__ void next(const Params &p) {
+    key += 64;
+    if (key >= end) {
+      c = c + 1 == p.n_chunks ? 0 : c + 1;
+      key = chunk_lo(p, c);
+      end = chunk_lo(p, c + 1);
+    }
+  }
+};
+// Ring mode (queries and keys are the same sequence): a query block starts at
+// the chunk that holds its first row, as a ring rank starts with its own KV
+// chunk before the others arrive.  Otherwise every item starts at chunk 0.
+__device__ __forceinline__ int start_chunk(const Params &p, int q0) {
+  if (!p.ring) return 0;
+  int c = (int)(((long long)q0 * p.n_chunks) / (p.kv1 - p.kv0));
+  while (c + 1 < p.n_chunks && chunk_lo(p, c + 1) <= q0) ++c;
+  while (c > 0 && chunk_lo(p, c) > q0) --c;
+  return c;
 }
 
 // Work item -> (q block, head, frame); q block fastest so that the CTAs that
@@ -437,7 +476,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const st::Geom &g = p.g;
   const int n_items = p.q_blocks * g.H * p.n_frames * g.B;
-  const int n_kv = (p.kv1 - p.kv0 + BLOCK_N - 1) / BLOCK_N;
+  const int n_kv = p.n_kv;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < QB; ++i) {
@@ -502,10 +541,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_5d(dst, &tq0, q_full + qb, 0, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
             if (K::C1) tma_load_5d(dst + K::QT0, &tq1, q_full + qb, 64, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
           }
-          for (int j = 0; j < n_kv; ++j, ++kv) {
+          KeyWalk kw;
+          kw.begin(p, start_chunk(p, it.q0));
+          for (int j = 0; j < n_kv; ++j, ++kv, kw.next(p)) {
             const int st = kv % NS;
             const uint32_t ph = (kv / NS) & 1;
-            const int key = p.kv0 + j * BLOCK_N;
+            const int key = kw.key;
             if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 1))) break;
             mbar_expect_tx(k_full + st, K::KTILE);
             uint8_t *dk = sK + st * K::KTILE;
@@ -683,7 +724,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Item it = decode(p, x);
       if (X >= it.n_qt) continue;
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_kv; ++j, ++gs) {
+      KeyWalk kw;
+      kw.begin(p, start_chunk(p, it.q0));
+      for (int j = 0; j < n_kv; ++j, ++gs, kw.next(p)) {
         const uint32_t b = gs & 1;
         if (!(ok = mbar_wait(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
         tc_fence_after();
@@ -691,7 +734,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < BLOCK_N / 16; ++c) TMEM_LD16(tS + b * BLOCK_N + c * 16, (sr + c * 16));
         tmem_wait_ld();
-        const int nvalid = p.kv1 - (p.kv0 + j * BLOCK_N);
+        const int nvalid = kw.end - kw.key;
         if (nvalid < BLOCK_N) {
 #pragma unroll
           for (int c = 0; c < BLOCK_N; ++c)
@@ -1046,6 +1089,19 @@ __global__ void wait_timeout_probe(unsigned long long limit_ns, uint32_t epoch) 
   }
 }
 
+// Evaluates the softmax's two exponentials element by element, for the
+// self test of their error: the FMA-pipe polynomial (ex2_poly2) and the MUFU
+// instruction (ex2_mufu), exactly as the softmax calls them.
+__global__ void ex2_probe(const float *__restrict__ x, float *__restrict__ y_poly, float *__restrict__ y_mufu,
+                          int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float a = x[i];
+  const float2 r = ex2_poly2(make_float2(a, a));
+  y_poly[i] = r.x;
+  y_mufu[i] = ex2_mufu(a);
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
@@ -1108,7 +1164,7 @@ std::atomic<uint32_t> g_epoch{0};
 template <int D, bool MERGE>
 st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, float scale, const void *q,
                          const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
-                         const float *o_acc, const float *lse_acc) {
+                         const float *o_acc, const float *lse_acc, int n_chunks, int ring) {
   using K = Cfg<D, MERGE>;
   const int tmode = g.tblk != g.T ? 1 : 0;
   CUtensorMap m[8];
@@ -1130,6 +1186,17 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   p.n_frames = hi - lo;
   p.kv0 = kv0;
   p.kv1 = kv1;
+  p.n_chunks = n_chunks;
+  p.ring = ring;
+  {
+    long long steps = 0;                       // 64-key steps over every chunk
+    for (int c = 0; c < n_chunks; ++c) {
+      const long long a = kv0 + ((long long)c * (kv1 - kv0)) / n_chunks;
+      const long long b = kv0 + ((long long)(c + 1) * (kv1 - kv0)) / n_chunks;
+      steps += (b - a + BLOCK_N - 1) / BLOCK_N;
+    }
+    p.n_kv = int(steps);
+  }
   p.q_blocks = (g.S + 2 * BLOCK_M - 1) / (2 * BLOCK_M);
   p.tmode = tmode;
   p.scale = scale;
@@ -1178,10 +1245,13 @@ unsigned int read_and_clear_attn_error(cudaStream_t stream, cudaError_t *err) {
 
 st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, float scale, const void *q,
                              const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
-                             const float *o_acc, const float *lse_acc) {
+                             const float *o_acc, const float *lse_acc, int n_chunks, int ring) {
   if (hi <= lo) return ST_OK;
+  if (n_chunks < 1 || (n_chunks > 1 && n_chunks > kv1 - kv0) || (ring && (kv0 != 0 || kv1 != g.S || o_acc)))
+    return ST_ERR_SHAPE;
   // merge mode with head dims up to 80 stages the accumulated rows in shared memory
-#define ST_SPATIAL(DD, MM) launch_spatial<DD, MM>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc)
+#define ST_SPATIAL(DD, MM) \
+  launch_spatial<DD, MM>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc, n_chunks, ring)
   const bool staged = o_acc != nullptr;
   switch (g.D) {
     case 32: return staged ? ST_SPATIAL(32, true) : ST_SPATIAL(32, false);
@@ -1196,6 +1266,16 @@ st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, fl
 }
 
 }  // namespace st
+
+ST_API st_status st_selftest_ex2(const float *x, float *y_poly, float *y_mufu, int n, st_stream_t stream) {
+  if (n < 0) return ST_ERR_SHAPE;
+  if (n == 0) return ST_OK;
+  if (!x || !y_poly || !y_mufu) return ST_ERR_NULL;
+  if (!st::is_aligned(x, 4) || !st::is_aligned(y_poly, 4) || !st::is_aligned(y_mufu, 4)) return ST_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ex2_probe<<<(n + 255) / 256, 256, 0, s>>>(x, y_poly, y_mufu, n);
+  return st::launch_status();
+}
 
 ST_API st_status st_selftest_wait_timeout(st_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -168,6 +168,20 @@ ST_API st_status attn_chunk_merge(int n_chunks, const float *const *o_parts, con
   }
   if (!st::is_aligned(o_out, out_dtype == ST_BF16 ? 8 : 16)) return ST_ERR_ALIGN;
   const long long rows_h = n_units * S * (long long)H;
+  {
+    // the outputs are written while other threads (other CTAs) still read
+    // the parts: an output that overlaps any part would corrupt the weights
+    // or the partials of rows not yet merged
+    const long long ob = rows_h * D * (out_dtype == ST_BF16 ? 2 : 4), pb = rows_h * D * 4, lb = rows_h * 4;
+    const char *o0 = static_cast<const char *>(o_out), *l0 = reinterpret_cast<const char *>(lse_out);
+    auto hit = [](const char *a, long long na, const char *b, long long nb) { return a < b + nb && b < a + na; };
+    for (int c = 0; c < n_chunks; ++c) {
+      const char *pc = reinterpret_cast<const char *>(o_parts[c]), *lc = reinterpret_cast<const char *>(lse_parts[c]);
+      if (hit(o0, ob, pc, pb) || hit(o0, ob, lc, lb)) return ST_ERR_SHAPE;
+      if (lse_out && (hit(l0, lb, pc, pb) || hit(l0, lb, lc, lb))) return ST_ERR_SHAPE;
+    }
+    if (lse_out && hit(o0, ob, l0, lb)) return ST_ERR_SHAPE;
+  }
   const long long total = rows_h * (D / 4);
   const long long want = (total + 255) / 256;
   const long long cap = (long long)st::num_sms() * 16;

@@ -767,7 +767,9 @@ constexpr long long kStaticTiles = kStaticMaxTokens / TILE;
 __device__ __align__(256) int g_vmajor_static_counts[kStaticTiles];
 
 // Device address of the array on the current device.  The first call on a
-// device looks it up with that device current and caches it.
+// device looks it up with that device current and caches it for the life of
+// the process (so the entry point must not be used after a cudaDeviceReset of
+// that device: the cached address would belong to the old context).
 int *static_counts_on_current_device() {
   static std::mutex mu;
   static int *addr[64] = {nullptr};

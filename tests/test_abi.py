@@ -131,6 +131,27 @@ def test_attention_rejects(st):
     assert spatial(st, "st_attn_temporal", D=40) == st.ST_ERR_UNSUPPORTED
 
 
+def ring(st, n_chunks, q=FAKE_IN, **kw):
+    d = dict(B=1, T=2, S=64, H=2, D=128, dtype=st.ST_BF16)
+    d.update(kw)
+    desc = st.make_desc(**d)
+    return st._c["st_attn_ring"](ctypes.byref(desc), q, FAKE_IN, FAKE_IN, FAKE_OUT, None, n_chunks, None)
+
+
+def test_ring_attention_rejects(st):
+    """The ring-chunk call validates its chunk count and key range before any launch."""
+    assert st._c["st_attn_ring"](None, FAKE_IN, FAKE_IN, FAKE_IN, FAKE_OUT, None, 2, None) == st.ST_ERR_NULL
+    assert ring(st, 2, q=None) == st.ST_ERR_NULL
+    assert ring(st, 0) == st.ST_ERR_SHAPE
+    assert ring(st, -3) == st.ST_ERR_SHAPE
+    assert ring(st, 65) == st.ST_ERR_SHAPE                       # at most 64 chunks
+    assert ring(st, 9, S=8) == st.ST_ERR_SHAPE                   # more chunks than keys
+    assert ring(st, 2, kv_begin=0, kv_end=32) == st.ST_ERR_SHAPE  # the chunks partition the whole frame
+    assert ring(st, 2, kv_begin=8, kv_end=64) == st.ST_ERR_SHAPE
+    assert ring(st, 2, D=48) == st.ST_ERR_UNSUPPORTED
+    assert ring(st, 2, q=ctypes.c_void_p(0x100008)) == st.ST_ERR_ALIGN
+
+
 def test_merge_and_vmajor_reject(st):
     VP = ctypes.c_void_p
     arr = (VP * 2)(0x100000, 0x200000)
@@ -140,6 +161,13 @@ def test_merge_and_vmajor_reject(st):
     assert f(2, arr, arr, 1, 8, 2, 66, FAKE_OUT, st.ST_BF16, None, None) == st.ST_ERR_ALIGN
     assert f(2, arr, arr, 1, 8, 2, 64, None, st.ST_BF16, None, None) == st.ST_ERR_NULL
     assert f(2, arr, arr, 1, 8, 2, 64, FAKE_OUT, 9, None, None) == st.ST_ERR_DTYPE
+    # outputs overlapping a part (in place, or an LSE over an LSE part) are refused
+    lse = (VP * 2)(0x300000, 0x400000)
+    assert f(2, arr, lse, 1, 8, 2, 64, VP(0x200000), st.ST_F32, None, None) == st.ST_ERR_SHAPE
+    assert f(2, arr, lse, 1, 8, 2, 64, VP(0x100000 + 512), st.ST_BF16, None, None) == st.ST_ERR_SHAPE
+    assert f(2, arr, lse, 1, 8, 2, 64, FAKE_OUT, st.ST_BF16, VP(0x400000), None) == st.ST_ERR_SHAPE
+    assert f(2, arr, lse, 1, 8, 2, 64, FAKE_OUT, st.ST_BF16, VP(0x200000 + 64), None) == st.ST_ERR_SHAPE
+    assert f(2, arr, lse, 1, 8, 2, 64, FAKE_OUT, st.ST_BF16, VP(0x90000000 + 64), None) == st.ST_ERR_SHAPE
     g = st._c["vmajor_mask_compact"]
     ws = st.vmajor_workspace_bytes(100)
     assert g(None, FAKE_IN, 100, 64, st.ST_BF16, 1.0, 0, FAKE_OUT, FAKE_OUT, FAKE_OUT, None, FAKE_OUT, ws, None) == st.ST_ERR_NULL

@@ -4,7 +4,8 @@ vmajor_mask_compact_noalloc exists for callers that may not allocate device
 memory while they run (a serving loop bound to a fixed memory pool, or code
 that cannot risk cudaMalloc stalling or failing in the middle of a step).  It
 keeps its scratch in the library's own static device array, so this test
-calls it twice in a row, on inputs of different sizes, through the C ABI, and
+calls it three times in a row, on inputs of different sizes (smaller, larger,
+smaller), through the C ABI, and
 checks mask, indices, count and per-token L1 against vmajor_mask_compact with a
 caller workspace.  The file sorts last so that a failure here stops a -x run
 only after every other test has run.
@@ -47,7 +48,9 @@ def outputs(n):
 def test_noalloc_matches_workspace_entry_point_twice(st):
     fn = st._c["vmajor_mask_compact_noalloc"]
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for name, f in (("vmajor_2304px", 0.5), ("opensora_low", 0.5)):
+    # smaller, larger, smaller: every call finds in the shared array what a
+    # call of another size left there, and its results must not depend on it
+    for name, f in (("opensora_low", 0.5), ("vmajor_2304px", 0.5), ("opensora_low", 0.5)):
         cur, prev, tau = workload_inputs(name, f)
         n, C = cur.shape
         mask_a, idx_a, cnt_a, l1_a = outputs(n)
