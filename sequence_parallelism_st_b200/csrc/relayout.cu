@@ -396,6 +396,158 @@ st_status launch_rms(const Map &m, const char *in, char *out, const float *gamma
   }
 }
 
+// ---------------------------------------------------------------- sequence <-> head exchange
+// Rows of D elements whose byte length is 8, 16 or 32 vectors of 16 bytes
+// (VPR).  The kernel walks the SEQUENCE side [P, B, N/P, H, D] -- where the H
+// rows of a token are contiguous -- in chunks of 32 * U vectors per warp, in
+// order, so that side is read (SEQ2HEAD) or written (HEAD2SEQ) in long runs;
+// the other side is addressed row by row: row (q, b, h1, n) of the head side
+// is ((q*B + b)*Hp + h1)*N + n.  A warp holds U vectors per lane in flight
+// (all loads before any store).  The VPR lanes holding one row are
+// consecutive (VPR divides 32), so the optional per-head RMSNorm reduces the
+// row's sum of squares with VPR-lane butterfly shuffles; every lane keeps the
+// gains of its own columns in registers.  The index arithmetic per vector is
+// two multiply-shift divisions (by H and by Hp; and by N/P and B when B > 1).
+struct SeqHead {
+  uint32_t N, H, Hp, Np, B;
+  st::FastDiv div_h, div_hp, div_np, div_b;
+  long long n_vecs;          // B * N * H * VPR
+};
+
+template <typename T, int VPR, int U, bool RMS, bool TO_HEAD>
+__global__ void __launch_bounds__(256) seqhead_move(SeqHead m, const char *__restrict__ in, char *__restrict__ out,
+                                                    const float *__restrict__ gamma, float eps) {
+  constexpr int EPV = 16 / int(sizeof(T));
+  constexpr int LOG_VPR = VPR == 8 ? 3 : (VPR == 16 ? 4 : 5);
+  st::pdl_trigger();
+  st::pdl_wait();
+  in = st::after_wait(in);
+  const int lane = threadIdx.x & 31;
+  const int col = lane & (VPR - 1);                  // this lane's 16-byte column of every row it touches
+  float g[EPV];
+  if constexpr (RMS) {
+    gamma = st::after_wait(gamma);
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) g[e] = gamma[col * EPV + e];
+  }
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const long long chunk = 32LL * U;
+  for (long long c0 = warp * chunk; c0 < m.n_vecs; c0 += n_warps * chunk) {
+    uint4 v[U];
+    long long head_off[U];                           // byte offset of the vector on the head side
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long vi = c0 + u * 32 + lane;       // vector index on the sequence side
+      head_off[u] = -1;
+      if (vi < m.n_vecs) {
+        // sequence-side row ((p*B + b)*Np + n1)*H + h holds token n = p*Np + n1, head h
+        const uint32_t row = uint32_t(vi >> LOG_VPR);
+        const uint32_t t = st::fdiv(row, m.div_h);
+        const uint32_t h = row - t * m.H;
+        uint32_t b = 0, n = t;                         // B = 1: t = p*Np + n1 = n
+        if (m.B > 1) {
+          const uint32_t pb = st::fdiv(t, m.div_np);
+          const uint32_t p = st::fdiv(pb, m.div_b);
+          b = pb - p * m.B;
+          n = p * m.Np + (t - pb * m.Np);
+        }
+        const uint32_t q = st::fdiv(h, m.div_hp), h1 = h - q * m.Hp;
+        const long long hrow = ((long long)(q * m.B + b) * m.Hp + h1) * m.N + n;
+        head_off[u] = (hrow * VPR + col) * 16;
+        const char *src = TO_HEAD ? in + vi * 16 : in + head_off[u];
+        v[u] = __ldg(reinterpret_cast<const uint4 *>(src));
+      } else {
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    if constexpr (RMS) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        float ss = 0.f;
+        if constexpr (sizeof(T) == 2) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float a = __uint_as_float(w[k] << 16), c = __uint_as_float(w[k] & 0xffff0000u);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(c, c, ss);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) ss = fmaf(__uint_as_float(w[k]), __uint_as_float(w[k]), ss);
+        }
+#pragma unroll
+        for (int off = VPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float inv = rsqrtf(ss * (1.0f / float(VPR * EPV)) + eps);
+        st::RotVec<T> none;
+        v[u] = st::rms_rope_vec<T, false>(v[u], inv, g, none);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (head_off[u] < 0) continue;
+      const long long vi = c0 + u * 32 + lane;
+      char *dst = TO_HEAD ? out + head_off[u] : out + vi * 16;
+      *reinterpret_cast<uint4 *>(dst) = v[u];
+    }
+  }
+}
+
+template <typename T, int VPR, bool RMS>
+st_status launch_seqhead_v(const SeqHead &m, bool to_head, const char *in, char *out, const float *gamma, float eps,
+                           int sms, cudaStream_t s) {
+  constexpr int U = 8;
+  const long long chunks = (m.n_vecs + 32LL * U - 1) / (32LL * U);
+  const long long want = (chunks + 7) / 8;           // 8 warps per CTA
+  const long long cap = (long long)sms * 8;
+  const int grid = int(want < cap ? want : cap);
+  return to_head ? st::launch_pdl(seqhead_move<T, VPR, U, RMS, true>, grid, 256, 0, s, m, in, out, gamma, eps)
+                 : st::launch_pdl(seqhead_move<T, VPR, U, RMS, false>, grid, 256, 0, s, m, in, out, gamma, eps);
+}
+
+// Returns ST_ERR_UNSUPPORTED when the rows do not fit the kernel (the caller
+// then takes the general segment kernels).
+st_status launch_seqhead(const Map &mp, int B, int elem_bytes, const char *in, char *out, const float *gamma,
+                         float eps, int sms, cudaStream_t s) {
+  const long long rb = mp.row_bytes;
+  const int vpr = int(rb / 16);
+  if (rb % 16 || !(vpr == 8 || vpr == 16 || vpr == 32)) return ST_ERR_UNSUPPORTED;
+  if (!st::is_aligned(in, 16) || !st::is_aligned(out, 16)) return ST_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * mp.N * mp.H;
+  if (rows >= (1LL << 31) || (long long)B * mp.N >= (1LL << 31)) return ST_ERR_UNSUPPORTED;   // 32-bit row maths
+  if (gamma && elem_bytes != 2 && elem_bytes != 4) return ST_ERR_UNSUPPORTED;
+  SeqHead m;
+  m.N = uint32_t(mp.N); m.H = uint32_t(mp.H); m.Hp = uint32_t(mp.Hp); m.Np = uint32_t(mp.Np); m.B = uint32_t(B);
+  m.div_h = st::make_fastdiv(m.H);
+  m.div_hp = st::make_fastdiv(m.Hp);
+  m.div_np = st::make_fastdiv(m.Np);
+  m.div_b = st::make_fastdiv(m.B);
+  m.n_vecs = rows * vpr;
+  const bool to_head = mp.mode == ST_SEQ2HEAD;
+#define ST_SH(TT, V, R) launch_seqhead_v<TT, V, R>(m, to_head, in, out, gamma, eps, sms, s)
+  if (!gamma) {
+    switch (vpr) {
+      case 8: return ST_SH(uint16_t, 8, false);
+      case 16: return ST_SH(uint16_t, 16, false);
+      default: return ST_SH(uint16_t, 32, false);
+    }
+  }
+  if (elem_bytes == 2) {
+    switch (vpr) {
+      case 8: return ST_SH(uint16_t, 8, true);
+      case 16: return ST_SH(uint16_t, 16, true);
+      default: return ST_SH(uint16_t, 32, true);
+    }
+  }
+  switch (vpr) {
+    case 8: return ST_SH(float, 8, true);
+    case 16: return ST_SH(float, 16, true);
+    default: return ST_SH(float, 32, true);
+  }
+#undef ST_SH
+}
+
 template <int VEC>
 st_status launch_copy(const Map &m, const char *in, char *out, int grid, cudaStream_t s) {
   const long long seg_vecs = m.seg_bytes / VEC;
@@ -479,10 +631,18 @@ st_status relayout_impl(st_relayout_mode mode, const void *in, void *out, int el
       if (!st::is_aligned(rope_table, 16)) return ST_ERR_ALIGN;
       rope = reinterpret_cast<const float2 *>(rope_table);
     }
+    if (!rope && (mode == ST_SEQ2HEAD || mode == ST_HEAD2SEQ)) {
+      const st_status r = launch_seqhead(m, B, elem_bytes, src, dst, rms_gamma, rms_eps, sms, s);
+      if (r != ST_ERR_UNSUPPORTED) return r;
+    }
     return elem_bytes == 2 ? launch_rms<uint16_t>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s, rope)
                            : launch_rms<float>(m, src, dst, rms_gamma, rms_head_dim, rms_eps, sms, s, rope);
   }
   if (rope_table) return ST_ERR_NULL;               // the rotation rides on the RMSNorm pass
+  if (mode == ST_SEQ2HEAD || mode == ST_HEAD2SEQ) {
+    const st_status r = launch_seqhead(m, B, elem_bytes, src, dst, nullptr, 0.f, sms, s);
+    if (r != ST_ERR_UNSUPPORTED) return r;
+  }
   // widest vector that divides the row pitch and both base addresses
   int vec = 16;
   while (vec > elem_bytes && (m.row_bytes % vec || !st::is_aligned(in, vec) || !st::is_aligned(out, vec)))
