@@ -78,19 +78,20 @@ def peaks():
     return FALLBACK, "fallback"
 
 
-def kernel_traffic(workload):
-    """DRAM bytes per launch of the spatial kernel from the committed ncu summary,
-    or None when the kernel source changed since the capture or the bench runs
-    another workload than the captured one."""
+def kernel_traffic(workload, launch):
+    """DRAM bytes per launch of the roofline's attention launch from the
+    committed ncu record (profiles/traffic.json: one entry per workload and
+    launch kind), or None when the kernel source changed since the capture or
+    nothing was captured for this workload."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     h = hashlib.sha256(open(SPATIAL_SRC, "rb").read()).hexdigest()[:16]
-    e = d.get("st_attn_spatial", {})
-    if e.get("source_sha") != h or e.get("workload") != workload:
-        return None
-    return e.get("dram_bytes_per_launch")
+    for e in d.get("attn_fwd_sm100", []):
+        if e.get("source_sha") == h and e.get("workload") == workload and e.get("launch") == launch:
+            return e.get("dram_bytes_per_launch")
+    return None
 
 
 class ClockSampler:
@@ -451,6 +452,9 @@ class Step:
     def group_bytes(self, frac_active):
         return kernel_bytes(self.w, frac_active, self.sender_vmajor)
 
+    def roofline_name(self):
+        return "chunk0"
+
     def roofline_launch(self, ktimes):
         """(flop of one launch of the dominant kernel, its mean duration in ms):
         the chunk-0 spatial launch."""
@@ -570,6 +574,9 @@ class ImageStep:
         t = self.w.tensor_bytes()
         return {"relayout_seq2head": 3 * 2 * t, "relayout_head2seq": 2 * t}
 
+    def roofline_name(self):
+        return "ring" if self.attn == "ring" else "chunk0"
+
     def roofline_launch(self, ktimes):
         """The ring launch (all R chunks), or the chunk-0 launch of the chunk chain."""
         sp = self.w.spatial_flops()
@@ -663,6 +670,9 @@ class VMajorStep:
         # V and its previous value read; the active rows of K and V read and written into the caches
         t = self.w.tensor_bytes()
         return {"vmajor": 2 * t + 4 * frac_active * t}
+
+    def roofline_name(self):
+        return "cached_kv"
 
     def roofline_launch(self, ktimes):
         return self.w.spatial_flops(), ktimes["spatial"]
@@ -879,7 +889,7 @@ def run_ours(args, w, rank, world, dev):
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_sm100 (st_attn_*)", "achieved": round(achieved, 2),
                      "peak": tc_peak, "peak_source": tc_src, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_peak, 4), "frac_of_burst": round(achieved / pk["bf16_tflops"], 4),
-                     "traffic": kernel_traffic(w.name),
+                     "traffic": kernel_traffic(w.name, stp.roofline_name()),
                      "algorithmic_flop_per_launch": fl_launch, "launch_ms": round(launch_ms, 5)},
         "kernels": kernels,
         "gpu_launches": launches * n_steps,
@@ -1055,7 +1065,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="image_4096px", choices=sorted(synth.BY_NAME))
-    ap.add_argument("--attn", choices=["ring", "chunks"], default="chunks",
+    ap.add_argument("--attn", choices=["ring", "chunks"], default="ring",
                     help="image step: ring = one launch over every KV ring chunk (stationary chunk first); "
                          "chunks = one launch per chunk, later chunks merged inside the attention kernel")
     ap.add_argument("--vmajor-f", type=float, default=0.5, choices=[0.1, 0.5, 0.9],

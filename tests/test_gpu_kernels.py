@@ -137,7 +137,12 @@ def taus():
 
 
 VM_CASES = [("vmajor_2304px", 0.5), ("vmajor_2304px", 0.1), ("vmajor_2304px", 0.9), ("opensora_low", 0.5),
-            ("tiny", 0.5)]
+            ("video_1080p", 0.5), ("tiny", 0.5)]
+
+
+def l1_sliced(cur, prev, rows=32768):
+    """oracle.l1_change over slices of tokens (bounds the fp64 copies on the host)."""
+    return np.concatenate([oracle.l1_change(cur[a:a + rows], prev[a:a + rows]) for a in range(0, cur.shape[0], rows)])
 
 
 @pytest.mark.parametrize("name,f", VM_CASES)
@@ -145,7 +150,7 @@ def test_vmajor_mask_compact_bit_exact(st, name, f):
     w = synth.BY_NAME[name]
     n, C = w.B * w.T * w.S, w.C
     cur, prev = synth.vmajor_pair(w, n, C)
-    l1 = oracle.l1_change(cur, prev)
+    l1 = l1_sliced(cur, prev)
     tau, margin, _ = oracle.tau_for_fraction(l1, f)
     assert tau == pytest.approx(taus()[name][str(f)]["tau"], rel=1e-12)
     # decision is precision independent: margin above the fp32 summation bound
