@@ -155,7 +155,8 @@ st_status st_attn_spatial_merge(const st_attn_desc *desc, const void *q, const v
  *   desc: as st_attn_spatial; kv_begin and kv_end must be 0 (the chunks
  *     partition the whole frame).  o_fp32 may be set.
  *   lse: optional fp32 [B, T, H, S], the merged natural-log LSE.
- *   n_chunks: 1..64 and at most S.  ST_ERR_SHAPE otherwise.
+ *   n_chunks: 1..64, at most S, and S * n_chunks < 2^32.  ST_ERR_SHAPE
+ *     otherwise.
  *   fp32 Q/K/V run the fp32 FMA kernel over the keys in natural order.
  *   Other errors as st_attn_spatial.  The pages give no API for this form. */
 st_status st_attn_ring(const st_attn_desc *desc, const void *q, const void *k,

@@ -375,8 +375,9 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
 // 64-key steps whose last one may be ragged; the running max, row sum and O
 // carry over from one chunk to the next, which is the log-sum-exp merge of the
 // chunks in unnormalised form.
+// (kv1 - kv0) * n_chunks < 2^32 (the host checks it): 32-bit arithmetic.
 __device__ __forceinline__ int chunk_lo(const Params &p, int c) {
-  return p.kv0 + (int)(((long long)c * (p.kv1 - p.kv0)) / p.n_chunks);
+  return p.kv0 + int((uint32_t(c) * uint32_t(p.kv1 - p.kv0)) / uint32_t(p.n_chunks));
 }
 struct KeyWalk {
   int c, key, end;           // chunk, first key of the step, end of the chunk
@@ -399,7 +400,7 @@ struct KeyWalk {
 // chunk before the others arrive.  Otherwise every item starts at chunk 0.
 __device__ __forceinline__ int start_chunk(const Params &p, int q0) {
   if (!p.ring) return 0;
-  int c = (int)(((long long)q0 * p.n_chunks) / (p.kv1 - p.kv0));
+  int c = int((uint32_t(q0) * uint32_t(p.n_chunks)) / uint32_t(p.kv1 - p.kv0));
   while (c + 1 < p.n_chunks && chunk_lo(p, c + 1) <= q0) ++c;
   while (c > 0 && chunk_lo(p, c) > q0) --c;
   return c;
@@ -434,7 +435,7 @@ __device__ __forceinline__ Item decode(const Params &p, int x) {
   return it;
 }
 
-template <int D, bool MERGE>
+template <int D, bool MERGE, bool RING>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
                    const __grid_constant__ CUtensorMap tk0, const __grid_constant__ CUtensorMap tk1,
@@ -476,7 +477,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const st::Geom &g = p.g;
   const int n_items = p.q_blocks * g.H * p.n_frames * g.B;
-  const int n_kv = p.n_kv;
+  // one key range: ceil((kv1 - kv0) / 64) steps; ring mode: the steps of every chunk
+  const int n_kv = RING ? p.n_kv : (p.kv1 - p.kv0 + BLOCK_N - 1) / BLOCK_N;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < QB; ++i) {
@@ -542,11 +544,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (K::C1) tma_load_5d(dst + K::QT0, &tq1, q_full + qb, 64, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
           }
           KeyWalk kw;
-          kw.begin(p, start_chunk(p, it.q0));
-          for (int j = 0; j < n_kv; ++j, ++kv, kw.next(p)) {
+          if constexpr (RING) kw.begin(p, start_chunk(p, it.q0));
+          for (int j = 0; j < n_kv; ++j, ++kv) {
             const int st = kv % NS;
             const uint32_t ph = (kv / NS) & 1;
-            const int key = kw.key;
+            const int key = RING ? kw.key : p.kv0 + j * BLOCK_N;
+            if constexpr (RING) kw.next(p);
             if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 1))) break;
             mbar_expect_tx(k_full + st, K::KTILE);
             uint8_t *dk = sK + st * K::KTILE;
@@ -725,8 +728,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (X >= it.n_qt) continue;
       float m = -INFINITY, l = 0.f;
       KeyWalk kw;
-      kw.begin(p, start_chunk(p, it.q0));
-      for (int j = 0; j < n_kv; ++j, ++gs, kw.next(p)) {
+      if constexpr (RING) kw.begin(p, start_chunk(p, it.q0));
+      for (int j = 0; j < n_kv; ++j, ++gs) {
         const uint32_t b = gs & 1;
         if (!(ok = mbar_wait(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
         tc_fence_after();
@@ -734,7 +737,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < BLOCK_N / 16; ++c) TMEM_LD16(tS + b * BLOCK_N + c * 16, (sr + c * 16));
         tmem_wait_ld();
-        const int nvalid = kw.end - kw.key;
+        const int nvalid = RING ? kw.end - kw.key : p.kv1 - (p.kv0 + j * BLOCK_N);
+        if constexpr (RING) kw.next(p);
         if (nvalid < BLOCK_N) {
 #pragma unroll
           for (int c = 0; c < BLOCK_N; ++c)
@@ -1161,7 +1165,7 @@ bool make_map(CUtensorMap *m, const void *ptr, const st::Geom &g, int tmode, int
 
 std::atomic<uint32_t> g_epoch{0};
 
-template <int D, bool MERGE>
+template <int D, bool MERGE, bool RING = false>
 st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, float scale, const void *q,
                          const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
                          const float *o_acc, const float *lse_acc, int n_chunks, int ring) {
@@ -1213,7 +1217,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   p.n_items = int(items);
   p.reverse = o_acc != nullptr ? 1 : 0;
   const int ctas = int(items < st::num_sms() ? items : st::num_sms());  // persistent: one CTA per SM
-  auto kern = attn_fwd_sm100<D, MERGE>;
+  auto kern = attn_fwd_sm100<D, MERGE, RING>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM) != cudaSuccess)
     return ST_ERR_CUDA;
   // The register split of the warpgroups (setmaxnreg) assumes the launch
@@ -1249,9 +1253,12 @@ st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, fl
   if (hi <= lo) return ST_OK;
   if (n_chunks < 1 || (n_chunks > 1 && n_chunks > kv1 - kv0) || (ring && (kv0 != 0 || kv1 != g.S || o_acc)))
     return ST_ERR_SHAPE;
+  if ((long long)(kv1 - kv0) * n_chunks >= (1LL << 32)) return ST_ERR_SHAPE;   // chunk edges in 32 bits
   // merge mode with head dims up to 80 stages the accumulated rows in shared memory
 #define ST_SPATIAL(DD, MM) \
-  launch_spatial<DD, MM>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc, n_chunks, ring)
+  (ring ? launch_spatial<DD, false, true>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc, n_chunks, \
+                                         ring)                                                                   \
+        : launch_spatial<DD, MM>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc, n_chunks, ring))
   const bool staged = o_acc != nullptr;
   switch (g.D) {
     case 32: return staged ? ST_SPATIAL(32, true) : ST_SPATIAL(32, false);
