@@ -667,9 +667,10 @@ class VMajorStep:
         return {"spatial": self.w.spatial_flops()}
 
     def group_bytes(self, frac_active):
-        # V and its previous value read; the active rows of K and V read and written into the caches
+        # the least traffic of the work: V and its previous value read, the
+        # active rows of K read, the active rows of K and V written into the caches
         t = self.w.tensor_bytes()
-        return {"vmajor": 2 * t + 4 * frac_active * t}
+        return {"vmajor": 2 * t + 3 * frac_active * t}
 
     def roofline_name(self):
         return "cached_kv"

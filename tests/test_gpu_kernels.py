@@ -216,11 +216,14 @@ def test_vmajor_scatter_rows(st):
         assert np.array_equal(f64(packed[:cnt_ref]), oracle.pack_rows(idx_ref, cnt_ref, cur))
 
 
-@pytest.mark.parametrize("name,f", [("vmajor_2304px", 0.5), ("vmajor_2304px", 0.1), ("opensora_low", 0.5),
-                                    ("tiny", 0.5)])
-def test_vmajor_mask_compact_scatter_fused(st, name, f):
+@pytest.mark.parametrize("name,f,keep", [("vmajor_2304px", 0.5, True), ("vmajor_2304px", 0.1, True),
+                                         ("vmajor_2304px", 0.9, False), ("opensora_low", 0.5, True),
+                                         ("opensora_low", 0.5, False), ("tiny", 0.5, True), ("tiny", 0.5, False)])
+def test_vmajor_mask_compact_scatter_fused(st, name, f, keep):
     """The fused call gives the mask, indices, count and caches of the oracle,
-    and the same bits as vmajor_mask_compact + vmajor_scatter_rows."""
+    and the same bits as vmajor_mask_compact + vmajor_scatter_rows.  keep: V's
+    cache takes rows of the very tensor the mask is taken on (the kernel then
+    writes them from the registers that hold them); otherwise from a copy."""
     w = synth.BY_NAME[name]
     n, C = w.B * w.T * w.S, w.C
     cur_v, prev_v = synth.vmajor_pair(w, n, C)
@@ -237,7 +240,8 @@ def test_vmajor_mask_compact_scatter_fused(st, name, f):
         count = torch.zeros(1, dtype=torch.int32, device=DEV)
         kc, vc = prev_k.to(DEV), prev_v.to(DEV)
         if fused:
-            st.vmajor_mask_compact_scatter(cv, pvd, tau, mask, idx, count, ws, [ck, cv], [kc, vc])
+            st.vmajor_mask_compact_scatter(cv, pvd, tau, mask, idx, count, ws, [ck, cv if keep else cv.clone()],
+                                           [kc, vc])
         else:
             st.vmajor_mask_compact(cv, pvd, tau, mask, idx, count, ws)
             st.vmajor_scatter_rows(idx, count, [ck, cv], [kc, vc])
