@@ -415,7 +415,7 @@ struct SeqHead {
 };
 
 template <typename T, int VPR, int U, bool RMS, bool TO_HEAD>
-__global__ void __launch_bounds__(256) seqhead_move(SeqHead m, const char *__restrict__ in, char *__restrict__ out,
+__global__ void __launch_bounds__(256, RMS ? 3 : 4) seqhead_move(SeqHead m, const char *__restrict__ in, char *__restrict__ out,
                                                     const float *__restrict__ gamma, float eps) {
   constexpr int EPV = 16 / int(sizeof(T));
   constexpr int LOG_VPR = VPR == 8 ? 3 : (VPR == 16 ? 4 : 5);
