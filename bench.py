@@ -171,7 +171,8 @@ class Step:
         self.vprev_y = vprev_y.to(dev)
         self.kcache0, self.vcache0 = kprev_y.to(dev), vprev_y.to(dev)
         self.kc, self.vc = self.kcache0.clone(), self.vcache0.clone()
-        mk = lambda dt=torch.bfloat16: torch.empty(n * C, dtype=dt, device=dev)
+        self.dt = st.ST_F32 if w.dtype == "f32" else st.ST_BF16       # the workload's element type
+        mk = lambda dt=w.torch_dtype: torch.empty(n * C, dtype=dt, device=dev)
         self.qy, self.ky, self.vy, self.oy, self.ox, self.ot = mk(), mk(), mk(), mk(), mk(), mk()
         self.parts = [torch.empty(n * C, dtype=torch.float32, device=dev) for _ in range(w.R)]
         self.lses = [torch.empty(n * H, dtype=torch.float32, device=dev) for _ in range(w.R)]
@@ -181,7 +182,7 @@ class Step:
         self.ws = torch.empty(max(16, st.vmajor_workspace_bytes(n)), dtype=torch.uint8, device=dev)
         # y layout with T/(N_T P) = 1: frames (q, i) of S contiguous tokens -> dense [1, T, S, H, D]
         assert T % (w.n_t * P) == 0 and T // (w.n_t * P) == 1
-        self.sdesc = [st.make_desc(1, T, S, H, D, st.ST_BF16, kv_begin=c * S // w.R, kv_end=(c + 1) * S // w.R,
+        self.sdesc = [st.make_desc(1, T, S, H, D, self.dt, kv_begin=c * S // w.R, kv_end=(c + 1) * S // w.R,
                                    o_fp32=1) for c in range(w.R)]
         # sender-side V-Major: the mask is taken on x and only active K/V rows move
         # (into the caches); receiver side: full relayouts, mask on y, scatter
@@ -192,10 +193,10 @@ class Step:
         # fused merge: chunk c >= 1 is merged into the accumulated fp32 partial
         # inside the attention kernel; the last chunk writes the bf16 result
         self.fused_merge = True
-        self.sdesc_last = st.make_desc(1, T, S, H, D, st.ST_BF16, kv_begin=(w.R - 1) * S // w.R, kv_end=S,
+        self.sdesc_last = st.make_desc(1, T, S, H, D, self.dt, kv_begin=(w.R - 1) * S // w.R, kv_end=S,
                                        o_fp32=0)
         Tb, Sb = T // w.n_t, S // (w.n_s * P)
-        self.tdesc = st.make_desc(P * B, T, S // P, H, D, st.ST_BF16, stride_b=w.n_t * w.n_s * Tb * Sb * C,
+        self.tdesc = st.make_desc(P * B, T, S // P, H, D, self.dt, stride_b=w.n_t * w.n_s * Tb * Sb * C,
                                   stride_t=Sb * C, stride_s=C, t_block=Tb, stride_tb=w.n_s * Tb * Sb * C,
                                   s_block=Sb, stride_sb=Tb * Sb * C)
         # per-kernel timing events (launching stream = torch's current stream)
@@ -320,10 +321,10 @@ class Step:
         n_sl_tok = self.n // n_slices
         self.counts = torch.zeros(n_slices, dtype=torch.int32, device=self.dev)
         T = w.T
-        self.sdesc_sl = [[self.st.make_desc(1, T, w.S, w.H, w.D, self.st.ST_BF16, kv_begin=c * w.S // w.R,
+        self.sdesc_sl = [[self.st.make_desc(1, T, w.S, w.H, w.D, self.dt, kv_begin=c * w.S // w.R,
                                             kv_end=(c + 1) * w.S // w.R, o_fp32=1, n_slices=n_slices, slice=i)
                           for c in range(w.R)] for i in range(n_slices)]
-        self.sdesc_last_sl = [self.st.make_desc(1, T, w.S, w.H, w.D, self.st.ST_BF16,
+        self.sdesc_last_sl = [self.st.make_desc(1, T, w.S, w.H, w.D, self.dt,
                                                 kv_begin=(w.R - 1) * w.S // w.R, kv_end=w.S, o_fp32=0,
                                                 n_slices=n_slices, slice=i) for i in range(n_slices)]
         self.n_sl_tok = n_sl_tok
