@@ -84,7 +84,7 @@ constexpr int EPI_BUF = 32 * EPI_COLS * 4;   // bytes of one staging buffer (32 
 // TMEM columns: per tile two S buffers of BLOCK_N fp32 columns, then O.
 constexpr int TM_O = 256;                    // O(tile X) at TM_O + X * 128
 
-template <int D, bool MERGE = false> struct Cfg {
+template <int D, bool MERGE = false, bool QTMEM = false> struct Cfg {
   static constexpr int C0 = D >= 64 ? 64 : 32;
   static constexpr int R1 = D > 64 ? D - 64 : 0;
   static constexpr int C1 = R1 == 0 ? 0 : (R1 <= 16 ? 16 : (R1 <= 32 ? 32 : 64));
@@ -103,6 +103,17 @@ template <int D, bool MERGE = false> struct Cfg {
   // softmax need not add up its exponentials.  (Only when O fits one register
   // group of the epilogue, which reads the sum before normalising.)
   static constexpr bool ONES = DPV > D && (D + 15) / 16 <= 5;
+  // With QTMEM (head dims up to 80; chosen for items of at least 24 key
+  // steps) Q lives in TMEM, in the columns of the tile's O region that O does
+  // not use (DPV + DP / 2 <= 128): S = Q K^T is then a TS product that reads
+  // only K from shared memory (2 KB per MMA at N = 64 instead of 6 KB), which
+  // relieves the shared-memory bandwidth both tiles' S products and PV share.
+  // The epilogue warps move each item's Q there from the TMA-loaded shared
+  // tiles once the tile's last S of the previous item is done; on short items
+  // that hand-over shows at every item boundary, hence the choice.
+  static constexpr bool QTM = QTMEM && D <= 80;
+  static constexpr int QCOL = DPV;                    // Q columns at TM_O + X * 128 + QCOL
+  static_assert(!QTM || DPV + DP / 2 <= 128, "Q beside O in TMEM");
   // Merge mode (the accumulated partial of earlier KV chunks is merged into
   // the result in the epilogue): for head dims up to 80 the epilogue stages
   // the accumulated rows of one tile in shared memory (one 32 x 16 fp32 block
@@ -286,6 +297,11 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint3
                  "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),       \
                  "r"(r[14]), "r"(r[15])                                                                 \
                : "memory")
+#define TMEM_ST8(taddr, r)                                                                               \
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"                       \
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),  \
+                 "r"(r[7])                                                                              \
+               : "memory")
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -435,14 +451,14 @@ __device__ __forceinline__ Item decode(const Params &p, int x) {
   return it;
 }
 
-template <int D, bool MERGE, bool RING>
+template <int D, bool MERGE, bool RING, bool QTMEM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
                    const __grid_constant__ CUtensorMap tk0, const __grid_constant__ CUtensorMap tk1,
                    const __grid_constant__ CUtensorMap tv0, const __grid_constant__ CUtensorMap tv1,
                    const __grid_constant__ CUtensorMap to, const __grid_constant__ CUtensorMap tacc,
                    const Params p) {
-  using K = Cfg<D, MERGE>;
+  using K = Cfg<D, MERGE, QTMEM>;
   constexpr int NS = K::NS, QB = K::QB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -472,7 +488,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *stat_empty = stat_full + 2;        // 2, 128 arrivals (epilogue threads)
   uint64_t *v_ready = stat_empty + 2;          // NS: ones column written into the V stage
   uint64_t *acc_full = v_ready + NS;           // [epilogue warp][tile]: the item's accumulated rows landed
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 8);
+  // Q in TMEM (head dims up to 80), per tile: every S of the item done (its Q
+  // columns may take the next item's Q), Q of the item in TMEM (128 arrivals
+  // of the epilogue threads that moved it)
+  uint64_t *s_done = acc_full + 8;             // 2
+  uint64_t *qt_full = s_done + 2;              // 2
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qt_full + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const st::Geom &g = p.g;
@@ -483,7 +504,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < QB; ++i) {
       mbar_init(q_full + i, 1);
-      mbar_init(q_empty + i, 2);
+      mbar_init(q_empty + i, K::QTM ? BLOCK_M : 2);   // with Q in TMEM: the epilogue threads that moved it
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(k_full + i, 1);
@@ -505,6 +526,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(stat_empty + i, BLOCK_M);
     }
     for (int i = 0; i < 8; ++i) mbar_init(acc_full + i, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_done + i, 1);
+      mbar_init(qt_full + i, BLOCK_M);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == W_S0) {
@@ -592,7 +617,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++c) {
         const Item it = decode(p, x);
         const int qb = c % QB;
-        if (!(ok = mbar_wait(q_full + qb, (c / QB) & 1, epoch, 3))) break;
+        // the item's Q: in shared memory, or (head dims up to 80) moved into TMEM by the epilogue
+        if (!(ok = K::QTM ? mbar_wait(qt_full + X, c & 1, epoch, 3) : mbar_wait(q_full + qb, (c / QB) & 1, epoch, 3)))
+          break;
         if (X >= it.n_qt) {
           // tile absent from this item: release the shared K stages and Q in step
           for (int j = 0; j < n_kv && ok; ++j) {
@@ -601,11 +628,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_arrive(k_empty + g0 % NS);
           }
           if (!ok) break;
-          mbar_arrive(q_empty + qb);
+          if (K::QTM) mbar_arrive(s_done + X);
+          else mbar_arrive(q_empty + qb);
           kv += n_kv;
           continue;
         }
         const uint32_t qa = aQ + (qb * 2 + X) * K::QTILE;
+        const uint32_t qt = tmem + TM_O + X * 128 + K::QCOL;   // Q in TMEM: K-slice kk at columns 8 kk
         for (int j = 0; j < n_kv && ok; ++j, ++step) {
           const uint32_t g0 = kv + j;
           const int st = g0 % NS;
@@ -617,19 +646,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t d = tmem + X * 2 * BLOCK_N + b * BLOCK_N;
           const uint32_t ka = aK + st * K::KTILE;
   #pragma unroll
-          for (int kk = 0; kk < K::C0 / 16; ++kk)
-            mma_ss(d, sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(qa + kk * 32),
-                   sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(ka + kk * 32), IDS, kk > 0);
+          for (int kk = 0; kk < K::C0 / 16; ++kk) {
+            if constexpr (K::QTM)
+              mma_ts(d, qt + kk * 8, sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(ka + kk * 32), IDS, kk > 0);
+            else
+              mma_ss(d, sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(qa + kk * 32),
+                     sdesc_c<16, 8 * K::SW0, layout_of(K::SW0)>(ka + kk * 32), IDS, kk > 0);
+          }
           if (K::C1) {
   #pragma unroll
-            for (int kk = 0; kk < (K::C1 ? K::C1 : 16) / 16; ++kk)
-              mma_ss(d, sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(qa + K::QT0 + kk * 32),
-                     sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(ka + K::KT0 + kk * 32),
-                     IDS, 1);
+            for (int kk = 0; kk < (K::C1 ? K::C1 : 16) / 16; ++kk) {
+              if constexpr (K::QTM)
+                mma_ts(d, qt + K::C0 / 2 + kk * 8,
+                       sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(ka + K::KT0 + kk * 32),
+                       IDS, 1);
+              else
+                mma_ss(d, sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(qa + K::QT0 + kk * 32),
+                       sdesc_c<16, 8 * (K::SW1 ? K::SW1 : 32), layout_of(K::SW1 ? K::SW1 : 32)>(ka + K::KT0 + kk * 32),
+                       IDS, 1);
+            }
           }
           tc_commit(s_full + 2 * X + b);
           tc_commit(k_empty + st);
-          if (j + 1 == n_kv) tc_commit(q_empty + qb);   // last S of this item issued
+          // last S of this item issued: its Q (shared tiles, or the TMEM columns) may be replaced
+          if (j + 1 == n_kv) tc_commit(K::QTM ? s_done + X : q_empty + qb);
         }
         kv += n_kv;
       }
@@ -853,7 +893,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     acc_pending[XX] = true;                                                                                  \
     acc_par[XX] = ((XX) ? oc1 : oc0) & 1; /* items of the tile so far = the phase of these copies */        \
   }
-    for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x) {
+    // Q in TMEM (head dims up to 80): the epilogue warps move each item's Q
+    // rows (lane = row, this warp's quadrant of 32 rows) from the swizzled
+    // shared tiles the TMA loaded into the tile's Q columns beside O -- for
+    // item c + 1 as soon as the tile's last S of item c is done, before item
+    // c's O is read out -- and then release the shared tiles to the loader.
+    auto move_q = [&](int c) -> bool {
+      const int qb = c % QB;
+      if (!mbar_wait(q_full + qb, (c / QB) & 1, epoch, 24)) return false;
+      const int row = qd * 32 + lane;
+      for (int X = 0; X < 2; ++X) {
+        if (c > 0 && !mbar_wait(s_done + X, (c - 1) & 1, epoch, 25 + X)) return false;
+        tc_fence_after();
+        const uint8_t *tile = sQ + (qb * 2 + X) * K::QTILE;
+        const uint32_t tq = tmem + lane_off + TM_O + X * 128 + K::QCOL;
+        // the 16-byte chunks of one row of a part, un-swizzled: 128-byte rows
+        // swizzle chunk f to f ^ (r & 7), 64-byte rows to f ^ ((r >> 1) & 3),
+        // 32-byte rows to f ^ ((r >> 2) & 1); every 16 bytes are 4 columns
+        auto part = [&](const uint8_t *base, int row_bytes, uint32_t col) {
+          const uint8_t *src = base + row * row_bytes;
+          const int sw = row_bytes == 128 ? (row & 7) : (row_bytes == 64 ? ((row >> 1) & 3) : ((row >> 2) & 1));
+          for (int f0 = 0; f0 < row_bytes / 16; f0 += 4) {
+            uint32_t v[16];
+            const int nf = row_bytes / 16 - f0 < 4 ? row_bytes / 16 - f0 : 4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (i < nf) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(src + (((f0 + i) ^ sw) << 4));
+                v[4 * i] = w.x;
+                v[4 * i + 1] = w.y;
+                v[4 * i + 2] = w.z;
+                v[4 * i + 3] = w.w;
+              }
+            }
+            if (nf == 4) TMEM_ST16(tq + col + f0 * 4, v);
+            else TMEM_ST8(tq + col + f0 * 4, v);            // a 32-byte part: 8 columns
+          }
+        };
+        part(tile, K::SW0, 0);
+        if (K::C1) part(tile + K::QT0, K::SW1 ? K::SW1 : 32, K::C0 / 2);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(qt_full + X);
+      }
+      mbar_arrive(q_empty + qb);
+      return true;
+    };
+    if (K::QTM && n_kv > 0 && (int)blockIdx.x < n_items) ok = move_q(0);
+    int citem = 0;                             // items of this CTA so far
+    for (int x = blockIdx.x; x < n_items && ok; x += gridDim.x, ++citem) {
       const Item it = decode(p, x);
       float la_t[2] = {-INFINITY, -INFINITY};  // merge mode: accumulated LSE of this lane's row per tile
       if ((MERGE || K::NCH > 5) && p.o_acc && n_kv > 0) {
@@ -872,6 +960,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      // the next item's Q goes into TMEM once this item's S products are done
+      // (after the accumulated rows above were requested, so those copies run
+      // during this item's steps)
+      if (K::QTM && n_kv > 0 && x + (int)gridDim.x < n_items && !(ok = move_q(citem + 1))) break;
       for (int X = 0; X < it.n_qt && ok; ++X) {
         const int r = qd * 32 + lane;
         const int qrow = it.q0 + X * BLOCK_M + r;
@@ -1165,11 +1257,11 @@ bool make_map(CUtensorMap *m, const void *ptr, const st::Geom &g, int tmode, int
 
 std::atomic<uint32_t> g_epoch{0};
 
-template <int D, bool MERGE, bool RING = false>
+template <int D, bool MERGE, bool RING = false, bool QTMEM = false>
 st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, float scale, const void *q,
                          const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
                          const float *o_acc, const float *lse_acc, int n_chunks, int ring) {
-  using K = Cfg<D, MERGE>;
+  using K = Cfg<D, MERGE, QTMEM>;
   const int tmode = g.tblk != g.T ? 1 : 0;
   CUtensorMap m[8];
   const int c1 = K::C1 ? K::C1 : 16;
@@ -1217,7 +1309,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   p.n_items = int(items);
   p.reverse = o_acc != nullptr ? 1 : 0;
   const int ctas = int(items < st::num_sms() ? items : st::num_sms());  // persistent: one CTA per SM
-  auto kern = attn_fwd_sm100<D, MERGE, RING>;
+  auto kern = attn_fwd_sm100<D, MERGE, RING, QTMEM>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM) != cudaSuccess)
     return ST_ERR_CUDA;
   // The register split of the warpgroups (setmaxnreg) assumes the launch
@@ -1254,19 +1346,34 @@ st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, fl
   if (n_chunks < 1 || (n_chunks > 1 && n_chunks > kv1 - kv0) || (ring && (kv0 != 0 || kv1 != g.S || o_acc)))
     return ST_ERR_SHAPE;
   if ((long long)(kv1 - kv0) * n_chunks >= (1LL << 32)) return ST_ERR_SHAPE;   // chunk edges in 32 bits
+  // 64-key steps per item: head dims 72 and 80 keep Q in TMEM when an item
+  // has at least 24 of them (the per-item hand-over of Q costs more than the
+  // shared-memory bandwidth it frees on shorter items)
+  long long steps = 0;
+  for (int c = 0; c < n_chunks; ++c) {
+    const long long a = kv0 + ((long long)c * (kv1 - kv0)) / n_chunks;
+    const long long b = kv0 + ((long long)(c + 1) * (kv1 - kv0)) / n_chunks;
+    steps += (b - a + BLOCK_N - 1) / BLOCK_N;
+  }
+  const bool qtm = steps >= 24;
   // merge mode with head dims up to 80 stages the accumulated rows in shared memory
-#define ST_SPATIAL(DD, MM) \
-  (ring ? launch_spatial<DD, false, true>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc, n_chunks, \
-                                         ring)                                                                   \
-        : launch_spatial<DD, MM>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc, n_chunks, ring))
+#define ST_SPATIAL(DD, MM, QQ)                                                                                   \
+  (ring ? launch_spatial<DD, false, true, QQ>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc, \
+                                             n_chunks, ring)                                                     \
+        : launch_spatial<DD, MM, false, QQ>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc,  \
+                                           n_chunks, ring))
   const bool staged = o_acc != nullptr;
   switch (g.D) {
-    case 32: return staged ? ST_SPATIAL(32, true) : ST_SPATIAL(32, false);
-    case 64: return staged ? ST_SPATIAL(64, true) : ST_SPATIAL(64, false);
-    case 72: return staged ? ST_SPATIAL(72, true) : ST_SPATIAL(72, false);
-    case 80: return staged ? ST_SPATIAL(80, true) : ST_SPATIAL(80, false);
-    case 96: return ST_SPATIAL(96, false);
-    case 128: return ST_SPATIAL(128, false);
+    case 32: return staged ? ST_SPATIAL(32, true, false) : ST_SPATIAL(32, false, false);
+    case 64: return staged ? ST_SPATIAL(64, true, false) : ST_SPATIAL(64, false, false);
+    case 72:
+      if (qtm) return staged ? ST_SPATIAL(72, true, true) : ST_SPATIAL(72, false, true);
+      return staged ? ST_SPATIAL(72, true, false) : ST_SPATIAL(72, false, false);
+    case 80:
+      if (qtm) return staged ? ST_SPATIAL(80, true, true) : ST_SPATIAL(80, false, true);
+      return staged ? ST_SPATIAL(80, true, false) : ST_SPATIAL(80, false, false);
+    case 96: return ST_SPATIAL(96, false, false);
+    case 128: return ST_SPATIAL(128, false, false);
   }
 #undef ST_SPATIAL
   return ST_ERR_UNSUPPORTED;

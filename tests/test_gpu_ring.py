@@ -35,7 +35,8 @@ def ring(st, q, k, v, R, o_fp32=0):
 
 
 CASES = [(1, 2, 700, 2, 72, 3), (1, 1, 1030, 2, 128, 8), (2, 1, 513, 1, 64, 5), (1, 3, 390, 2, 96, 4),
-         (1, 1, 260, 3, 80, 7), (1, 2, 333, 2, 32, 2), (1, 1, 2048, 2, 128, 8), (1, 1, 130, 1, 128, 64)]
+         (1, 1, 260, 3, 80, 7), (1, 2, 333, 2, 32, 2), (1, 1, 2048, 2, 128, 8), (1, 1, 130, 1, 128, 64),
+         (1, 1, 1800, 2, 72, 3), (1, 2, 1700, 1, 80, 5)]          # >= 24 steps per item: Q in TMEM
 
 
 @pytest.mark.parametrize("B,T,S,H,D,R", CASES)

@@ -37,7 +37,9 @@ def run(st, q, k, v, o_fp32=0, lse=True, **kw):
 
 
 SMALL = [(1, 2, 128, 2, 64), (1, 2, 200, 2, 72), (1, 1, 256, 3, 128), (2, 1, 300, 2, 128), (1, 1, 513, 1, 72),
-         (1, 3, 77, 2, 32), (1, 1, 260, 2, 80), (1, 1, 390, 2, 96), (1, 1, 1030, 1, 128)]
+         (1, 3, 77, 2, 32), (1, 1, 260, 2, 80), (1, 1, 390, 2, 96), (1, 1, 1030, 1, 128),
+         # 24 or more 64-key steps per item: head dims 72 and 80 keep Q in TMEM (last query block: one tile)
+         (1, 2, 1600, 2, 72), (2, 1, 1540, 1, 80), (1, 1, 1537, 3, 72)]
 
 
 @pytest.mark.parametrize("B,T,S,H,D", SMALL)

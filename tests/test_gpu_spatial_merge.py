@@ -129,3 +129,18 @@ def test_fused_merge_opensora_sampled(st):
     ro, rl = oracle.spatial(q, k, v, frames=frames)
     assert_close(out.cpu()[:, frames], ro, "bf16", "opensora fused merge")
     assert_lse_close(lout.cpu()[:, frames], rl, "opensora fused merge lse")
+
+
+@pytest.mark.parametrize("D,S,edges", [(72, 3300, [0, 1540, 1541, 3300]), (80, 3100, [0, 1600, 3100])])
+def test_fused_merge_long_chunks_q_in_tmem(st, D, S, edges):
+    """Chunks of 24 or more 64-key steps take the kernel that keeps Q in TMEM
+    (head dims 72 and 80), also in merge mode; the last query block of each
+    frame leaves the second tile empty."""
+    w = synth.Workload("m", 23, B=1, T=1, S=S, H=2, D=D, dtype="bf16")
+    q, k, v = synth.qkv(w)
+    out, lout = chain(st, q.to(DEV), k.to(DEV), v.to(DEV), edges, torch.bfloat16)
+    rows = np.sort(np.random.default_rng(D).choice(S, 300, replace=False))
+    ro, rl = oracle.spatial(q, k, v, rows=rows)
+    r = torch.from_numpy(rows)
+    assert_close(out.cpu()[:, :, r], ro, "bf16", f"long chunks D={D}")
+    assert_lse_close(lout.cpu()[:, :, :, r], rl, f"long chunks lse D={D}")
