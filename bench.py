@@ -47,7 +47,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import sys
@@ -697,10 +696,6 @@ def step_kind(w):
     if w.T == 1:
         return "image"
     return "st"
-
-
-def flops(w):
-    return w.spatial_flops() + w.temporal_flops()
 
 
 def kernel_bytes(w, frac_active, sender=False):
