@@ -23,11 +23,16 @@ batch of seeded synthetic inputs.  ``--workload`` picks the block:
      (vmajor_mask_compact, vmajor_scatter_rows) instead;
   2. all-to-all S->T of Q with the fused per-head RMSNorm (ulysses_relayout);
   3. spatial attention of the fresh Q against the cached K/V in R KV chunks
-     and their log-sum-exp merge: chunk 0 writes the fp32 partial and its LSE
-     (st_attn_spatial), every later chunk merges into it inside the attention
-     kernel and the last one writes the bf16 result (st_attn_spatial_merge);
-     ``--merge separate`` writes R partials and merges them with
-     attn_chunk_merge instead;
+     and their log-sum-exp merge: either all R chunks in one launch
+     (``--attn ring``, st_attn_ring: each query block from its own chunk, the
+     running statistics carried across the chunks) or ``--attn chunks``:
+     chunk 0 writes
+     the fp32 partial and its LSE (st_attn_spatial), every later chunk merges
+     into it inside the attention kernel and the last one writes the result
+     (st_attn_spatial_merge); ``--merge separate`` writes R partials and
+     merges them with attn_chunk_merge instead; the default (auto) takes the
+     ring when a chunk holds under 24 key steps of 64 and the chain otherwise,
+     the faster of the two on each workload as measured;
   4. all-to-all T->S of the spatial output;
   5. temporal attention over the T frames of every token, read in place from
      the spatially sharded slice layout (st_attn_temporal).
@@ -192,6 +197,10 @@ class Step:
         # fused merge: chunk c >= 1 is merged into the accumulated fp32 partial
         # inside the attention kernel; the last chunk writes the bf16 result
         self.fused_merge = True
+        # ring: the R chunks in one launch (each query block from its own
+        # chunk, the running statistics carried across chunks, no partial)
+        self.ring = False
+        self.rdesc = st.make_desc(1, T, S, H, D, self.dt)
         self.sdesc_last = st.make_desc(1, T, S, H, D, self.dt, kv_begin=(w.R - 1) * S // w.R, kv_end=S,
                                        o_fp32=0)
         Tb, Sb = T // w.n_t, S // (w.n_s * P)
@@ -259,7 +268,11 @@ class Step:
             st.vmajor_scatter_rows(self.idx, self.count, [self.ky.view(self.n, C), self.vy.view(self.n, C)],
                                    [self.kc.view(self.n, C), self.vc.view(self.n, C)])
             self._mark("vmajor", False)
-        if self.fused_merge:
+        if self.ring:
+            self._mark("spatial", True)
+            st.st_attn_ring(self.qy, self.kc, self.vc, self.oy, self.lses[0], w.R, desc=self.rdesc)
+            self._mark("spatial", False)
+        elif self.fused_merge:
             self._spatial_fused(None)
         else:
             self._mark("spatial", True)
@@ -439,12 +452,15 @@ class Step:
         if hasattr(self, "n_sl"):
             return (3 + 3 + w.R + (1 if self.fused_merge else 2)) * self.n_sl + 1
         # sender-side V-Major: V mask-relayout, compaction and K rows (3) replace 2 relayouts + 3 V-Major launches
-        return LAUNCHES_PER_STEP_BASE + w.R - (1 if self.fused_merge else 0) - (2 if self.sender_vmajor else 0)
+        spatial = 1 if self.ring else w.R - (1 if self.fused_merge else 0)
+        return LAUNCHES_PER_STEP_BASE + spatial - (2 if self.sender_vmajor else 0)
 
     def group_flops(self):
         """Attention FLOP of each timed kernel group (the tensor-bound ones)."""
         w, R = self.w, self.w.R
         sp = w.spatial_flops()
+        if self.ring:
+            return {"spatial": sp, "temporal": w.temporal_flops()}
         if self.fused_merge:
             return {"spatial": sp / R, "spatial_merge": sp * (R - 1) / R, "temporal": w.temporal_flops()}
         return {"spatial": sp, "temporal": w.temporal_flops()}
@@ -453,12 +469,14 @@ class Step:
         return kernel_bytes(self.w, frac_active, self.sender_vmajor)
 
     def roofline_name(self):
-        return "chunk0"
+        return "ring" if self.ring else "chunk0"
 
     def roofline_launch(self, ktimes):
         """(flop of one launch of the dominant kernel, its mean duration in ms):
-        the chunk-0 spatial launch."""
+        the ring launch, or the chunk-0 spatial launch of the chunk chain."""
         w = self.w
+        if self.ring:
+            return w.spatial_flops(), ktimes["spatial"]
         return w.spatial_flops() / w.R, ktimes["spatial"] / (1 if self.fused_merge else w.R)
 
     def describe(self, args):
@@ -467,7 +485,9 @@ class Step:
                 "kv_chunks": w.R,
                 "schedule": "serial" if not hasattr(self, "n_sl") else
                 f"overlap: {self.n_sl} shard ranges, attention on {self.att_sms} SMs",
-                "chunk_merge": "fused into the attention kernel" if self.fused_merge else "attn_chunk_merge",
+                "chunk_merge": ("one launch, stationary chunk first, running (m, l, O) carried across chunks"
+                                if self.ring else "fused into the attention kernel" if self.fused_merge
+                                else "attn_chunk_merge"),
                 "vmajor": "sender side (mask on x, active K/V rows into the caches)" if self.sender_vmajor else
                 "receiver side (full relayouts, mask on y, scatter)",
                 "qk_rope": self.rope_table is not None}
@@ -732,14 +752,24 @@ def whole_job_value(world, flop_per_replica_step, ms_per_step):
     return world * flop_per_replica_step / (ms_per_step * 1e-3) / 1e12
 
 
+def ring_pays(w):
+    """ST-DiT spatial chunks: one ring launch beats the chunk chain when a
+    chunk is short (opensora_low, 600 keys: the chain pays a second fill and
+    the fp32 partial's round trip on items of 10 steps, ~11% of the step); on
+    long chunks (video_1080p, 4080 keys) the chain measured ~1% faster."""
+    return -(-(w.S // w.R) // 64) < 24
+
+
 def make_step(st, args, w, dev):
     kind = step_kind(w)
     if kind == "image":
-        return ImageStep(st, w, dev, attn=args.attn)
+        return ImageStep(st, w, dev, attn="chunks" if args.attn == "chunks" else "ring")
     if kind == "vmajor":
         return VMajorStep(st, w, dev, frac=args.vmajor_f)
     stp = Step(st, w, dev)
     stp.fused_merge = args.merge == "fused"
+    ring = args.attn == "ring" or (args.attn == "auto" and ring_pays(w))
+    stp.ring = ring and args.merge == "fused" and args.schedule == "serial"
     stp.sender_vmajor = args.vmajor == "sender"
     if args.rope:
         stp.rope_table = st.st_rope_table(w.S, w.D, 10000.0, device=dev)
@@ -1062,9 +1092,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="image_4096px", choices=sorted(synth.BY_NAME))
-    ap.add_argument("--attn", choices=["ring", "chunks"], default="ring",
-                    help="image step: ring = one launch over every KV ring chunk (stationary chunk first); "
-                         "chunks = one launch per chunk, later chunks merged inside the attention kernel")
+    ap.add_argument("--attn", choices=["auto", "ring", "chunks"], default="auto",
+                    help="ring = one launch over every KV chunk (each query block from its own chunk); "
+                         "chunks = one launch per chunk, later chunks merged inside the attention kernel "
+                         "(--merge separate: attn_chunk_merge); auto = the faster of the two as measured: "
+                         "ring for the image step and for ST-DiT chunks under 24 key steps, else chunks")
     ap.add_argument("--vmajor-f", type=float, default=0.5, choices=[0.1, 0.5, 0.9],
                     help="V-Major step: target active fraction of the golden threshold")
     ap.add_argument("--cpu-budget", type=float, default=15.0,

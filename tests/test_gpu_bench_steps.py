@@ -106,15 +106,18 @@ def ibits(t):
     return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
 
 
-@pytest.mark.parametrize("name", ["tiny", "opensora_low", "video_1080p"])
-def test_st_step_against_oracle(st, name):
-    """Sender-side V-Major -> S->T of Q (+RMSNorm) -> two KV chunks with the
-    fused merge -> T->S -> temporal attention, against the oracle composition
+@pytest.mark.parametrize("name,ring", [("tiny", False), ("tiny", True), ("opensora_low", False),
+                                       ("opensora_low", True), ("video_1080p", False), ("video_1080p", True)])
+def test_st_step_against_oracle(st, name, ring):
+    """Sender-side V-Major -> S->T of Q (+RMSNorm) -> two KV chunks (one ring
+    launch, or the chain with the fused merge) -> T->S -> temporal attention,
+    against the oracle composition
     (mask, indices, count and the V cache bit-exact; the K cache's moved rows,
     the spatial output and the temporal output at the float bar)."""
     bench = bench_mod()
     w = synth.BY_NAME[name]
     stp = bench.Step(st, w, "cuda")
+    stp.ring = ring                                            # R chunks in one launch, or the chunk chain
     stp.reset_caches()
     stp.run()
     torch.cuda.synchronize()
