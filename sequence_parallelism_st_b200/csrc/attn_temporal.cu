@@ -89,10 +89,12 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
   constexpr int KF = D / 16;      // full k16 steps over D
   constexpr int TILE = TP * RS;   // elements of one Q, K or V tile
   extern __shared__ __align__(16) uint16_t smem[];
-  long long *ftab = reinterpret_cast<long long *>(smem + STAGES * 3 * TILE);   // [B * T] frame offsets
+  // frame offsets of batch 0 (batch b adds b * sb): T entries, so that four
+  // single-stage CTAs still fit in an SM whatever B is
+  long long *ftab = reinterpret_cast<long long *>(smem + STAGES * 3 * TILE);
   const int T = g.T;
   st::pdl_trigger();
-  for (int i = threadIdx.x; i < g.B * T; i += blockDim.x) ftab[i] = g.frame(i / T, i % T);
+  for (int i = threadIdx.x; i < T; i += blockDim.x) ftab[i] = g.frame(0, i);
   // rows past T are never loaded: zero them once in every tile
   for (int i = threadIdx.x; i < STAGES * 3 * (TP - T) * RS; i += blockDim.x) {
     const int tile = i / ((TP - T) * RS), r = i - tile * (TP - T) * RS;
@@ -110,8 +112,8 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
     const int s = lo + (item / n_hg) % n_sel;
     const int b = item / (n_hg * n_sel);
     const int heads_here = min(G, g.H - hg * G);
-    const long long tok = g.token(s) + (long long)hg * G * D;
-    const long long *fb = ftab + b * T;
+    const long long tok = g.token(s) + b * g.sb + (long long)hg * G * D;
+    const long long *fb = ftab;
     uint16_t *st_base = smem + stage * 3 * TILE;
     // a thread owns a (tensor, 16-byte column) pair and walks the T frames:
     // one shared-table read, one add and one copy per 16 bytes
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
     const int s = lo + (item / n_hg) % n_sel;
     const int b = item / (n_hg * n_sel);
     const int heads_here = min(G, g.H - hg * G);
-    const long long tok = g.token(s) + (long long)hg * G * D;
+    const long long tok = g.token(s) + b * g.sb + (long long)hg * G * D;
     uint16_t *sQ = smem + stage * 3 * TILE;
     uint16_t *sK = sQ + TILE;
     uint16_t *sV = sK + TILE;
@@ -250,10 +252,10 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
 #pragma unroll
           for (int n = 0; n < DT; ++n) {
             if (r0 < T)
-              *reinterpret_cast<float2 *>(of + ftab[b * T + r0] + tok + warp * D + n * 8 + 2 * cq) =
+              *reinterpret_cast<float2 *>(of + ftab[r0] + tok + warp * D + n * 8 + 2 * cq) =
                   make_float2(oc[n][0] * i0, oc[n][1] * i0);
             if (r1 < T)
-              *reinterpret_cast<float2 *>(of + ftab[b * T + r1] + tok + warp * D + n * 8 + 2 * cq) =
+              *reinterpret_cast<float2 *>(of + ftab[r1] + tok + warp * D + n * 8 + 2 * cq) =
                   make_float2(oc[n][2] * i1, oc[n][3] * i1);
           }
           (void)h;
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
     __syncthreads();
     if (!o_f32) {
       uint16_t *ob = static_cast<uint16_t *>(o);
-      const long long *fb = ftab + b * T;
+      const long long *fb = ftab;
       for (int i = threadIdx.x; i < T * CH; i += blockDim.x) {
         const int t = i / CH;
         const int c = i - t * CH;
@@ -293,10 +295,9 @@ st_status launch_t(const st::Geom &g, int lo, int n_sel, float scale, const void
   const int n_hg = (g.H + G - 1) / G;
   const long long items = (long long)g.B * n_sel * n_hg;
   if (items > 0x7fffffffLL) return ST_ERR_SHAPE;
-  if ((long long)g.B * g.T > 4096) return ST_ERR_UNSUPPORTED;  // frame table in shared memory
   constexpr size_t stage_bytes = size_t(3) * TP * (G * D + 8) * sizeof(uint16_t);
   constexpr int STAGES = 2 * stage_bytes <= 64 * 1024 ? 2 : 1;
-  const size_t smem = STAGES * stage_bytes + size_t(g.B) * g.T * sizeof(long long);
+  const size_t smem = STAGES * stage_bytes + size_t(g.T) * sizeof(long long);
   auto kern = temporal_bf16<D, TP, STAGES>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return ST_ERR_CUDA;
