@@ -1030,7 +1030,7 @@ def cpu_baseline(w, budget_s=15.0):
     st_kind = smp.kind == "st"
     cap = w.T if st_kind else w.S
     probe = 1 if st_kind else 64
-    n_tok = 1200 if st_kind else 0
+    n_tok = min(1200, w.S) if st_kind else 0       # tokens of the temporal sample (a frame's worth at most)
     units = _fit_units(smp, budget_s, cap, probe, n_tok)
     dt, fl = smp.run(units, n_tok)
     val = fl / dt / 1e12
@@ -1056,12 +1056,12 @@ def run_reference(args, w):
     smp = OracleSample(w)
     st_kind = smp.kind == "st"
     cap = w.T if st_kind else w.S
-    n_tok = 300 if st_kind else 0
+    n_tok = min(300, w.S) if st_kind else 0
     units = _fit_units(smp, args.cpu_budget / max(args.steps, 1), cap, 1 if st_kind else 16, n_tok)
     if not st_kind:
         units = max(8, units // 8 * 8)
     for _ in range(args.warmup):
-        smp.run(1 if st_kind else 8, 64 if st_kind else 0)
+        smp.run(1 if st_kind else 8, min(64, w.S) if st_kind else 0)
     times, fls = [], []
     for _ in range(args.steps):
         dt, fl = smp.run(units, n_tok)

@@ -65,3 +65,17 @@ def test_whole_job_value_counts_every_replica():
     assert bench.whole_job_value(8, f, 0.36) == pytest.approx(8 * one)
     # the max-over-ranks time decides: a slower rank lowers the job's value
     assert bench.whole_job_value(2, f, 0.40) < bench.whole_job_value(2, f, 0.36)
+
+
+@pytest.mark.parametrize("name", ["tiny", "opensora_low"])
+def test_oracle_arm_samples_fit_the_workload(name):
+    """The timed oracle samples (cpu_baseline and the reference arm) stay
+    inside the workload: the temporal sample takes at most a frame's tokens,
+    so a frame smaller than the default sample (tiny: 64 tokens) still runs."""
+    import argparse
+    import synth
+    w = synth.BY_NAME[name]
+    cb = bench.cpu_baseline(w, budget_s=0.2)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["single_thread"]["value"] > 0
+    line = bench.run_reference(argparse.Namespace(cpu_budget=0.2, steps=1, warmup=3), w)
+    assert line["impl"] == "reference" and line["value"] > 0
