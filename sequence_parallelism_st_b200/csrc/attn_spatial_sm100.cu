@@ -330,6 +330,7 @@ struct Params {
   int lo, n_frames;          // selected frames
   int kv0, kv1;              // key range
   int n_chunks;              // KV chunks the key range is cut into (1: one range)
+  int cs[65];                // chunk c starts at key cs[c]; cs[n_chunks] = kv1 (host-computed)
   int ring;                  // 1: every query block starts at the chunk holding its first row
   int n_kv;                  // 64-key steps per item (over all chunks)
   int q_blocks;              // ceil(S / 256)
@@ -391,10 +392,9 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
 // 64-key steps whose last one may be ragged; the running max, row sum and O
 // carry over from one chunk to the next, which is the log-sum-exp merge of the
 // chunks in unnormalised form.
-// (kv1 - kv0) * n_chunks < 2^32 (the host checks it): 32-bit arithmetic.
-__device__ __forceinline__ int chunk_lo(const Params &p, int c) {
-  return p.kv0 + int((uint32_t(c) * uint32_t(p.kv1 - p.kv0)) / uint32_t(p.n_chunks));
-}
+// The host computes the chunk edges once per launch (a table in the kernel
+// parameters), so the walk does no division.
+__device__ __forceinline__ int chunk_lo(const Params &p, int c) { return p.cs[c]; }
 struct KeyWalk {
   int c, key, end;           // chunk, first key of the step, end of the chunk
   __device__ __forceinline__ void begin(const Params &p, int c0) {
@@ -416,6 +416,8 @@ struct KeyWalk {
 // chunk before the others arrive.  Otherwise every item starts at chunk 0.
 __device__ __forceinline__ int start_chunk(const Params &p, int q0) {
   if (!p.ring) return 0;
+  // a first guess, then corrected against the edges; 32-bit arithmetic since
+  // q0 * n_chunks < S * n_chunks < 2^32 (the host checks it)
   int c = int((uint32_t(q0) * uint32_t(p.n_chunks)) / uint32_t(p.kv1 - p.kv0));
   while (c + 1 < p.n_chunks && chunk_lo(p, c + 1) <= q0) ++c;
   while (c > 0 && chunk_lo(p, c) > q0) --c;
@@ -451,13 +453,17 @@ __device__ __forceinline__ Item decode(const Params &p, int x) {
   return it;
 }
 
-template <int D, bool MERGE, bool RING, bool QTMEM>
+// RING: 0 = one key range; 1 = KV chunks walked in ring order (KeyWalk, the
+// last step of a chunk may be ragged); 2 = the same walk when every chunk is a
+// whole number of 64-key steps: a rotation of the one-range walk with no
+// ragged step, so the softmax needs no key bookkeeping at all.
+template <int D, bool MERGE, int RING, bool QTMEM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
                    const __grid_constant__ CUtensorMap tk0, const __grid_constant__ CUtensorMap tk1,
                    const __grid_constant__ CUtensorMap tv0, const __grid_constant__ CUtensorMap tv1,
                    const __grid_constant__ CUtensorMap to, const __grid_constant__ CUtensorMap tacc,
-                   const Params p) {
+                   const __grid_constant__ Params p) {
   using K = Cfg<D, MERGE, QTMEM>;
   constexpr int NS = K::NS, QB = K::QB;
   extern __shared__ uint8_t smem_raw[];
@@ -569,12 +575,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (K::C1) tma_load_5d(dst + K::QT0, &tq1, q_full + qb, 64, it.h, it.q0 + X * BLOCK_M, it.c3, it.c4);
           }
           KeyWalk kw;
-          if constexpr (RING) kw.begin(p, start_chunk(p, it.q0));
+          if constexpr (RING == 1) kw.begin(p, start_chunk(p, it.q0));
+          int rot = 0;                                  // RING == 2: the step's index in the one-range walk
+          if constexpr (RING == 2) rot = (chunk_lo(p, start_chunk(p, it.q0)) - p.kv0) / BLOCK_N;
           for (int j = 0; j < n_kv; ++j, ++kv) {
             const int st = kv % NS;
             const uint32_t ph = (kv / NS) & 1;
-            const int key = RING ? kw.key : p.kv0 + j * BLOCK_N;
-            if constexpr (RING) kw.next(p);
+            const int key = RING == 1 ? kw.key : p.kv0 + (RING == 2 ? rot : j) * BLOCK_N;
+            if constexpr (RING == 1) kw.next(p);
+            if constexpr (RING == 2) rot = rot + 1 == n_kv ? 0 : rot + 1;
             if (!(ok = mbar_wait(k_empty + st, ph ^ 1, epoch, 1))) break;
             mbar_expect_tx(k_full + st, K::KTILE);
             uint8_t *dk = sK + st * K::KTILE;
@@ -768,7 +777,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (X >= it.n_qt) continue;
       float m = -INFINITY, l = 0.f;
       KeyWalk kw;
-      if constexpr (RING) kw.begin(p, start_chunk(p, it.q0));
+      if constexpr (RING == 1) kw.begin(p, start_chunk(p, it.q0));
       for (int j = 0; j < n_kv; ++j, ++gs) {
         const uint32_t b = gs & 1;
         if (!(ok = mbar_wait(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
@@ -777,8 +786,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < BLOCK_N / 16; ++c) TMEM_LD16(tS + b * BLOCK_N + c * 16, (sr + c * 16));
         tmem_wait_ld();
-        const int nvalid = RING ? kw.end - kw.key : p.kv1 - (p.kv0 + j * BLOCK_N);
-        if constexpr (RING) kw.next(p);
+        const int nvalid = RING == 2 ? BLOCK_N : (RING == 1 ? kw.end - kw.key : p.kv1 - (p.kv0 + j * BLOCK_N));
+        if constexpr (RING == 1) kw.next(p);
         if (nvalid < BLOCK_N) {
 #pragma unroll
           for (int c = 0; c < BLOCK_N; ++c)
@@ -1257,7 +1266,7 @@ bool make_map(CUtensorMap *m, const void *ptr, const st::Geom &g, int tmode, int
 
 std::atomic<uint32_t> g_epoch{0};
 
-template <int D, bool MERGE, bool RING = false, bool QTMEM = false>
+template <int D, bool MERGE, int RING = 0, bool QTMEM = false>
 st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, float scale, const void *q,
                          const void *k, const void *v, void *o, float *lse, int o_f32, cudaStream_t s,
                          const float *o_acc, const float *lse_acc, int n_chunks, int ring) {
@@ -1285,12 +1294,10 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   p.n_chunks = n_chunks;
   p.ring = ring;
   {
+    if (n_chunks < 1 || n_chunks > 64) return ST_ERR_SHAPE;
     long long steps = 0;                       // 64-key steps over every chunk
-    for (int c = 0; c < n_chunks; ++c) {
-      const long long a = kv0 + ((long long)c * (kv1 - kv0)) / n_chunks;
-      const long long b = kv0 + ((long long)(c + 1) * (kv1 - kv0)) / n_chunks;
-      steps += (b - a + BLOCK_N - 1) / BLOCK_N;
-    }
+    for (int c = 0; c <= n_chunks; ++c) p.cs[c] = int(kv0 + ((long long)c * (kv1 - kv0)) / n_chunks);
+    for (int c = 0; c < n_chunks; ++c) steps += (p.cs[c + 1] - p.cs[c] + BLOCK_N - 1) / BLOCK_N;
     p.n_kv = int(steps);
   }
   p.q_blocks = (g.S + 2 * BLOCK_M - 1) / (2 * BLOCK_M);
@@ -1350,18 +1357,22 @@ st_status attn_spatial_sm100(const Geom &g, int lo, int hi, int kv0, int kv1, fl
   // has at least 24 of them (the per-item hand-over of Q costs more than the
   // shared-memory bandwidth it frees on shorter items)
   long long steps = 0;
+  bool aligned = true;                         // every chunk a whole number of 64-key steps
   for (int c = 0; c < n_chunks; ++c) {
     const long long a = kv0 + ((long long)c * (kv1 - kv0)) / n_chunks;
     const long long b = kv0 + ((long long)(c + 1) * (kv1 - kv0)) / n_chunks;
     steps += (b - a + BLOCK_N - 1) / BLOCK_N;
+    aligned = aligned && (b - a) % BLOCK_N == 0;
   }
   const bool qtm = steps >= 24;
   // merge mode with head dims up to 80 stages the accumulated rows in shared memory
 #define ST_SPATIAL(DD, MM, QQ)                                                                                   \
-  (ring ? launch_spatial<DD, false, true, QQ>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc, \
-                                             n_chunks, ring)                                                     \
-        : launch_spatial<DD, MM, false, QQ>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc,  \
-                                           n_chunks, ring))
+  (ring ? (aligned ? launch_spatial<DD, false, 2, QQ>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc,   \
+                                                     lse_acc, n_chunks, ring)                                   \
+                   : launch_spatial<DD, false, 1, QQ>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc,   \
+                                                     lse_acc, n_chunks, ring))                                  \
+        : launch_spatial<DD, MM, 0, QQ>(g, lo, hi, kv0, kv1, scale, q, k, v, o, lse, o_f32, s, o_acc, lse_acc,      \
+                                        n_chunks, ring))
   const bool staged = o_acc != nullptr;
   switch (g.D) {
     case 32: return staged ? ST_SPATIAL(32, true, false) : ST_SPATIAL(32, false, false);

@@ -1,8 +1,8 @@
 """GPU parity of st_attn_ring, full attention over R KV ring chunks walked in
 one launch (each query block from its own chunk onwards, the running row
 statistics carried across the chunk boundaries), against the fp64 oracle:
-ragged chunks and ragged query tiles, every supported head dim, one chunk
-(bit-equal to the plain call), the chunk-by-chunk merge chain, and the
+ragged chunks and ragged query tiles, chunks of whole 64-key steps, every
+supported head dim, one chunk (bit-equal to the plain call), the chunk-by-chunk merge chain, and the
 image-DiT 4096px shape on sampled rows."""
 import numpy as np
 import pytest
@@ -36,7 +36,10 @@ def ring(st, q, k, v, R, o_fp32=0):
 
 CASES = [(1, 2, 700, 2, 72, 3), (1, 1, 1030, 2, 128, 8), (2, 1, 513, 1, 64, 5), (1, 3, 390, 2, 96, 4),
          (1, 1, 260, 3, 80, 7), (1, 2, 333, 2, 32, 2), (1, 1, 2048, 2, 128, 8), (1, 1, 130, 1, 128, 64),
-         (1, 1, 1800, 2, 72, 3), (1, 2, 1700, 1, 80, 5)]          # >= 24 steps per item: Q in TMEM
+         (1, 1, 1800, 2, 72, 3), (1, 2, 1700, 1, 80, 5),          # >= 24 steps per item: Q in TMEM
+         # every chunk a whole number of 64-key steps (the walk is a rotation of the one-range walk)
+         (1, 2, 1536, 2, 72, 3), (2, 1, 512, 2, 64, 2), (1, 1, 768, 2, 96, 3), (1, 1, 640, 2, 80, 5),
+         (1, 1, 1024, 2, 128, 16), (1, 1, 4096, 1, 128, 8)]
 
 
 @pytest.mark.parametrize("B,T,S,H,D,R", CASES)
@@ -66,9 +69,11 @@ def test_ring_equals_merge_of_chunk_partials(st):
     assert_lse_close(L.cpu(), ml, "ring lse vs merged")
 
 
-def test_ring_one_chunk_is_the_plain_call(st):
-    """R = 1 walks the same keys in the same order as st_attn_spatial: same bits."""
-    w = synth.Workload("r", 23, B=1, T=2, S=777, H=2, D=128, dtype="bf16")
+@pytest.mark.parametrize("S", [777, 768])
+def test_ring_one_chunk_is_the_plain_call(st, S):
+    """R = 1 walks the same keys in the same order as st_attn_spatial: same
+    bits (a ragged last step, and whole 64-key steps only)."""
+    w = synth.Workload("r", 23, B=1, T=2, S=S, H=2, D=128, dtype="bf16")
     q, k, v = (x.to(DEV) for x in synth.qkv(w))
     o1, L1 = ring(st, q, k, v, 1)
     o2 = torch.empty_like(q)
