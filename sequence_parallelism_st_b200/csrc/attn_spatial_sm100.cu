@@ -331,6 +331,8 @@ struct Params {
   int kv0, kv1;              // key range
   int n_chunks;              // KV chunks the key range is cut into (1: one range)
   int cs[65];                // chunk c starts at key cs[c]; cs[n_chunks] = kv1 (host-computed)
+  int nst[64];               // 64-key steps of chunk c
+  int tail[64];              // keys in the last step of chunk c
   int ring;                  // 1: every query block starts at the chunk holding its first row
   int n_kv;                  // 64-key steps per item (over all chunks)
   int q_blocks;              // ceil(S / 256)
@@ -776,8 +778,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Item it = decode(p, x);
       if (X >= it.n_qt) continue;
       float m = -INFINITY, l = 0.f;
-      KeyWalk kw;
-      if constexpr (RING == 1) kw.begin(p, start_chunk(p, it.q0));
+      // RING == 1: the chunk whose last (possibly ragged) step comes next, and
+      // that step's index in the item's walk
+      int rc = 0, jr = 0;
+      if constexpr (RING == 1) {
+        rc = start_chunk(p, it.q0);
+        jr = p.nst[rc] - 1;
+      }
       for (int j = 0; j < n_kv; ++j, ++gs) {
         const uint32_t b = gs & 1;
         if (!(ok = mbar_wait(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
@@ -786,8 +793,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < BLOCK_N / 16; ++c) TMEM_LD16(tS + b * BLOCK_N + c * 16, (sr + c * 16));
         tmem_wait_ld();
-        const int nvalid = RING == 2 ? BLOCK_N : (RING == 1 ? kw.end - kw.key : p.kv1 - (p.kv0 + j * BLOCK_N));
-        if constexpr (RING == 1) kw.next(p);
+        int nvalid = BLOCK_N;
+        if constexpr (RING == 1) {
+          if (j == jr) {                       // a chunk's last step: mask past its end, go to the next chunk
+            nvalid = p.tail[rc];
+            rc = rc + 1 == p.n_chunks ? 0 : rc + 1;
+            jr += p.nst[rc];
+          }
+        } else if constexpr (RING == 0) {
+          nvalid = p.kv1 - (p.kv0 + j * BLOCK_N);
+        }
         if (nvalid < BLOCK_N) {
 #pragma unroll
           for (int c = 0; c < BLOCK_N; ++c)
@@ -1297,7 +1312,11 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
     if (n_chunks < 1 || n_chunks > 64) return ST_ERR_SHAPE;
     long long steps = 0;                       // 64-key steps over every chunk
     for (int c = 0; c <= n_chunks; ++c) p.cs[c] = int(kv0 + ((long long)c * (kv1 - kv0)) / n_chunks);
-    for (int c = 0; c < n_chunks; ++c) steps += (p.cs[c + 1] - p.cs[c] + BLOCK_N - 1) / BLOCK_N;
+    for (int c = 0; c < n_chunks; ++c) {
+      p.nst[c] = (p.cs[c + 1] - p.cs[c] + BLOCK_N - 1) / BLOCK_N;
+      p.tail[c] = p.cs[c + 1] - p.cs[c] - (p.nst[c] - 1) * BLOCK_N;
+      steps += p.nst[c];
+    }
     p.n_kv = int(steps);
   }
   p.q_blocks = (g.S + 2 * BLOCK_M - 1) / (2 * BLOCK_M);
