@@ -23,16 +23,14 @@ batch of seeded synthetic inputs.  ``--workload`` picks the block:
      (vmajor_mask_compact, vmajor_scatter_rows) instead;
   2. all-to-all S->T of Q with the fused per-head RMSNorm (ulysses_relayout);
   3. spatial attention of the fresh Q against the cached K/V in R KV chunks
-     and their log-sum-exp merge: either all R chunks in one launch
-     (``--attn ring``, st_attn_ring: each query block from its own chunk, the
-     running statistics carried across the chunks) or ``--attn chunks``:
-     chunk 0 writes
-     the fp32 partial and its LSE (st_attn_spatial), every later chunk merges
-     into it inside the attention kernel and the last one writes the result
-     (st_attn_spatial_merge); ``--merge separate`` writes R partials and
-     merges them with attn_chunk_merge instead; the default (auto) takes the
-     ring when a chunk holds under 24 key steps of 64 and the chain otherwise,
-     the faster of the two on each workload as measured;
+     and their log-sum-exp merge: by default all R chunks in one launch
+     (st_attn_ring: each query block from its own chunk, the running
+     statistics carried across the chunks); ``--attn chunks``, ``--merge
+     separate`` or ``--schedule overlap`` take the chain instead: chunk 0
+     writes the fp32 partial and its LSE (st_attn_spatial), every later chunk
+     merges into it inside the attention kernel and the last one writes the
+     result (st_attn_spatial_merge), or with ``--merge separate`` writes R
+     partials merged by attn_chunk_merge;
   4. all-to-all T->S of the spatial output;
   5. temporal attention over the T frames of every token, read in place from
      the spatially sharded slice layout (st_attn_temporal).
@@ -752,14 +750,6 @@ def whole_job_value(world, flop_per_replica_step, ms_per_step):
     return world * flop_per_replica_step / (ms_per_step * 1e-3) / 1e12
 
 
-def ring_pays(w):
-    """ST-DiT spatial chunks: one ring launch beats the chunk chain when a
-    chunk is short (opensora_low, 600 keys: the chain pays a second fill and
-    the fp32 partial's round trip on items of 10 steps, ~11% of the step); on
-    long chunks (video_1080p, 4080 keys) the chain measured ~1% faster."""
-    return -(-(w.S // w.R) // 64) < 24
-
-
 def make_step(st, args, w, dev):
     kind = step_kind(w)
     if kind == "image":
@@ -768,8 +758,7 @@ def make_step(st, args, w, dev):
         return VMajorStep(st, w, dev, frac=args.vmajor_f)
     stp = Step(st, w, dev)
     stp.fused_merge = args.merge == "fused"
-    ring = args.attn == "ring" or (args.attn == "auto" and ring_pays(w))
-    stp.ring = ring and args.merge == "fused" and args.schedule == "serial"
+    stp.ring = args.attn == "ring" and args.merge == "fused" and args.schedule == "serial"
     stp.sender_vmajor = args.vmajor == "sender"
     if args.rope:
         stp.rope_table = st.st_rope_table(w.S, w.D, 10000.0, device=dev)
@@ -1092,11 +1081,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="image_4096px", choices=sorted(synth.BY_NAME))
-    ap.add_argument("--attn", choices=["auto", "ring", "chunks"], default="auto",
+    ap.add_argument("--attn", choices=["ring", "chunks"], default="ring",
                     help="ring = one launch over every KV chunk (each query block from its own chunk); "
                          "chunks = one launch per chunk, later chunks merged inside the attention kernel "
-                         "(--merge separate: attn_chunk_merge); auto = the faster of the two as measured: "
-                         "ring for the image step and for ST-DiT chunks under 24 key steps, else chunks")
+                         "(--merge separate: attn_chunk_merge)")
     ap.add_argument("--vmajor-f", type=float, default=0.5, choices=[0.1, 0.5, 0.9],
                     help="V-Major step: target active fraction of the golden threshold")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
