@@ -75,10 +75,15 @@ constexpr int W_PV0 = 15;                    // PV issuer of tile A (tile B: W_P
 constexpr int W_ONES = 17;                   // writes the ones column into V tiles (padded head dims); 18-19 idle
 // Registers per thread after the split (setmaxnreg): the launch gives every
 // thread 96 (640 x 96 = 61440); the two softmax warpgroups and the epilogue
-// take 128, and the issuer / loader warpgroups give back down to 48:
-// 256 x 128 + 128 x 128 + 256 x 48 = 61440.
-constexpr int REG_SOFTMAX = 128, REG_EPI = 128, REG_ISSUE = 48;
-static_assert(256 * REG_SOFTMAX + 128 * REG_EPI + 256 * REG_ISSUE <= NUM_THREADS * 96, "register split");
+// take more, and the issuer / loader warpgroups give back:
+// 256 x 128 + 128 x 128 + 256 x 48 = 61440 in general, and
+// 256 x 152 + 128 x 96 + 256 x 40 = 61440 for head dims up to 80 without the
+// merge, whose epilogue holds at most 80 columns of O (measured 2% faster at
+// S = 1200 and 8160, D = 72; 1-2% slower at D = 128).
+template <bool WIDE> struct RegSplit {
+  static constexpr int SOFTMAX = WIDE ? 152 : 128, EPI = WIDE ? 96 : 128, ISSUE = WIDE ? 40 : 48;
+  static_assert(256 * SOFTMAX + 128 * EPI + 256 * ISSUE <= NUM_THREADS * 96, "register split");
+};
 constexpr int EPI_COLS = 16;                 // O columns per staged store
 constexpr int EPI_BUF = 32 * EPI_COLS * 4;   // bytes of one staging buffer (32 rows, fp32)
 // TMEM columns: per tile two S buffers of BLOCK_N fp32 columns, then O.
@@ -139,6 +144,7 @@ template <int D, bool MERGE = false, bool QTMEM = false> struct Cfg {
   static constexpr int QB = (4 * QTILE + 4 * (KTILE + VTILE) <= BUDGET) ? 2 : 1;   // Q double buffer if 4 stages fit
   static constexpr int NS_RAW = (BUDGET - 2 * QB * QTILE) / (KTILE + VTILE);
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;   // K/V ring depth
+  using Regs = RegSplit<D <= 80 && !MERGE>;            // the setmaxnreg split of this instantiation
   static constexpr int SMEM = 1024 + 2 * QB * QTILE + NS * (KTILE + VTILE) + ACCS + EPI + 1024;   // + barriers
   static_assert(SMEM <= 232448, "shared memory");
   static_assert(DP <= 128 && DPV <= 128, "head dim too large");
@@ -558,7 +564,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp >= W_LOAD) {
     // warpgroups 3 and 4: TMA producer, MMA issuers, idle warps
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_ISSUE));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(K::Regs::ISSUE));
     if (warp == W_LOAD) {
       if (lane == 0 && n_kv > 0) {
         // ================= TMA producer =================
@@ -763,7 +769,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp < 8) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(K::Regs::SOFTMAX));
     // ================= softmax warpgroups =================
     const int X = warp >> 2;                   // tile
     const int r = ((warp & 3) << 5) + lane;    // row in tile == TMEM lane
@@ -886,7 +892,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ++oc;
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_EPI));
+    // the epilogue keeps the launch's 96 registers in the wide split
+    if constexpr (K::Regs::EPI > 96) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(K::Regs::EPI));
     // ================= epilogue warpgroup =================
     // Per tile: wait for the last PV and the row statistics, read O out of
     // TMEM into registers (TMEM is released right after), divide by the row
@@ -1345,7 +1352,7 @@ st_status launch_spatial(const st::Geom &g, int lo, int hi, int kv0, int kv1, fl
   if (regs_ok < 0) {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ST_ERR_CUDA;
-    regs_ok = fa.numRegs * NUM_THREADS >= 256 * REG_SOFTMAX + 128 * REG_EPI + 256 * REG_ISSUE ? 1 : 0;
+    regs_ok = fa.numRegs * NUM_THREADS >= 256 * K::Regs::SOFTMAX + 128 * K::Regs::EPI + 256 * K::Regs::ISSUE ? 1 : 0;
   }
   if (!regs_ok) return ST_ERR_UNSUPPORTED;
   return st::launch_pdl(kern, ctas, NUM_THREADS, K::SMEM, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], p);
