@@ -28,7 +28,8 @@
 
 namespace {
 
-constexpr int G = 4;  // heads per CTA, one warp each
+// G: heads per work item and CTA, one warp each (4, or 8 for sequences of at
+// most 16 frames, whose items are small)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -75,8 +76,8 @@ __device__ __forceinline__ void mma1688(float *c, uint32_t a0, uint32_t a1, uint
       : "r"(a0), "r"(a1), "r"(b0));
 }
 
-template <int D, int TP, int STAGES>
-__global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_sel, int n_hg, int n_items,
+template <int D, int TP, int STAGES, int G>
+__global__ void __launch_bounds__(32 * G) temporal_bf16(st::Geom g, int lo, int n_sel, int n_hg, int n_items,
                                                      float scale_log2, float scale,
                                                      const uint16_t *__restrict__ q,
                                                      const uint16_t *__restrict__ k,
@@ -292,22 +293,27 @@ __global__ void __launch_bounds__(128) temporal_bf16(st::Geom g, int lo, int n_s
 template <int D, int TP>
 st_status launch_t(const st::Geom &g, int lo, int n_sel, float scale, const void *q, const void *k,
                    const void *v, void *o, float *lse, int o_f32, cudaStream_t s) {
+  // items of 8 heads when the sequence is short (per item the CTA pays three
+  // barriers and one pipeline turn; 8 heads of 16 frames move as many bytes as
+  // 4 heads of 32), else 4
+  constexpr int G = TP <= 16 && D <= 80 ? 8 : 4;
   const int n_hg = (g.H + G - 1) / G;
   const long long items = (long long)g.B * n_sel * n_hg;
   if (items > 0x7fffffffLL) return ST_ERR_SHAPE;
   constexpr size_t stage_bytes = size_t(3) * TP * (G * D + 8) * sizeof(uint16_t);
-  constexpr int STAGES = 2 * stage_bytes <= 64 * 1024 ? 2 : 1;
+  // two stages when they fit in 16 KB per warp (the next item's rows load while this one computes)
+  constexpr int STAGES = 2 * stage_bytes <= size_t(G) * 16 * 1024 ? 2 : 1;
   const size_t smem = STAGES * stage_bytes + size_t(g.T) * sizeof(long long);
-  auto kern = temporal_bf16<D, TP, STAGES>;
+  auto kern = temporal_bf16<D, TP, STAGES, G>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return ST_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, smem) != cudaSuccess || per_sm < 1)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * G, smem) != cudaSuccess || per_sm < 1)
     per_sm = 1;
   const long long cap = (long long)st::num_sms() * per_sm;
   const int grid = int(items < cap ? items : cap);
   const float log2e = 1.4426950408889634f;
-  return st::launch_pdl(kern, grid, 128, smem, s, g, lo, n_sel, n_hg, int(items), scale * log2e, scale,
+  return st::launch_pdl(kern, grid, 32 * G, smem, s, g, lo, n_sel, n_hg, int(items), scale * log2e, scale,
                         static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k),
                         static_cast<const uint16_t *>(v), o, lse, o_f32);
 }

@@ -315,7 +315,7 @@ def test_temporal_video_sampled_and_slices(st):
 
 
 @pytest.mark.parametrize("T,D,H", [(1, 72, 4), (7, 64, 6), (16, 32, 8), (33, 128, 3), (64, 80, 4), (24, 96, 5),
-                                   (48, 72, 2)])
+                                   (48, 72, 2), (12, 72, 11), (16, 80, 9), (16, 128, 5)])
 def test_temporal_shapes(st, T, D, H):
     w = synth.Workload("t", 9, B=2, T=T, S=37, H=H, D=D, dtype="bf16")
     q, k, v = synth.qkv(w)
