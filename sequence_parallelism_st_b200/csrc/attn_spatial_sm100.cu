@@ -237,6 +237,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
   }
 }
 
+// Non-blocking test of the phase.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// The waits on the MMA chain (the issuers' operands and buffers, the
+// softmax's S) poll the barrier N times before the sleeping wait: a thread
+// woken from a suspended wait resumes later than one that polls, and on
+// this chain every cycle of that delay is paid by the tensor pipe (measured:
+// 5% of the image-DiT ring launch, 8% of the cached-K/V launch, 3-4% at
+// head dim 72).  Bounded: after N polls it is mbar_wait.
+constexpr int SPIN_ISSUE = 32, SPIN_SOFTMAX = 8;
+template <int N>
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, uint32_t epoch, int site) {
+  for (int i = 0; i < N; ++i)
+    if (mbar_test(bar, parity)) return true;
+  return mbar_wait(bar, parity, epoch, site);
+}
+
 __device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
                                             int c2, int c3, int c4) {
   asm volatile(
@@ -657,8 +683,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int st = g0 % NS;
           const uint32_t b = step & 1;
           // S(step) overwrites P(step - 2) in the same buffer: PV(step - 2) must be done
-          if (step >= 2 && !(ok = mbar_wait(pv_done + 2 * X + b, ((step - 2) >> 1) & 1, epoch, 5))) break;
-          if (!(ok = mbar_wait(k_full + st, (g0 / NS) & 1, epoch, 4))) break;
+          if (step >= 2 && !(ok = mbar_wait_spin<SPIN_ISSUE>(pv_done + 2 * X + b, ((step - 2) >> 1) & 1, epoch, 5))) break;
+          if (!(ok = mbar_wait_spin<SPIN_ISSUE>(k_full + st, (g0 / NS) & 1, epoch, 4))) break;
           tc_fence_after();
           const uint32_t d = tmem + X * 2 * BLOCK_N + b * BLOCK_N;
           const uint32_t ka = aK + st * K::KTILE;
@@ -718,8 +744,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t g0 = kv + j;
           const int st = g0 % NS;
           const uint32_t b = step & 1;
-          if (!(ok = mbar_wait((K::ONES ? v_ready : v_full) + st, (g0 / NS) & 1, epoch, 6))) break;
-          if (!(ok = mbar_wait(p_full + 2 * X + b, (step >> 1) & 1, epoch, 7 + X))) break;
+          if (!(ok = mbar_wait_spin<SPIN_ISSUE>((K::ONES ? v_ready : v_full) + st, (g0 / NS) & 1, epoch, 6))) break;
+          if (!(ok = mbar_wait_spin<SPIN_ISSUE>(p_full + 2 * X + b, (step >> 1) & 1, epoch, 7 + X))) break;
           // O of the tile's previous item read out by the epilogue
           if (j == 0 && !(ok = mbar_wait(o_empty + X, (oc & 1) ^ 1u, epoch, 9 + X))) break;
           tc_fence_after();
@@ -793,7 +819,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int j = 0; j < n_kv; ++j, ++gs) {
         const uint32_t b = gs & 1;
-        if (!(ok = mbar_wait(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
+        if (!(ok = mbar_wait_spin<SPIN_SOFTMAX>(s_full + 2 * X + b, (gs >> 1) & 1, epoch, 11 + X))) break;
         tc_fence_after();
         uint32_t sr[BLOCK_N];
 #pragma unroll
