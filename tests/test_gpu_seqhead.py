@@ -4,7 +4,6 @@ handle: rows of 8, 16 and 32 sixteen-byte vectors (the row-walking kernel),
 other widths (the segment kernel), B = 1 and B > 1 (shards stacked outermost,
 batches inside), with and without the fused per-head RMSNorm, and the round
 trip."""
-import numpy as np
 import pytest
 import torch
 
