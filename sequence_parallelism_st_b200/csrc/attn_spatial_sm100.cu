@@ -15,13 +15,20 @@
 //   * Tensor-core work runs on four issuer warps, one per (tile, product):
 //     S = Q K^T into TMEM (fp32) for tile A (warp 13) and tile B (warp 14),
 //     O += P V (warps 15 and 16) with P read straight from TMEM (the "TS"
-//     form).  A single thread issues about one tcgen05 operation (MMA or
-//     commit) per hundred cycles, so the streams are split over four warps to
-//     keep the tensor pipe fed.  Registers are rebalanced per warpgroup with
-//     setmaxnreg: the single-thread roles give theirs to the softmax.  S is
-//     double-buffered per tile, so S of step j+1 is ready before the softmax
-//     of step j ends; S(j+2) reuses the buffer of S(j) once PV(j) has read
-//     P(j) from it.
+//     form).  The four streams enter the tensor pipe independently, so no
+//     stream waits behind another's MMAs that are held up by the shared-
+//     memory reads they all share.  Registers are rebalanced per warpgroup
+//     with setmaxnreg: the single-thread roles give theirs to the softmax.  S
+//     is double-buffered per tile, so S of step j+1 is ready before the
+//     softmax of step j ends; S(j+2) reuses the buffer of S(j) once PV(j) has
+//     read P(j) from it.  The waits along this chain poll their barrier a few
+//     times before sleeping (mbar_wait_spin).
+//   * Ring mode (st_attn_ring): an item walks the R KV chunks from the one
+//     holding its first row, carrying its running statistics across them;
+//     the chunk edges come from host tables, and when every chunk is a whole
+//     number of 64-key steps the walk is a plain rotation (RING = 2).
+//   * Head dims 72/80 with long items keep Q in TMEM beside O (QTMEM), so S
+//     becomes a TS product that reads only K from shared memory.
 //   * Warps 0-3 (tile A) and 4-7 (tile B) are the softmax warpgroups: one
 //     thread per query row (TMEM lane), 64 scores per step loaded with
 //     tcgen05.ld, row max, exp2 with the softmax scale folded in (part of the
