@@ -79,3 +79,29 @@ def test_oracle_arm_samples_fit_the_workload(name):
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["single_thread"]["value"] > 0
     line = bench.run_reference(argparse.Namespace(cpu_budget=0.2, steps=1, warmup=3), w)
     assert line["impl"] == "reference" and line["value"] > 0
+
+
+def test_step_kind_per_workload():
+    """Each workload takes the step its layout calls for: the image-DiT block
+    (T = 1 with the Q/K RMSNorm), the V-Major step (T = 1 with change
+    fractions) or the ST-DiT block."""
+    import synth
+    kinds = {w.name: bench.step_kind(w) for w in synth.WORKLOADS}
+    assert kinds == {"tiny": "st", "opensora_low": "st", "video_1080p": "st", "image_4096px": "image",
+                     "vmajor_2304px": "vmajor"}
+
+
+@pytest.mark.parametrize("workload,launch", [("image_4096px", "ring"), ("opensora_low", "ring"),
+                                             ("video_1080p", "ring"), ("vmajor_2304px", "cached_kv")])
+def test_traffic_record_matches_the_attention_source(workload, launch):
+    """The committed DRAM counters of each workload's roofline launch belong to
+    the attention source as it stands (the bench reports them as
+    roofline.traffic only then), and lie between what the launch must read (Q,
+    K and V once; part of O may still be in L2 when the launch ends) and its
+    algorithmic bytes plus the K/V re-reads of the ring walk."""
+    import synth
+    got = bench.kernel_traffic(workload, launch)
+    assert got is not None, "profiles/traffic.json was captured on another attention source"
+    w = synth.BY_NAME[workload]
+    t = w.B * w.T * w.S * w.C * w.elem_bytes
+    assert 0.98 * 3 * t <= got <= 1.6 * 4 * t
