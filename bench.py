@@ -1065,7 +1065,10 @@ def run_reference(args, w):
     else:
         sample = (f"fp64 numpy oracle per step: attention rows of {units} of {w.S} query tokens (all {w.H} heads, "
                   f"all {w.S} keys)")
-    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": 1,
+    # n_gpus: the launch's N, so the line pairs with ours at the same N (the
+    # oracle itself runs on rank 0's host cores, as cpu_baseline says)
+    n_launch = int(os.environ.get("WORLD_SIZE", 1))
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": n_launch,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "H": w.H, "D": w.D},
